@@ -1,0 +1,162 @@
+"""fp64 CPU oracle for Kimi Delta Attention (KDA).
+
+TEST INFRASTRUCTURE ONLY.  Only `tests/`, the smoke check in `__graft_entry__.py`
+and the CPU-baseline leg of `bench.py` may import this package.  The CUDA library
+never calls it and has no fallback to it; the two share no code.
+
+* `prefill` / `decode`: the token-by-token fp64 recurrence of kda_oracle.c
+  ("SemiAnalysis Kimi K3", KDA section: the delta rule with a diagonal forget gate).
+* `oracle.chunked`: an independent fp64 restatement of the chunkwise form
+  (FlashKDA section), used only to pin the chunk algebra against the recurrence.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "_kda_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile kda_oracle.c with gcc (no fast-math: IEEE fp64 as written)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        lib.kda_oracle_prefill.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, P,
+                                           ctypes.c_int]
+        lib.kda_oracle_prefill.restype = ctypes.c_int
+        lib.kda_oracle_decode.argtypes = [P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, P]
+        lib.kda_oracle_decode.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f32(x) -> np.ndarray:
+    """Exact upcast of bf16/fp16/fp32 inputs to a contiguous fp32 numpy array."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().to("cpu", torch.float32).numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _f64(x) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().to("cpu", torch.float64).numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def prefill(q, k, v, g, beta, cu_seqlens, s0=None, heads: Optional[Sequence[int]] = None,
+            nthreads: Optional[int] = None):
+    """fp64 KDA prefill over packed sequences.
+
+    q, k, g [T, H, dk]; v [T, H, dv]; beta [T, H]; cu_seqlens [N+1]; s0 [N, Hs, dk, dv]
+    or None; heads: subset of heads to compute (Hs = len(heads)), default all.
+    Returns (out [T, Hs, dv] fp64, s_final [N, Hs, dk, dv] fp64).
+    """
+    lib = _load()
+    q, k, v, g, beta = _f32(q), _f32(k), _f32(v), _f32(g), _f32(beta)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    N = cu.shape[0] - 1
+    hs = None if heads is None else np.ascontiguousarray(np.asarray(heads, dtype=np.int32))
+    Hs = H if hs is None else hs.shape[0]
+    s0a = None if s0 is None else _f64(s0)
+    if s0a is not None:
+        assert s0a.shape == (N, Hs, dk, dv), s0a.shape
+    out = np.zeros((T, Hs, dv), dtype=np.float64)
+    sf = np.zeros((N, Hs, dk, dv), dtype=np.float64)
+    rc = lib.kda_oracle_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0a),
+                                _ptr(cu), N, H, dk, dv, _ptr(hs), Hs, _ptr(out), _ptr(sf),
+                                nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("kda_oracle_prefill failed with code %d" % rc)
+    return out, sf
+
+
+def decode(q, k, v, g, beta, state):
+    """One fp64 KDA decode step.  q, k, g [N, H, dk]; v [N, H, dv]; beta [N, H];
+    state [N, H, dk, dv].  Returns (out [N, H, dv], new_state) as fp64 arrays."""
+    lib = _load()
+    q, k, v, g, beta = _f32(q), _f32(k), _f32(v), _f32(g), _f32(beta)
+    S = _f64(state).copy()
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    out = np.zeros((N, H, dv), dtype=np.float64)
+    rc = lib.kda_oracle_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                               N, H, dk, dv, _ptr(out))
+    if rc != 0:
+        raise RuntimeError("kda_oracle_decode failed with code %d" % rc)
+    return out, S
+
+
+def rel_frobenius(x, ref) -> float:
+    """||x - ref||_F / ||ref||_F (absolute error when ||ref|| < 1e-30)."""
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    num = float(np.linalg.norm((x - ref).ravel()))
+    den = float(np.linalg.norm(ref.ravel()))
+    return num / den if den >= 1e-30 else num
+
+
+def max_rel_frobenius_per_slice(out, ref, cu_seqlens) -> float:
+    """Max over (sequence, head) of the relative Frobenius error of the output slice
+    [len_n, dv] (outputs [T, H, dv])."""
+    cu = [int(x) for x in np.asarray(cu_seqlens)]
+    out = np.asarray(out, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    worst = 0.0
+    for n in range(len(cu) - 1):
+        if cu[n + 1] == cu[n]:
+            continue
+        for h in range(ref.shape[1]):
+            worst = max(worst, rel_frobenius(out[cu[n]:cu[n + 1], h], ref[cu[n]:cu[n + 1], h]))
+    return worst
+
+
+def max_rel_frobenius_states(S, ref) -> float:
+    """Max over (sequence, head) of the relative Frobenius error of [dk, dv] states."""
+    S = np.asarray(S, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    worst = 0.0
+    for n in range(ref.shape[0]):
+        for h in range(ref.shape[1]):
+            worst = max(worst, rel_frobenius(S[n, h], ref[n, h]))
+    return worst
