@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""KDA benchmark: prefill tokens/s (H=32, D=128) + decode state GB/s, as % of roofline.
+
+One JSON line on rank 0.  The timed "step" is one call of the whole prefill path
+(kda_prefill: chunking, cumulative decay, decayed operands, L / Aqk, UT transform,
+pseudo-values, chunk recurrence, final state) on the single-sequence workload
+B=1, H=32, T=8192, D=128, C=64, bf16 inputs, inputs resident in HBM.  The decode step
+(N=256 x H=32, D=128, 64 consecutive in-place steps) is timed in the same run and
+reported under "decode".  Multi-GPU runs are independent replicas (every rank owns its
+own problem; there is no exchange on the path), so scaling is weak and the job value
+is the sum of tokens over ranks divided by the slowest rank's time.
+
+--impl reference runs the fp64 CPU oracle instead (bounded samples of the same
+workload on the host cores); under torchrun only rank 0 does, the others exit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s (H=32,D=128) + decode state GB/s, as % of B200 roofline"
+PREFILL_CFG = 1
+DECODE_CFG = 3
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- host logic
+def rank_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each replica draws its own independent problem of the same shape."""
+    return base_seed + 104_729 * rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def prefill_page_counts(lengths, H, D, C):
+    """The pages' per-chunk-head counts (FlashKDA section): 12C^3 + 8C^2 D + 6 C D^2 FLOPs
+    and 8C^2 + 22 C D bytes per chunk per head, plus 8 D^2 bytes of state per head.
+    A partial chunk counts as a whole chunk."""
+    chunks = sum((n + C - 1) // C for n in lengths)
+    ch = chunks * H
+    flops = ch * (12 * C ** 3 + 8 * C * C * D + 6 * C * D * D)
+    bytes_ = ch * (8 * C * C + 22 * C * D) + 8 * D * D * len(lengths) * H
+    return flops, bytes_
+
+
+def prefill_strict_bytes(lengths, H, D, in_bytes, has_s0, has_final):
+    """Bytes the method itself must move: q, k, v, out in the input dtype, g fp32 (dk per
+    token-head), beta fp32, and the fp32 states read/written."""
+    T = sum(lengths)
+    per_tok_head = 4 * D * in_bytes + 4 * D + 4
+    states = 4 * D * D * len(lengths) * H * ((1 if has_s0 else 0) + (1 if has_final else 0))
+    return T * H * per_tok_head + states
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a background thread."""
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device, period_s: float = 0.002):
+        self.period = period_s
+        self.samples, self.max_mhz, self.ok = [], None, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            p = torch.cuda.get_device_properties(device)
+            bus = "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML unavailable: report no clocks
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        reasons = [n for b, n in self.REASONS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample_tokens_per_s(inp, target_s: float):
+    """Time the fp64 oracle on the first Ts tokens (all heads) of the prefill workload,
+    Ts sized for about `target_s` seconds.  Returns (tokens/s, Ts, seconds, threads)."""
+    import oracle
+    T = inp["q"].shape[0]
+    H = inp["q"].shape[1]
+    threads = min(oracle.default_threads(), H)
+
+    def run(ts):
+        t0 = time.perf_counter()
+        oracle.prefill(inp["q"][:ts], inp["k"][:ts], inp["v"][:ts], inp["g"][:ts],
+                       inp["beta"][:ts], [0, ts], nthreads=threads)
+        return time.perf_counter() - t0
+
+    ts = 32
+    dt = run(ts)
+    ts = int(max(32, min(T, ts * target_s / max(dt, 1e-6))))
+    dt = run(ts)
+    return ts / dt, ts, dt, threads
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def bench_gpu(args):
+    import torch
+    from linear_attention_rule_b200 import kda, synthetic
+
+    rank, local_rank, world = rank_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    peaks = load_peaks()
+
+    # ---- prefill workload (resident inputs) --------------------------------------------
+    cfg = synthetic.CONFIGS[PREFILL_CFG]
+    lengths = synthetic.draw_lengths(cfg)
+    D, H, C = cfg.D, cfg.H, cfg.C
+    inp = synthetic.make_prefill_inputs(lengths, H, D, D, cfg.dtype, cfg.g_mean, cfg.s0_std,
+                                        rank_seed(cfg.seed, rank))
+    T = inp["q"].shape[0]
+    N = len(lengths)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    out = torch.empty(T, H, D, dtype=cfg.dtype, device=dev)
+    fin = torch.empty(N, H, D, D, dtype=torch.float32, device=dev)
+    ws_bytes = kda.kda_prefill_workspace_size(T, N, H, D, D, C, cfg.dtype)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes_total = sum(d[k].numel() * d[k].element_size() for k in ("q", "k", "v", "g", "beta"))
+
+    def prefill_step():
+        kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out,
+                        initial_state=d["s0"], final_state=fin, C=C, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        prefill_step()
+    torch.cuda.synchronize(dev)
+    assert kda.kda_get_device_status(stream) == kda.KDA_OK
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            prefill_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms_local, world, dev)
+    value = world * T / (ms * 1e-3)
+    launches_per_prefill = kda.prefill_launches(cfg.dtype)
+
+    flops, page_bytes = prefill_page_counts(lengths, H, D, C)
+    strict = prefill_strict_bytes(lengths, H, D, 2 if cfg.dtype == torch.bfloat16 else 4,
+                                  inp["s0"] is not None, True)
+    t_s = ms_local * 1e-3
+    achieved_gbs = page_bytes / t_s / 1e9
+    roofline = {
+        "bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
+        "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
+        "traffic": None, "kernel": "kda_prefill (whole path)",
+        "bytes_per_launch": page_bytes, "counts": "page counts 8C^2+22CD B per chunk-head + 8D^2 per head",
+        "peak_source": peaks["source"],
+        "tensor_frac": round(flops / t_s / 1e12 / peaks["bf16_tflops"], 4),
+        "strict_frac": round(strict / t_s / 1e9 / peaks["hbm_gbs"], 4),
+    }
+    clocks = clk.summary()
+
+    # ---- decode workload ---------------------------------------------------------------
+    dcfg = synthetic.CONFIGS[DECODE_CFG]
+    Nd, Hd, Dd = dcfg.N, dcfg.H, dcfg.D
+    S = synthetic.make_decode_state(Nd, Hd, Dd, Dd, dcfg.s0_std, rank_seed(dcfg.seed, rank)).to(dev)
+    steps_in = []
+    for s in range(dcfg.steps):
+        x = synthetic.make_decode_step_inputs(Nd, Hd, Dd, Dd, dcfg.dtype, dcfg.g_mean,
+                                              rank_seed(dcfg.seed, rank), s)
+        steps_in.append({k: v.to(dev) for k, v in x.items()})
+    dout = torch.empty(Nd, Hd, Dd, dtype=dcfg.dtype, device=dev)
+
+    def decode_step():
+        for x in steps_in:
+            kda.kda_decode(x["q"], x["k"], x["v"], x["g"], x["beta"], S, dout, stream=stream)
+
+    for _ in range(args.warmup):
+        decode_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    with ClockSampler(dev) as dclk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            decode_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    dms_local = e0.elapsed_time(e1) / args.steps
+    dms = max_over_ranks(dms_local, world, dev)
+    state_bytes = 8 * Dd * Dd * Nd * Hd * dcfg.steps
+    d_gbs = world * state_bytes / (dms * 1e-3) / 1e9
+    d_gbs_local = state_bytes / (dms_local * 1e-3) / 1e9
+    decode = {
+        "workload": dcfg.name, "value": round(d_gbs, 1), "unit": "GB/s (fp32 state read+write)",
+        "ms_per_step": round(dms, 4), "steps_per_call": dcfg.steps,
+        "seq_tokens_per_s": round(world * Nd * dcfg.steps / (dms * 1e-3), 1),
+        "roofline": {"bound": "hbm", "achieved": round(d_gbs_local, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(d_gbs_local / peaks["hbm_gbs"], 4),
+                     "traffic": None, "kernel": "kda::decode_kernel",
+                     "bytes_per_launch": 8 * Dd * Dd * Nd * Hd,
+                     "counts": "page count 8 D^2 bytes per head-token",
+                     "peak_source": peaks["source"]},
+        "clocks": dclk.summary(), "gpu_launches": dcfg.steps * args.steps,
+    }
+    del steps_in, S
+
+    # ---- end to end from pinned host buffers -------------------------------------------
+    e2e = None
+    if not args.no_e2e:
+        h = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+        hout = torch.empty(T, H, D, dtype=cfg.dtype).pin_memory()
+        hfin = torch.empty(N, H, D, D, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            for k in ("q", "k", "v", "g", "beta", "cu_seqlens"):
+                d[k].copy_(h[k], non_blocking=True)
+            prefill_step()
+            hout.copy_(out, non_blocking=True)
+            hfin.copy_(fin, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+        h2d = sum(h[k].numel() * h[k].element_size() for k in ("q", "k", "v", "g", "beta", "cu_seqlens"))
+        d2h = hout.numel() * hout.element_size() + hfin.numel() * hfin.element_size()
+        e2e = {"value": round(world * T / (ems * 1e-3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ems, 4)}
+
+    # ---- CPU oracle baseline (rank 0, one GPU only) ------------------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, ts, secs, threads = oracle_sample_tokens_per_s(inp, args.cpu_seconds)
+        cpu = {"value": round(tps, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": "first %d tokens x all %d heads of the same workload, fp64, %.1f s" % (ts, H, secs)}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": kda.prefill_compute_dtype(cfg.dtype),
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "T": T, "H": H, "D": D, "C": C,
+                   "l2": "inputs larger than L2 (%.0f MB resident per step)" % (in_bytes_total / 1e6),
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": roofline, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
+        "clocks": clocks, "gpu_launches": launches_per_prefill * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+def bench_reference(args):
+    rank, _, world = rank_env()
+    if rank != 0:
+        return
+    import oracle
+    from linear_attention_rule_b200 import synthetic
+    cfg = synthetic.CONFIGS[PREFILL_CFG]
+    lengths = synthetic.draw_lengths(cfg)
+    inp = synthetic.make_prefill_inputs(lengths, cfg.H, cfg.D, cfg.D, cfg.dtype, cfg.g_mean,
+                                        cfg.s0_std, cfg.seed)
+    H = cfg.H
+    threads = min(oracle.default_threads(), H)
+    # size one step for about args.cpu_seconds / 2 of fp64 work
+    _, ts, _, _ = oracle_sample_tokens_per_s(inp, max(1.0, args.cpu_seconds / 2))
+
+    def step():
+        oracle.prefill(inp["q"][:ts], inp["k"][:ts], inp["v"][:ts], inp["g"][:ts],
+                       inp["beta"][:ts], [0, ts], nthreads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    secs = (time.perf_counter() - t0) / args.steps
+    value = ts / secs
+    sample = "first %d tokens x all %d heads of %s per step, fp64 oracle" % (ts, H, cfg.name)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": sum(lengths), "H": H, "D": cfg.D, "C": cfg.C},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    _, _, world = rank_env()
+    if world != args.gpus:
+        print("note: --gpus %d but WORLD_SIZE %d; using WORLD_SIZE" % (args.gpus, world),
+              file=sys.stderr)
+    if args.impl == "reference":
+        bench_reference(args)
+    else:
+        bench_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

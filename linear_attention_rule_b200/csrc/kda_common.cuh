@@ -1,0 +1,38 @@
+// Shared device helpers for the libkda kernels (one translation unit: libkda.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "libkda.h"
+
+// First error a kernel detected since the host last read it (kda_get_device_status).
+__device__ int g_kda_status;
+
+__device__ __forceinline__ void kda_set_status(int s) { atomicCAS(&g_kda_status, 0, s); }
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Checks the part of cu_seqlens that sequence n depends on; records KDA_ERR_BAD_SEQLENS
+// and returns false when it is inconsistent.
+__device__ __forceinline__ bool kda_seq_bounds(const int32_t* cu, int n, int num_seqs,
+                                               int64_t total, int64_t& t_begin, int64_t& t_end) {
+    t_begin = cu[n];
+    t_end = cu[n + 1];
+    bool ok = t_begin >= 0 && t_end >= t_begin && t_end <= total;
+    if (n == 0) ok = ok && t_begin == 0;
+    if (n == num_seqs - 1) ok = ok && t_end == total;
+    if (!ok) kda_set_status(KDA_ERR_BAD_SEQLENS);
+    return ok;
+}

@@ -1,0 +1,133 @@
+// libkda C-ABI: argument checking, workspace sizing and dispatch to the kernels.
+// Everything here is host code; the kernels live in the included .cuh files so the
+// whole library is one translation unit (one device status word, no relocatable code).
+#include <stdint.h>
+#include <string.h>
+
+#include "libkda.h"
+#include "kda_common.cuh"
+#include "kda_decode.cuh"
+#include "kda_prefill_simt.cuh"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_dim(int32_t dk, int32_t dv) { return dk == dv && (dk == 64 || dk == 128); }
+
+bool valid_chunk(kda_dtype dt, int32_t C) {
+    if (dt == KDA_BF16) return C == 64;
+    return C == 16 || C == 32 || C == 64;
+}
+
+template <typename T>
+cudaError_t dispatch_simt(int32_t dk, int32_t C, const void* q, const void* k, const void* v,
+                          const float* g, const float* beta, const float* s0, const int32_t* cu,
+                          int num_seqs, int64_t total, int H, void* out, float* sf,
+                          cudaStream_t st) {
+#define KDA_SIMT_CASE(D, CC)                                                                  \
+    if (dk == D && C == CC)                                                                   \
+        return kda::launch_prefill_simt<T, D, CC>(q, k, v, g, beta, s0, cu, num_seqs, total, H, \
+                                                  out, sf, st);
+    KDA_SIMT_CASE(64, 16) KDA_SIMT_CASE(64, 32) KDA_SIMT_CASE(64, 64)
+    KDA_SIMT_CASE(128, 16) KDA_SIMT_CASE(128, 32) KDA_SIMT_CASE(128, 64)
+#undef KDA_SIMT_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t kda_abi_version(void) { return 1; }
+
+const char* kda_status_string(kda_status s) {
+    switch (s) {
+        case KDA_OK: return "ok";
+        case KDA_ERR_INVALID_ARG: return "invalid argument";
+        case KDA_ERR_UNSUPPORTED: return "unsupported problem size or chunk size";
+        case KDA_ERR_CUDA: return "CUDA runtime error";
+        case KDA_ERR_TIMEOUT: return "a bounded device wait expired";
+        case KDA_ERR_BAD_SEQLENS: return "cu_seqlens inconsistent with total_tokens";
+    }
+    return "unknown status";
+}
+
+size_t kda_prefill_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
+                                  int32_t dv, int32_t C, kda_dtype dt) {
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0 || !supported_dim(dk, dv) ||
+        !valid_chunk(dt, C))
+        return 0;
+    return 0;
+}
+
+kda_status kda_prefill(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                       int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                       kda_dtype dt, void* out, float* final_state, int32_t C, void* workspace,
+                       size_t ws_bytes, kda_stream_t stream) {
+    if (num_seqs < 0 || total_tokens < 0 || H <= 0 || dk <= 0 || dv <= 0)
+        return KDA_ERR_INVALID_ARG;
+    if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (total_tokens > INT32_MAX) return KDA_ERR_UNSUPPORTED;  // cu_seqlens is int32
+    if (!supported_dim(dk, dv) || !valid_chunk(dt, C)) return KDA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return KDA_OK;
+    if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, beta, out, initial_state, final_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return KDA_ERR_INVALID_ARG;
+    const size_t need = kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, dt);
+    if (ws_bytes < need || (need > 0 && (!workspace ||
+                                         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)))
+        return KDA_ERR_INVALID_ARG;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    if (dt == KDA_F32)
+        err = dispatch_simt<float>(dk, C, q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
+                                   total_tokens, H, out, final_state, st);
+    else
+        err = dispatch_simt<__nv_bfloat16>(dk, C, q, k, v, g, beta, initial_state, cu_seqlens,
+                                           num_seqs, total_tokens, H, out, final_state, st);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, float* state_inout, void* out, int32_t N, int32_t H,
+                      int32_t dk, int32_t dv, kda_dtype dt, kda_stream_t stream) {
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return KDA_OK;
+    if ((int64_t)N * H > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !g || !beta || !state_inout || !out) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, beta, state_inout, out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    if (dt == KDA_F32)
+        err = dk == 64 ? kda::launch_decode<64, float>(q, k, v, g, beta, state_inout, out, N, H, st)
+                       : kda::launch_decode<128, float>(q, k, v, g, beta, state_inout, out, N, H, st);
+    else
+        err = dk == 64
+                  ? kda::launch_decode<64, __nv_bfloat16>(q, k, v, g, beta, state_inout, out, N, H, st)
+                  : kda::launch_decode<128, __nv_bfloat16>(q, k, v, g, beta, state_inout, out, N, H, st);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_get_device_status(kda_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KDA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_kda_status, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_kda_status, &zero, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return static_cast<kda_status>(v);
+}
+
+}  // extern "C"

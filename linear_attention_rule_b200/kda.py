@@ -1,0 +1,155 @@
+"""Thin Python binding of libkda (ctypes).  Argument marshalling only.
+
+Every function has the name of the C entry point it calls (include/libkda.h) and
+passes torch tensors' device pointers, sizes and the current CUDA stream straight
+through; all of the computation runs in the library's kernels.  There is no
+fallback: if libkda.so is missing or a call fails, a RuntimeError is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_OK = 0
+KDA_ERR_INVALID_ARG = 1
+KDA_ERR_UNSUPPORTED = 2
+KDA_ERR_CUDA = 3
+KDA_ERR_TIMEOUT = 4
+KDA_ERR_BAD_SEQLENS = 5
+KDA_F32 = 0
+KDA_BF16 = 1
+
+# Every symbol include/libkda.h declares (checked by the CPU tests).
+EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_status_string",
+            "kda_get_device_status", "kda_abi_version")
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__("%s failed: %s (status %d)" % (fn, kda_status_string(status), status))
+        self.status = status
+
+
+def load() -> ctypes.CDLL:
+    """Load libkda.so (built in-tree by linear_attention_rule_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libkda.so is not built (%s); run __graft_entry__.build()" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    lib.kda_prefill.argtypes = [P, P, P, P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, P, P,
+                                I32, P, SZ, P]
+    lib.kda_prefill.restype = ctypes.c_int
+    lib.kda_prefill_workspace_size.argtypes = [I64, I32, I32, I32, I32, I32, ctypes.c_int]
+    lib.kda_prefill_workspace_size.restype = SZ
+    lib.kda_decode.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, ctypes.c_int, P]
+    lib.kda_decode.restype = ctypes.c_int
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_get_device_status.argtypes = [P]
+    lib.kda_get_device_status.restype = ctypes.c_int
+    lib.kda_abi_version.argtypes = []
+    lib.kda_abi_version.restype = I32
+    _lib = lib
+    return lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KDA_F32
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    raise TypeError("q/k/v/out must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libkda must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def kda_status_string(status: int) -> str:
+    return load().kda_status_string(int(status)).decode()
+
+
+def kda_abi_version() -> int:
+    return int(load().kda_abi_version())
+
+
+def kda_prefill_workspace_size(total_tokens: int, num_seqs: int, H: int, dk: int, dv: int,
+                               C: int, dtype: torch.dtype) -> int:
+    code = KDA_F32 if dtype == torch.float32 else KDA_BF16
+    return int(load().kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, code))
+
+
+def kda_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state=None, final_state=None,
+                C: int = 64, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Chunkwise KDA prefill (see kda_prefill in include/libkda.h).
+
+    q, k [T, H, dk], v/out [T, H, dv] (fp32 or bf16); g [T, H, dk] and beta [T, H] fp32;
+    cu_seqlens int32 [N+1] on the device; initial_state / final_state fp32 [N, H, dk, dv]
+    or None.  The workspace is allocated with torch when not given.
+    """
+    lib = load()
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    dt = _dtype_code(q)
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    need = int(lib.kda_prefill_workspace_size(T, N, H, dk, dv, C, dt))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                         _ptr(cu_seqlens), N, T, H, dk, dv, dt, _ptr(out), _ptr(final_state), C,
+                         _ptr(workspace), ws_bytes, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError("kda_prefill", st)
+    return out, final_state
+
+
+def kda_decode(q, k, v, g, beta, state, out, stream=None):
+    """One KDA decode step in place on `state` [N, H, dk, dv] fp32 (kda_decode in libkda.h)."""
+    lib = load()
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    st = lib.kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
+                        N, H, dk, dv, _dtype_code(q), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError("kda_decode", st)
+    return out
+
+
+def kda_get_device_status(stream=None) -> int:
+    """Synchronise `stream`, return and clear the device status word."""
+    return int(load().kda_get_device_status(_stream(stream)))
+
+
+def prefill_launches(dtype: torch.dtype) -> int:
+    """Kernel launches one kda_prefill call makes for inputs of `dtype`."""
+    return 1
+
+
+def prefill_compute_dtype(dtype: torch.dtype) -> str:
+    """Arithmetic type of the prefill path for inputs of `dtype` (operands of the
+    contractions; accumulation and state are fp32 on every path)."""
+    return "f32"

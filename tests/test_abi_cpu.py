@@ -1,0 +1,103 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol the header declares,
+and rejects bad arguments with a status before launching anything (no GPU needed:
+argument checks return before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_rule_b200 import kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_attention_rule_b200 import build
+    build.build()
+    return kda.load()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "libkda.h")) as fh:
+        text = fh.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    assert set(declared_functions()) == set(kda.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    assert kda.kda_abi_version() == 1
+    for code in range(6):
+        s = kda.kda_status_string(code)
+        assert s and s != "unknown status"
+    assert kda.kda_status_string(99) == "unknown status"
+
+
+def _prefill(lib, **kw):
+    P = ctypes.c_void_p
+    a = dict(q=P(4096), k=P(4096), v=P(4096), g=P(4096), beta=P(4096), s0=None, cu=P(4096),
+             N=1, T=64, H=2, dk=64, dv=64, dt=kda.KDA_F32, out=P(4096), sf=None, C=64,
+             ws=None, ws_bytes=0, stream=None)
+    a.update(kw)
+    return lib.kda_prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], a["s0"], a["cu"], a["N"],
+                           a["T"], a["H"], a["dk"], a["dv"], a["dt"], a["out"], a["sf"], a["C"],
+                           a["ws"], a["ws_bytes"], a["stream"])
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    P = ctypes.c_void_p
+    assert _prefill(lib, H=0) == kda.KDA_ERR_INVALID_ARG
+    assert _prefill(lib, N=-1) == kda.KDA_ERR_INVALID_ARG
+    assert _prefill(lib, T=-5) == kda.KDA_ERR_INVALID_ARG
+    assert _prefill(lib, dt=7) == kda.KDA_ERR_INVALID_ARG
+    assert _prefill(lib, dk=96, dv=96) == kda.KDA_ERR_UNSUPPORTED
+    assert _prefill(lib, dk=64, dv=128) == kda.KDA_ERR_UNSUPPORTED
+    assert _prefill(lib, C=48) == kda.KDA_ERR_UNSUPPORTED
+    assert _prefill(lib, dt=kda.KDA_BF16, C=32) == kda.KDA_ERR_UNSUPPORTED
+    assert _prefill(lib, T=1 << 31) == kda.KDA_ERR_UNSUPPORTED
+    assert _prefill(lib, cu=None) == kda.KDA_ERR_INVALID_ARG
+    assert _prefill(lib, q=None) == kda.KDA_ERR_INVALID_ARG
+    assert _prefill(lib, out=None) == kda.KDA_ERR_INVALID_ARG
+    assert _prefill(lib, k=P(4100)) == kda.KDA_ERR_INVALID_ARG       # misaligned
+    assert _prefill(lib, sf=P(4104)) == kda.KDA_ERR_INVALID_ARG      # misaligned
+    assert _prefill(lib, cu=P(4098)) == kda.KDA_ERR_INVALID_ARG      # misaligned int32
+    # nothing to do: valid, returns before touching the device
+    assert _prefill(lib, N=0) == kda.KDA_OK
+
+
+def test_prefill_workspace_check(lib):
+    need = lib.kda_prefill_workspace_size(8192, 1, 32, 128, 128, 64, kda.KDA_BF16)
+    if need > 0:
+        assert _prefill(lib, dk=128, dv=128, H=32, T=8192, dt=kda.KDA_BF16,
+                        ws=ctypes.c_void_p(4096), ws_bytes=need - 1) == kda.KDA_ERR_INVALID_ARG
+        assert _prefill(lib, dk=128, dv=128, H=32, T=8192, dt=kda.KDA_BF16,
+                        ws=ctypes.c_void_p(4096 + 16), ws_bytes=need) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_prefill_workspace_size(100, 1, 2, 96, 96, 64, kda.KDA_F32) == 0
+    assert lib.kda_prefill_workspace_size(-1, 1, 2, 64, 64, 64, kda.KDA_F32) == 0
+
+
+def test_decode_rejects_bad_arguments(lib):
+    P = ctypes.c_void_p
+    def dec(**kw):
+        a = dict(q=P(4096), k=P(4096), v=P(4096), g=P(4096), beta=P(4096), S=P(4096), out=P(4096),
+                 N=4, H=2, dk=128, dv=128, dt=kda.KDA_BF16, stream=None)
+        a.update(kw)
+        return lib.kda_decode(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S"], a["out"], a["N"],
+                              a["H"], a["dk"], a["dv"], a["dt"], a["stream"])
+    assert dec(N=-1) == kda.KDA_ERR_INVALID_ARG
+    assert dec(H=0) == kda.KDA_ERR_INVALID_ARG
+    assert dec(dk=32, dv=32) == kda.KDA_ERR_UNSUPPORTED
+    assert dec(S=None) == kda.KDA_ERR_INVALID_ARG
+    assert dec(g=P(4097)) == kda.KDA_ERR_INVALID_ARG
+    assert dec(dt=5) == kda.KDA_ERR_INVALID_ARG
+    assert dec(N=0) == kda.KDA_OK

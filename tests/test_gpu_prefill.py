@@ -1,0 +1,137 @@
+"""GPU parity of kda_prefill against the fp64 oracle, through the C-ABI."""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_rule_b200 import kda, synthetic
+from tests.gpu_helpers import TOL, check_prefill, run_prefill, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(lens, H, D, dtype, s0_std=0.02, seed=5, g_mean=3.0):
+    return synthetic.make_prefill_inputs(lens, H, D, D, dtype, g_mean, s0_std, seed)
+
+
+def test_config0_tiny_fp32():
+    """Config 0: B=1, H=2, T=256, D=64, C=64, fp32, zero initial state; tolerance 1e-4."""
+    inp = synthetic.make_config_inputs(0)
+    out, fin = run_prefill(inp, C=64)
+    e_o, e_f = check_prefill(inp, out, fin, tol=1e-4)
+    print("config0 max rel err out %.3g final %.3g" % (e_o, e_f))
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+@pytest.mark.parametrize("D", [64, 128])
+def test_fp32_ragged_chunks(C, D):
+    """fp32: lengths around the chunk size (1, C-1, C, C+1, several chunks + tail, empty)."""
+    lens = [1, C - 1, C, C + 1, 0, 5 * C + 3]
+    inp = _inputs(lens, 3, D, torch.float32, seed=C + D)
+    out, fin = run_prefill(inp, C=C)
+    check_prefill(inp, out, fin, tol=1e-4)
+
+
+def test_bf16_ragged_varlen_small():
+    lens = [1000, 64, 63, 65, 1, 0, 300]
+    inp = _inputs(lens, 4, 128, torch.bfloat16, seed=11)
+    out, fin = run_prefill(inp, C=64)
+    check_prefill(inp, out, fin)
+
+
+def test_bf16_d64():
+    inp = _inputs([130, 64, 7], 2, 64, torch.bfloat16, seed=12)
+    out, fin = run_prefill(inp, C=64)
+    check_prefill(inp, out, fin)
+
+
+def test_config1_full_size_sampled_heads():
+    """Config 1 at full size (H=32, T=8192, D=128, bf16) in the benchmark's launch
+    configuration; the oracle checks every output and the final state of 3 heads."""
+    inp = synthetic.make_config_inputs(1)
+    out, fin = run_prefill(inp, C=64)
+    e_o, e_f = check_prefill(inp, out, fin, heads=[0, 13, 31])
+    print("config1 max rel err out %.3g final %.3g" % (e_o, e_f))
+
+
+def test_config2_full_size_sampled_heads():
+    """Config 2 at full size (16 sequences, lengths U[1024, 32768], S0 ~ N(0, 0.02^2))."""
+    inp = synthetic.make_config_inputs(2)
+    out, fin = run_prefill(inp, C=64)
+    e_o, e_f = check_prefill(inp, out, fin, heads=[5, 30])
+    print("config2 max rel err out %.3g final %.3g" % (e_o, e_f))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_continuation_equals_single_run(dtype):
+    """prefill(0:T1) then prefill(T1:T, initial=final) == prefill(0:T) (append-prefill)."""
+    T, T1 = 777, 300
+    inp = _inputs([T], 2, 128, dtype, seed=21)
+    out, fin = run_prefill(inp)
+    a = {k: (v[:T1] if k in ("q", "k", "v", "g", "beta") else v) for k, v in inp.items()}
+    a["cu_seqlens"] = torch.tensor([0, T1], dtype=torch.int32)
+    oA, fA = run_prefill(a)
+    b = {k: (v[T1:] if k in ("q", "k", "v", "g", "beta") else v) for k, v in inp.items()}
+    b["cu_seqlens"] = torch.tensor([0, T - T1], dtype=torch.int32)
+    b["s0"] = torch.from_numpy(fA).float()
+    oB, fB = run_prefill(b)
+    tol = TOL[dtype]
+    import oracle
+    assert oracle.rel_frobenius(np.concatenate([oA, oB]), out) <= tol
+    assert oracle.rel_frobenius(fB, fin) <= tol
+
+
+def test_varlen_equals_separate_runs_bitwise():
+    lens = [200, 64, 1, 129]
+    inp = _inputs(lens, 2, 128, torch.bfloat16, seed=31)
+    out, fin = run_prefill(inp)
+    cu = inp["cu_seqlens"].tolist()
+    for n in range(len(lens)):
+        a, b = cu[n], cu[n + 1]
+        sub = {k: (v[a:b] if k in ("q", "k", "v", "g", "beta") else v) for k, v in inp.items()}
+        sub["cu_seqlens"] = torch.tensor([0, b - a], dtype=torch.int32)
+        sub["s0"] = inp["s0"][n:n + 1]
+        o_n, f_n = run_prefill(sub)
+        np.testing.assert_array_equal(o_n, out[a:b])
+        np.testing.assert_array_equal(f_n, fin[n:n + 1])
+
+
+def test_final_state_may_alias_initial_state_and_be_null():
+    inp = _inputs([100, 70], 2, 64, torch.float32, seed=41)
+    out, fin = run_prefill(inp)
+    d = to_device(inp)
+    S = d["s0"].clone()
+    out2 = torch.empty_like(d["v"])
+    kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out2,
+                    initial_state=S, final_state=S, C=64)
+    np.testing.assert_array_equal(S.double().cpu().numpy(), fin)
+    np.testing.assert_array_equal(out2.double().cpu().numpy(), out)
+    o3, f3 = run_prefill(inp, want_final=False)
+    np.testing.assert_array_equal(o3, out)
+
+
+def test_zero_tokens_copies_initial_state():
+    inp = _inputs([0, 0], 2, 128, torch.float32, seed=51)
+    d = to_device(inp)
+    sf = torch.full_like(d["s0"], float("nan"))
+    out = torch.empty(0, 2, 128, device="cuda")
+    kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out,
+                    initial_state=d["s0"], final_state=sf, C=64)
+    assert kda.kda_get_device_status() == kda.KDA_OK
+    assert torch.equal(sf, d["s0"])
+    sf2 = torch.full_like(d["s0"], float("nan"))
+    kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out,
+                    initial_state=None, final_state=sf2, C=64)
+    assert torch.count_nonzero(sf2) == 0
+
+
+def test_bad_cu_seqlens_reported_by_device():
+    """cu_seqlens that do not end at total_tokens (or decrease) are detected on the
+    device and reported through the status word; no out-of-range access happens
+    because each CTA validates its own sequence bounds before touching tokens."""
+    inp = _inputs([40, 40], 2, 64, torch.float32, seed=61)
+    d = to_device(inp)
+    out = torch.empty_like(d["v"])
+    bad = torch.tensor([0, 50, 30], dtype=torch.int32, device="cuda")   # decreasing, short
+    kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], bad, out, C=64)
+    assert kda.kda_get_device_status() == kda.KDA_ERR_BAD_SEQLENS
+    assert kda.kda_get_device_status() == kda.KDA_OK   # cleared by the read
