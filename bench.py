@@ -226,7 +226,7 @@ def bench_gpu(args):
     ms_local = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms_local, world, dev)
     value = world * T / (ms * 1e-3)
-    launches_per_prefill = kda.prefill_launches(cfg.dtype)
+    launches_per_prefill = kda.prefill_launches(cfg.dtype, D)
 
     flops, page_bytes = prefill_page_counts(lengths, H, D, C)
     strict = prefill_strict_bytes(lengths, H, D, 2 if cfg.dtype == torch.bfloat16 else 4,
@@ -335,7 +335,7 @@ def bench_gpu(args):
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": kda.prefill_compute_dtype(cfg.dtype),
+        "dtype": kda.prefill_compute_dtype(cfg.dtype, D),
         "data": "synthetic",
         "config": {"workload": cfg.name, "T": T, "H": H, "D": D, "C": C,
                    "l2": "inputs larger than L2 (%.0f MB resident per step)" % (in_bytes_total / 1e6),

@@ -8,12 +8,16 @@
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
 #include "kda_prefill_simt.cuh"
+#include "kda_prefill_tc.cuh"
 
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool supported_dim(int32_t dk, int32_t dv) { return dk == dv && (dk == 64 || dk == 128); }
+
+// bf16 with d = 128 runs on the tensor cores; fp32 (and bf16 with d = 64) on CUDA cores.
+bool tensor_core_path(kda_dtype dt, int32_t dk) { return dt == KDA_BF16 && dk == 128; }
 
 bool valid_chunk(kda_dtype dt, int32_t C) {
     if (dt == KDA_BF16) return C == 64;
@@ -58,7 +62,8 @@ size_t kda_prefill_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_
     if (total_tokens < 0 || num_seqs < 0 || H <= 0 || !supported_dim(dk, dv) ||
         !valid_chunk(dt, C))
         return 0;
-    return 0;
+    if (!tensor_core_path(dt, dk)) return 0;
+    return kda::tc::workspace_bytes(total_tokens, num_seqs, H);
 }
 
 kda_status kda_prefill(const void* q, const void* k, const void* v, const float* g,
@@ -85,7 +90,10 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t err;
-    if (dt == KDA_F32)
+    if (tensor_core_path(dt, dk))
+        err = kda::tc::launch_prefill(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
+                                      total_tokens, H, out, final_state, workspace, st);
+    else if (dt == KDA_F32)
         err = dispatch_simt<float>(dk, C, q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
                                    total_tokens, H, out, final_state, st);
     else

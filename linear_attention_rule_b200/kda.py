@@ -144,12 +144,18 @@ def kda_get_device_status(stream=None) -> int:
     return int(load().kda_get_device_status(_stream(stream)))
 
 
-def prefill_launches(dtype: torch.dtype) -> int:
-    """Kernel launches one kda_prefill call makes for inputs of `dtype`."""
-    return 1
+def _tensor_core_path(dtype: torch.dtype, D: int) -> bool:
+    # mirrors tensor_core_path() in csrc/libkda.cu
+    return dtype == torch.bfloat16 and D == 128
 
 
-def prefill_compute_dtype(dtype: torch.dtype) -> str:
-    """Arithmetic type of the prefill path for inputs of `dtype` (operands of the
-    contractions; accumulation and state are fp32 on every path)."""
-    return "f32"
+def prefill_launches(dtype: torch.dtype, D: int = 128) -> int:
+    """Kernel launches one kda_prefill call makes: chunk index, preparation and
+    recurrence on the tensor-core path; one chunk-serial kernel on the CUDA-core path."""
+    return 3 if _tensor_core_path(dtype, D) else 1
+
+
+def prefill_compute_dtype(dtype: torch.dtype, D: int = 128) -> str:
+    """Operand type of the prefill contractions (accumulation and the state are fp32
+    on every path)."""
+    return "bf16" if _tensor_core_path(dtype, D) else "f32"
