@@ -117,6 +117,42 @@ kda_status kda_decode(const void *q, const void *k, const void *v, const float *
                       const float *beta, float *state_inout, void *out, int32_t N,
                       int32_t H, int32_t dk, int32_t dv, kda_dtype dt, kda_stream_t stream);
 
+/*
+ * Allocation-free prefill.  The pages have no counterpart: this is a library
+ * convenience, not part of the method.
+ *
+ * Some callers cannot hand kda_prefill a workspace: their device memory is owned by
+ * another allocator (for instance a serving engine that reserved nearly all HBM for its
+ * own pools, where a cudaMalloc fails or fragments that pool), or they run on a
+ * latency-critical path where a cudaMalloc stall or the device-wide synchronisation of
+ * cudaFree is not acceptable.  kda_prefill_noalloc serves them from scratch memory that
+ * lives inside the library: a static device array of KDA_NOALLOC_SCRATCH_BYTES (64 MiB)
+ * that every GPU which loads the library holds until the process exits.  It never calls
+ * cudaMalloc, cudaFree or any other allocating routine.
+ *
+ *   - Arguments and layouts are those of kda_prefill without workspace / ws_bytes.
+ *   - Only the tensor-core problem (bf16, dk = dv = 128, C = 64) is served; any other
+ *     problem returns KDA_ERR_UNSUPPORTED (the CUDA-core path needs no scratch: call
+ *     kda_prefill with a NULL workspace instead).
+ *   - A problem whose kda_prefill_workspace_size exceeds KDA_NOALLOC_SCRATCH_BYTES returns
+ *     KDA_ERR_UNSUPPORTED before anything is launched (with H = 32 and one sequence that
+ *     is anything beyond 1,791 tokens).
+ *   - The first call on each device looks the scratch address up (cudaGetSymbolAddress,
+ *     with that device current); make that first call before any stream capture begins.
+ *   - All calls on a device share the one scratch array, which keeps whatever the last
+ *     call left in it.  Every byte a call reads from it is written earlier by the same
+ *     call, so nothing has to be cleared between calls.  Calls that overlap on the GPU
+ *     (two streams without ordering between them, or two threads) race on the array and
+ *     corrupt each other's results: order them on one stream.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *initial_state,
+                               const int32_t *cu_seqlens, int32_t num_seqs,
+                               int64_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                               kda_dtype dt, void *out, float *final_state, int32_t C,
+                               kda_stream_t stream);
+
 /* Static English text for a status code (never NULL). */
 const char *kda_status_string(kda_status s);
 

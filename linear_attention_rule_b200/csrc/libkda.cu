@@ -4,6 +4,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "libkda.h"
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
@@ -139,3 +141,51 @@ kda_status kda_get_device_status(kda_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// Allocation-free prefill: the tensor-core prefill with its workspace taken from a static
+// device array inside this library instead of from the caller (for callers that cannot
+// allocate device memory where they run).  Every GPU that loads the library holds the
+// array until the process exits; all calls on a device share it.
+static __device__ __align__(256) uint8_t g_kda_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once per device.
+// The array's name is only a host-side stand-in; the kernels must get this address.
+cudaError_t noalloc_scratch(void** ptr) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_kda_noalloc_scratch);
+        if (err != cudaSuccess) return err;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+}  // namespace
+
+extern "C" kda_status kda_prefill_noalloc(const void* q, const void* k, const void* v,
+                                          const float* g, const float* beta,
+                                          const float* initial_state, const int32_t* cu_seqlens,
+                                          int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                          int32_t dk, int32_t dv, kda_dtype dt, void* out,
+                                          float* final_state, int32_t C, kda_stream_t stream) {
+    if (num_seqs < 0 || total_tokens < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (dt != KDA_BF16 || dk != 128 || dv != 128 || C != 64) return KDA_ERR_UNSUPPORTED;
+    const size_t need = kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, dt);
+    if (need > KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return KDA_OK;
+    void* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
+    return kda_prefill(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_tokens, H,
+                       dk, dv, dt, out, final_state, C, scratch, KDA_NOALLOC_SCRATCH_BYTES, stream);
+}

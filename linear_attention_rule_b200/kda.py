@@ -27,7 +27,10 @@ KDA_BF16 = 1
 
 # Every symbol include/libkda.h declares (checked by the CPU tests).
 EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_status_string",
-            "kda_get_device_status", "kda_abi_version")
+            "kda_get_device_status", "kda_abi_version", "kda_prefill_noalloc")
+
+# Size of the library-owned scratch behind kda_prefill_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 
@@ -60,6 +63,9 @@ def load() -> ctypes.CDLL:
     lib.kda_get_device_status.restype = ctypes.c_int
     lib.kda_abi_version.argtypes = []
     lib.kda_abi_version.restype = I32
+    lib.kda_prefill_noalloc.argtypes = [P, P, P, P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int,
+                                        P, P, I32, P]
+    lib.kda_prefill_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -124,6 +130,27 @@ def kda_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state=None, final_sta
                          _ptr(workspace), ws_bytes, _stream(stream))
     if st != KDA_OK:
         raise KdaError("kda_prefill", st)
+    return out, final_state
+
+
+def kda_prefill_noalloc(q, k, v, g, beta, cu_seqlens, out, initial_state=None,
+                        final_state=None, C: int = 64, stream=None):
+    """kda_prefill without a workspace, for callers that cannot allocate device memory
+    where they run (their memory belongs to another allocator, or an allocation's stall
+    is not acceptable): the library's own static scratch is used instead.  bf16 with
+    d = 128 and C = 64 only; problems needing more than NOALLOC_SCRATCH_BYTES of scratch
+    are rejected.  Calls sharing a device must not overlap on the GPU."""
+    lib = load()
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    st = lib.kda_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                 _ptr(initial_state), _ptr(cu_seqlens), N, T, H, dk, dv,
+                                 _dtype_code(q), _ptr(out), _ptr(final_state), C, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError("kda_prefill_noalloc", st)
     return out, final_state
 
 
