@@ -171,80 +171,87 @@ def oracle_sample_tokens_per_s(inp, target_s: float):
     dt = run(ts)
     ts = int(max(32, min(T, ts * target_s / max(dt, 1e-6))))
     dt = run(ts)
-    return ts / dt, ts, dt, threads
+    reps, total = 1, dt
+    while total < target_s * 0.8 and reps < 1000:   # whole workload is quick: repeat it
+        total += run(ts)
+        reps += 1
+    return reps * ts / total, ts, total, threads
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def bench_gpu(args):
+def timed(stream, dev, world, steps, fn):
+    """Run fn `steps` times between CUDA events on `stream` (barrier + synchronize on
+    both sides); returns (this rank's ms per step, max over ranks, clock summary)."""
+    import torch
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms_local = e0.elapsed_time(e1) / steps
+    return ms_local, max_over_ranks(ms_local, world, dev), clk.summary()
+
+
+def setup_prefill(dev, rank):
     import torch
     from linear_attention_rule_b200 import kda, synthetic
-
-    rank, local_rank, world = rank_env()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-    peaks = load_peaks()
-
-    # ---- prefill workload (resident inputs) --------------------------------------------
     cfg = synthetic.CONFIGS[PREFILL_CFG]
     lengths = synthetic.draw_lengths(cfg)
     D, H, C = cfg.D, cfg.H, cfg.C
     inp = synthetic.make_prefill_inputs(lengths, H, D, D, cfg.dtype, cfg.g_mean, cfg.s0_std,
                                         rank_seed(cfg.seed, rank))
-    T = inp["q"].shape[0]
-    N = len(lengths)
+    T, N = inp["q"].shape[0], len(lengths)
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     out = torch.empty(T, H, D, dtype=cfg.dtype, device=dev)
     fin = torch.empty(N, H, D, D, dtype=torch.float32, device=dev)
     ws_bytes = kda.kda_prefill_workspace_size(T, N, H, D, D, C, cfg.dtype)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    in_bytes_total = sum(d[k].numel() * d[k].element_size() for k in ("q", "k", "v", "g", "beta"))
+    return dict(cfg=cfg, lengths=lengths, inp=inp, d=d, out=out, fin=fin, ws=ws, T=T, N=N,
+                D=D, H=H, C=C)
 
-    def prefill_step():
-        kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out,
-                        initial_state=d["s0"], final_state=fin, C=C, workspace=ws, stream=stream)
+
+def bench_prefill(args, P, dev, stream, world, peaks):
+    from linear_attention_rule_b200 import kda
+    cfg, d, D, H, C, T = P["cfg"], P["d"], P["D"], P["H"], P["C"], P["T"]
+
+    def step():
+        kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], P["out"],
+                        initial_state=d["s0"], final_state=P["fin"], C=C, workspace=P["ws"],
+                        stream=stream)
 
     for _ in range(args.warmup):
-        prefill_step()
-    torch.cuda.synchronize(dev)
+        step()
     assert kda.kda_get_device_status(stream) == kda.KDA_OK
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    with ClockSampler(dev) as clk:
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            prefill_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier(world)
-    ms_local = e0.elapsed_time(e1) / args.steps
-    ms = max_over_ranks(ms_local, world, dev)
-    value = world * T / (ms * 1e-3)
-    launches_per_prefill = kda.prefill_launches(cfg.dtype, D)
-
-    flops, page_bytes = prefill_page_counts(lengths, H, D, C)
-    strict = prefill_strict_bytes(lengths, H, D, 2 if cfg.dtype == torch.bfloat16 else 4,
-                                  inp["s0"] is not None, True)
+    ms_local, ms, clocks = timed(stream, dev, world, args.steps, step)
+    assert kda.kda_get_device_status(stream) == kda.KDA_OK
+    flops, page_bytes = prefill_page_counts(P["lengths"], H, D, C)
+    strict = prefill_strict_bytes(P["lengths"], H, D, 2 if cfg.dtype.itemsize == 2 else 4,
+                                  P["inp"]["s0"] is not None, True)
     t_s = ms_local * 1e-3
-    achieved_gbs = page_bytes / t_s / 1e9
+    achieved = page_bytes / t_s / 1e9
     roofline = {
-        "bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
-        "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
-        "traffic": None, "kernel": "kda_prefill (whole path)",
-        "bytes_per_launch": page_bytes, "counts": "page counts 8C^2+22CD B per chunk-head + 8D^2 per head",
+        "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+        "kernel": "kda_prefill (whole path: chunk index + prep + recurrence)",
+        "bytes_per_launch": page_bytes,
+        "counts": "pages' 8C^2+22CD bytes per chunk-head + 8D^2 per head",
         "peak_source": peaks["source"],
         "tensor_frac": round(flops / t_s / 1e12 / peaks["bf16_tflops"], 4),
         "strict_frac": round(strict / t_s / 1e9 / peaks["hbm_gbs"], 4),
     }
-    clocks = clk.summary()
+    return dict(value=world * T / (ms * 1e-3), ms=ms, ms_local=ms_local, roofline=roofline,
+                clocks=clocks, launches=kda.prefill_launches(cfg.dtype, D) * args.steps,
+                step=step)
 
-    # ---- decode workload ---------------------------------------------------------------
+
+def bench_decode(args, dev, stream, rank, world, peaks):
+    import torch
+    from linear_attention_rule_b200 import kda, synthetic
     dcfg = synthetic.CONFIGS[DECODE_CFG]
     Nd, Hd, Dd = dcfg.N, dcfg.H, dcfg.D
     S = synthetic.make_decode_state(Nd, Hd, Dd, Dd, dcfg.s0_std, rank_seed(dcfg.seed, rank)).to(dev)
@@ -255,95 +262,104 @@ def bench_gpu(args):
         steps_in.append({k: v.to(dev) for k, v in x.items()})
     dout = torch.empty(Nd, Hd, Dd, dtype=dcfg.dtype, device=dev)
 
-    def decode_step():
+    def step():
         for x in steps_in:
             kda.kda_decode(x["q"], x["k"], x["v"], x["g"], x["beta"], S, dout, stream=stream)
 
     for _ in range(args.warmup):
-        decode_step()
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    with ClockSampler(dev) as dclk:
-        e0.record(stream)
-        for _ in range(args.steps):
-            decode_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier(world)
-    dms_local = e0.elapsed_time(e1) / args.steps
-    dms = max_over_ranks(dms_local, world, dev)
+        step()
+    ms_local, ms, clocks = timed(stream, dev, world, args.steps, step)
     state_bytes = 8 * Dd * Dd * Nd * Hd * dcfg.steps
-    d_gbs = world * state_bytes / (dms * 1e-3) / 1e9
-    d_gbs_local = state_bytes / (dms_local * 1e-3) / 1e9
-    decode = {
-        "workload": dcfg.name, "value": round(d_gbs, 1), "unit": "GB/s (fp32 state read+write)",
-        "ms_per_step": round(dms, 4), "steps_per_call": dcfg.steps,
-        "seq_tokens_per_s": round(world * Nd * dcfg.steps / (dms * 1e-3), 1),
-        "roofline": {"bound": "hbm", "achieved": round(d_gbs_local, 1), "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": round(d_gbs_local / peaks["hbm_gbs"], 4),
+    gbs_local = state_bytes / (ms_local * 1e-3) / 1e9
+    return {
+        "workload": dcfg.name, "value": round(world * state_bytes / (ms * 1e-3) / 1e9, 1),
+        "unit": "GB/s (fp32 state read+write)", "ms_per_step": round(ms, 4),
+        "steps_per_call": dcfg.steps,
+        "seq_tokens_per_s": round(world * Nd * dcfg.steps / (ms * 1e-3), 1),
+        "roofline": {"bound": "hbm", "achieved": round(gbs_local, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(gbs_local / peaks["hbm_gbs"], 4),
                      "traffic": None, "kernel": "kda::decode_kernel",
                      "bytes_per_launch": 8 * Dd * Dd * Nd * Hd,
-                     "counts": "page count 8 D^2 bytes per head-token",
-                     "peak_source": peaks["source"]},
-        "clocks": dclk.summary(), "gpu_launches": dcfg.steps * args.steps,
+                     "counts": "pages' 8 D^2 bytes per head-token", "peak_source": peaks["source"]},
+        "clocks": clocks, "gpu_launches": dcfg.steps * args.steps,
     }
-    del steps_in, S
 
-    # ---- end to end from pinned host buffers -------------------------------------------
-    e2e = None
-    if not args.no_e2e:
-        h = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
-        hout = torch.empty(T, H, D, dtype=cfg.dtype).pin_memory()
-        hfin = torch.empty(N, H, D, D, dtype=torch.float32).pin_memory()
 
-        def e2e_step():
-            for k in ("q", "k", "v", "g", "beta", "cu_seqlens"):
-                d[k].copy_(h[k], non_blocking=True)
-            prefill_step()
-            hout.copy_(out, non_blocking=True)
-            hfin.copy_(fin, non_blocking=True)
+def bench_e2e(args, P, pre, dev, stream, world):
+    """Same metric through the public API with host buffers: pinned host -> device copies
+    of the step's inputs, the prefill, and device -> host copies of O and the final state,
+    all inside the timed region."""
+    import torch
+    d, out, fin, inp = P["d"], P["out"], P["fin"], P["inp"]
+    h = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+    hout = torch.empty_like(out, device="cpu").pin_memory()
+    hfin = torch.empty_like(fin, device="cpu").pin_memory()
+    keys = ("q", "k", "v", "g", "beta", "cu_seqlens") + (("s0",) if inp["s0"] is not None else ())
 
-        for _ in range(args.warmup):
-            e2e_step()
-        torch.cuda.synchronize(dev)
-        barrier(world)
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(world)
-        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
-        h2d = sum(h[k].numel() * h[k].element_size() for k in ("q", "k", "v", "g", "beta", "cu_seqlens"))
-        d2h = hout.numel() * hout.element_size() + hfin.numel() * hfin.element_size()
-        e2e = {"value": round(world * T / (ems * 1e-3), 1), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ems, 4)}
+    def step():
+        for k in keys:
+            d[k].copy_(h[k], non_blocking=True)
+        pre["step"]()
+        hout.copy_(out, non_blocking=True)
+        hfin.copy_(fin, non_blocking=True)
 
-    # ---- CPU oracle baseline (rank 0, one GPU only) ------------------------------------
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, ts, secs, threads = oracle_sample_tokens_per_s(inp, args.cpu_seconds)
-        cpu = {"value": round(tps, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": "first %d tokens x all %d heads of the same workload, fp64, %.1f s" % (ts, H, secs)}
+    for _ in range(args.warmup):
+        step()
+    _, ms, _ = timed(stream, dev, world, args.steps, step)
+    h2d = sum(h[k].numel() * h[k].element_size() for k in keys)
+    d2h = hout.numel() * hout.element_size() + hfin.numel() * hfin.element_size()
+    return {"value": round(world * P["T"] / (ms * 1e-3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4)}
 
+
+def bench_gpu(args):
+    import torch
+    from linear_attention_rule_b200 import kda
+
+    rank, local_rank, world = rank_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+
+    line = {}
+    if args.workload in ("all", "prefill"):
+        P = setup_prefill(dev, rank)
+        pre = bench_prefill(args, P, dev, stream, world, peaks)
+        decode = bench_decode(args, dev, stream, rank, world, peaks) if args.workload == "all" else None
+        e2e = None if args.no_e2e else bench_e2e(args, P, pre, dev, stream, world)
+        cpu = None
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            tps, ts, secs, threads = oracle_sample_tokens_per_s(P["inp"], args.cpu_seconds)
+            cpu = {"value": round(tps, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                   "sample": "first %d tokens x all %d heads of the same workload (repeated), "
+                             "fp64, %.1f s" % (ts, P["H"], secs)}
+        cfg = P["cfg"]
+        line = {
+            "metric": METRIC, "value": round(pre["value"], 1), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(pre["ms"], 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": kda.prefill_compute_dtype(cfg.dtype, P["D"]),
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "T": P["T"], "H": P["H"], "D": P["D"], "C": P["C"],
+                       "l2": "inputs larger than L2 (%.0f MB resident per step)" % (
+                           sum(P["d"][k].numel() * P["d"][k].element_size()
+                               for k in ("q", "k", "v", "g", "beta")) / 1e6),
+                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "roofline": pre["roofline"], "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
+            "clocks": pre["clocks"], "gpu_launches": pre["launches"],
+        }
+    else:
+        line = {"decode": bench_decode(args, dev, stream, rank, world, peaks)}
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
-    if rank != 0:
-        return
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": kda.prefill_compute_dtype(cfg.dtype, D),
-        "data": "synthetic",
-        "config": {"workload": cfg.name, "T": T, "H": H, "D": D, "C": C,
-                   "l2": "inputs larger than L2 (%.0f MB resident per step)" % (in_bytes_total / 1e6),
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
-        "roofline": roofline, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
-        "clocks": clocks, "gpu_launches": launches_per_prefill * args.steps,
-    }
-    print(json.dumps(line), flush=True)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -398,6 +414,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--workload", choices=["all", "prefill", "decode"], default="all",
+                    help="restrict the run (profiling); the JSON line needs 'all'")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -1,6 +1,7 @@
 """White-box check of the tensor-core preparation kernel: decode the per-(chunk, head)
-workspace record (shared-memory operand images, 128-byte swizzle) and compare every
-chunk tensor with the fp64 chunked form of the oracle."""
+workspace record (shared-memory operand images with a 128-byte swizzle, and value-channel
+slices) and compare every chunk tensor with the fp64 chunked form of the oracle:
+M = -K_res^T W, B = K_res^T U, P = Q_dec - Aqk W, R = Aqk U, gamma."""
 import numpy as np
 import pytest
 import torch
@@ -11,22 +12,23 @@ from tests.gpu_helpers import to_device
 
 pytestmark = pytest.mark.gpu
 
-REC_BYTES = 74240
-
-
-def _sw128(img: np.ndarray, rows: int) -> np.ndarray:
-    """bf16 image of `rows` rows x 64 elements, 128-byte swizzle -> float array."""
-    b = img[: rows * 128].reshape(rows, 8, 16)
-    out = np.empty((rows, 8, 16), dtype=np.uint8)
-    for r in range(rows):
-        for ch in range(8):
-            out[r, ch] = b[r, ch ^ (r % 8)]
-    return _bf16(out.reshape(rows, 128))
+REC_BYTES = 98816
+KB = 24576
 
 
 def _bf16(u8: np.ndarray) -> np.ndarray:
     u16 = u8.copy().view(np.uint16).astype(np.uint32) << 16
     return u16.view(np.float32).astype(np.float64)
+
+
+def _sw128(img: np.ndarray, rows: int) -> np.ndarray:
+    """bf16 image of `rows` rows x 64 elements, 128-byte swizzle -> float array."""
+    b = img[: rows * 128].reshape(rows, 8, 16)
+    out = np.empty_like(b)
+    for r in range(rows):
+        for ch in range(8):
+            out[r, ch] = b[r, ch ^ (r % 8)]
+    return _bf16(out.reshape(rows, 128))
 
 
 def _records(nrow, seed):
@@ -38,8 +40,7 @@ def _records(nrow, seed):
     kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out, C=64,
                     workspace=ws)
     assert kda.kda_get_device_status() == kda.KDA_OK
-    rec = ws.cpu().numpy()[1024:1024 + REC_BYTES]
-    return inp, rec
+    return inp, ws.cpu().numpy()[1024:1024 + REC_BYTES]
 
 
 @pytest.mark.parametrize("nrow", [64, 37])
@@ -49,27 +50,24 @@ def test_prep_record_matches_chunked_oracle(nrow):
     T = chunked.chunk_tensors(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["g"]),
                               inp["beta"][:, 0].double().numpy())
     n = nrow
-    Wt = _sw128(rec[0:16384], 128)            # [i][r] = W[r][i]
-    Qt = _sw128(rec[16384:32768], 128)        # [i][r] = Q_dec[r][i]
-    Kr = _sw128(rec[32768:49152], 128)        # [i][r] = K_res[r][i]
-    Aq = _sw128(rec[49152:57344], 64)         # [r][s]
-    Ut = _bf16(rec[57344:73728].reshape(128, 128))  # [j][r] = U[r][j]
-    gam = rec[73728:74240].copy().view(np.float32).astype(np.float64)
+    M_ref = -T["K_res"].T @ T["W"]
+    B_ref = T["K_res"].T @ T["U"]
+    P_ref = T["Q_dec"] - T["Aqk"] @ T["W"]
+    R_ref = T["Aqk"] @ T["U"]
+    P = np.concatenate([_sw128(rec[kb * KB:kb * KB + 8192], 64) for kb in range(2)], axis=1)
+    M = np.concatenate([_sw128(rec[8192 + kb * KB:8192 + kb * KB + 16384], 128) for kb in range(2)], axis=1)
+    B = np.concatenate([_bf16(rec[49152 + s * 8192:49152 + (s + 1) * 8192].reshape(128, 64))
+                        for s in range(4)], axis=1)
+    R = np.concatenate([_bf16(rec[81920 + s * 4096:81920 + (s + 1) * 4096].reshape(64, 64))
+                        for s in range(4)], axis=1)
+    gam = rec[98304:98816].copy().view(np.float32).astype(np.float64)
 
     def rel(a, b):
         return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
 
-    errs = {
-        "Q_dec": rel(Qt[:, :n].T, T["Q_dec"]),
-        "K_res": rel(Kr[:, :n].T, T["K_res"]),
-        "Aqk": rel(Aq[:n, :n], T["Aqk"]),
-        "W": rel(Wt[:, :n].T, T["W"]),
-        "U": rel(Ut[:, :n].T, T["U"]),
-        "gamma": rel(gam, T["gamma"]),
-    }
+    errs = {"M": rel(M, M_ref), "B": rel(B, B_ref), "P": rel(P[:n], P_ref), "R": rel(R[:n], R_ref),
+            "gamma": rel(gam, T["gamma"])}
     print(nrow, {k: "%.2e" % v for k, v in errs.items()})
     for k, e in errs.items():
-        assert e < 1e-2, (k, e)
-    # padded rows are exactly zero
-    assert np.all(Qt[:, n:] == 0) and np.all(Wt[:, n:] == 0) and np.all(Ut[:, n:] == 0)
-    assert np.all(Aq[n:, :] == 0)
+        assert e < 2e-2, (k, e)
+    assert np.all(P[n:] == 0) and np.all(R[n:] == 0)
