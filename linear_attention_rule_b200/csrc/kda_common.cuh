@@ -36,3 +36,18 @@ __device__ __forceinline__ bool kda_seq_bounds(const int32_t* cu, int n, int num
     if (!ok) kda_set_status(KDA_ERR_BAD_SEQLENS);
     return ok;
 }
+
+// Optional phase tracing (compile with -DKDA_TRACE): SM clock stamps of chosen points of
+// chosen CTAs, read back with kda_debug_read_trace.  Compiled out by default.
+#ifdef KDA_TRACE
+constexpr int kTraceSlots = 1 << 16;
+__device__ unsigned long long g_kda_trace[kTraceSlots];
+#define KDA_TRACE_POINT(cond, slot)                                                \
+    do {                                                                           \
+        if ((cond) && (slot) < kTraceSlots) g_kda_trace[(slot)] = clock64();       \
+    } while (0)
+#else
+#define KDA_TRACE_POINT(cond, slot) \
+    do {                            \
+    } while (0)
+#endif

@@ -14,20 +14,22 @@
 //
 //   chunk_index_kernel  cu_seqlens -> first chunk of every sequence (device side, no host
 //                       sync); validates cu_seqlens.
-//   prep_kernel         one CTA per (chunk, head), fully parallel, 2 CTAs per SM:
+//   prep_kernel         one CTA of 8 warps per (chunk, head), fully parallel, 2 CTAs per SM:
 //                         TMA: q, k, v tiles (128-byte swizzled) and g into shared memory
 //                         a, gamma, Q_dec = q e^a, K_dec = k e^a, K_inv = k e^-a      (FFMA/MUFU)
 //                         [K_dec; Q_dec] K_inv^T                                      (MMA 128x64x128)
 //                         L = strict_tril(beta K_dec K_inv^T), Aqk = tril(Q_dec K_inv^T)
-//                         INV = (I + L)^-1 by forward substitution (fp32)
+//                         INV = (I + L)^-1: 16x16 diagonal blocks by forward substitution,
+//                                               then block doubling 16 -> 32 -> 64 (fp32)
 //                         [W | U] = INV diag(beta) [K_dec | V]                       (MMA 128x256x64)
 //                         [M | B] = [-K_res^T W | K_res^T U]                         (MMA 128x256x64)
 //                         [Aqk W | Aqk U] -> P, R                                    (MMA 128x256x64)
 //                       and writes one record per (chunk, head): the shared-memory
 //                       operand images of M and P, value-channel slices of B and R, gamma.
-//   rec_kernel          one CTA per (sequence, head, 32 value channels): the chunk chain
-//                       with the fp32 state slice in registers, records streamed in by a
-//                       loader warp (3 stages of bulk copies).
+//   rec_kernel          one CTA per (sequence, head, 64 value channels): the chunk chain
+//                       with the fp32 state slice in registers; a loader warp streams the
+//                       records in (2 stages of bulk copies) and an issuer warp launches the
+//                       tensor-core products, hand-offs through mbarriers only.
 #pragma once
 
 #include <cuda.h>
@@ -42,32 +44,36 @@ using namespace kda::sm100;
 
 constexpr int D = 128;   // d_k = d_v
 constexpr int C = 64;    // chunk
-constexpr int NV = 32;   // value channels per recurrence CTA
+constexpr int NV = 64;   // value channels per recurrence CTA
 constexpr int NSL = D / NV;
 
 // ---- record of one (chunk, head) ---------------------------------------------------------
-// P and M as K-major A images (rows of 128 B, 128-byte swizzle), K blocks of 64 channels
-// interleaved so that a 128-row descriptor starting at P_kb covers P (rows 0-63) followed
-// by rows 0-63 of M_kb (finite filler rows whose products are never read).
-constexpr uint32_t kRecP0 = 0;          // P  rows r,   channels   0..63   (8 KB)
-constexpr uint32_t kRecM0 = 8192;       // M  rows i,   channels   0..63   (16 KB)
-constexpr uint32_t kRecKB = 24576;      // stride between the two K blocks
-constexpr uint32_t kRecB = 49152;       // B  [slice][i 128][32] bf16      (4 x 8 KB)
-constexpr uint32_t kRecR = 81920;       // R  [slice][r 64][32]  bf16      (4 x 4 KB)
+// Shared-memory operand images (rows of 128 B, 128-byte swizzle) and value-channel slices:
+constexpr uint32_t kRecP0 = 0;          // P  K-major rows r (64), channels 0..63 / 64..127 (2 x 8 KB)
+constexpr uint32_t kRecM0 = 16384;      // M  K-major rows i (128), channels 0..63 / 64..127 (2 x 16 KB)
+constexpr uint32_t kRecB = 49152;       // B  [slice][i 128][64] bf16, rows swizzled (2 x 16 KB)
+constexpr uint32_t kRecR = 81920;       // R  [slice][r 64][64]  bf16, rows swizzled (2 x 8 KB)
 constexpr uint32_t kRecGamma = 98304;   // gamma fp32 [128]
 constexpr uint32_t kRecBytes = 98816;
+// bf16 state entering each (chunk, head): 2 slices of the MN-major image [i 128][64], 128-byte
+// swizzle, written by the recurrence and read by the output kernel.
+constexpr uint32_t kStateImgBytes = 32768;
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace: [chunk offsets int32 (N+1)] [records (max_chunks x H)]
 __host__ __device__ inline size_t ws_records_offset(int num_seqs) {
     return align_up(sizeof(int32_t) * (size_t)(num_seqs + 1), 1024);
 }
 __host__ inline int64_t max_chunks(int64_t total_tokens, int num_seqs) {
     return total_tokens / C + num_seqs;
 }
-__host__ inline size_t workspace_bytes(int64_t total_tokens, int num_seqs, int H) {
+__host__ inline size_t ws_states_offset(int64_t total_tokens, int num_seqs, int H) {
     return ws_records_offset(num_seqs) + (size_t)max_chunks(total_tokens, num_seqs) * H * kRecBytes;
+}
+// Workspace: [chunk offsets int32 (N+1)] [records (max_chunks x H)] [chunk states (max_chunks x H)]
+__host__ inline size_t workspace_bytes(int64_t total_tokens, int num_seqs, int H) {
+    return ws_states_offset(total_tokens, num_seqs, H) +
+           (size_t)max_chunks(total_tokens, num_seqs) * H * kStateImgBytes;
 }
 
 // ------------------------------------------------------------------ chunk index
@@ -146,23 +152,25 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tma
 }
 
 // ------------------------------------------------------------------ chunk preparation
-constexpr int kPrepThreads = 128;
+constexpr int kPrepThreads = 256;
 struct PrepSmem {
     // operand region: 128-byte-swizzled tiles of 64 rows (tokens) x 64 channels
     static constexpr uint32_t KD0 = 0, QD0 = 8192, KD1 = 16384, QD1 = 24576;
     static constexpr uint32_t V0 = 32768, KI0 = 40960, V1 = 49152, KI1 = 57344;
     static constexpr uint32_t BLK = 16384;   // stride between the channel halves
-    // g tile fp32 [64][128] (plain); after the elementwise pass: Abar, Aqk, L
+    // g tile fp32 [64][128] (plain); after the decay: Abar image, Aqk image, L / INV fp32
     static constexpr uint32_t GR = 65536;
-    static constexpr uint32_t ABAR = GR, AQK = GR + 8192, LL = GR + 16384;
-    static constexpr uint32_t XCH = GR + 32768;       // [8 row blocks][128] fp32 partial sums
-    static constexpr uint32_t BETA = XCH + 4096;      // [64]
+    static constexpr uint32_t ABAR = GR, AQK = GR + 8192, LI = GR + 16384;   // LI: [64][68]
+    static constexpr uint32_t XCH = GR + 33792;      // decay partials [8][128]; later T [32][36]
+    static constexpr uint32_t BETA = XCH + 4608;     // [64]
     static constexpr uint32_t BAR = BETA + 256;
     static constexpr uint32_t TMEM = BAR + 8;
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;  // + alignment slack
 };
+constexpr int kLP = 68;                                   // row pitch of L / INV (16-byte rows)
+constexpr int kTP = 36;                                   // row pitch of the product scratch
 constexpr uint32_t kPrepTmemCols = 256;
-constexpr uint32_t kPrepTx = 3 * 16384 + 32768;        // q, k, v (2 boxes of 8 KB each) + g
+constexpr uint32_t kPrepTx = 3 * 16384 + 32768;           // q, k, v (2 boxes of 8 KB each) + g
 
 __device__ __forceinline__ bool prep_sync_ok(bool ok, int tid) {
     if (__syncthreads_or(!ok)) {
@@ -192,8 +200,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t bar = sb + S::BAR;
     float* sBeta = reinterpret_cast<float*>(sm + S::BETA);
     float* sX = reinterpret_cast<float*>(sm + S::XCH);
-    float* sL = reinterpret_cast<float*>(sm + S::LL);
+    float* sLI = reinterpret_cast<float*>(sm + S::LI);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, wh = warp >> 2;   // TMEM lane quarter, column half
     bool ok = true;
     uint32_t phase = 0;
 
@@ -207,6 +216,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
+    const uint32_t tl = tmem + ((uint32_t)(32 * wq) << 16);   // this warp's TMEM lanes
 
     // ---- (0) TMA: rows t0..t0+63 of q, k, v (two 64-channel boxes each) and g ----
     if (tid == 0) {
@@ -220,22 +230,25 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tma_load_2d(sb + S::V1, &tm_v, x0 + 64, t0, bar);
         tma_load_2d(sb + S::GR, &tm_g, x0, t0, bar);
     }
+    const bool ptr_ = blockIdx.x == 37 && blockIdx.y == 3 && tid == 0;
+    (void)ptr_;
+    KDA_TRACE_POINT(ptr_, 8192 + 0);
     ok = mbar_wait(bar, phase);
     phase ^= 1;
+    KDA_TRACE_POINT(ptr_, 8192 + 1);
     if (!prep_sync_ok(ok, tid)) goto done;
 
-    // ---- (1) decay: thread = (row block rb of 8 tokens, channel group cg of 8) ----
     {
-        const int cg = tid & 15, rb = tid >> 4;
+        // ---- (1) decay: thread = (block of 4 tokens rb, group of 8 channels cg) ----
+        const int cg = lane & 15, half = lane >> 4, rb = 2 * warp + half;
         const int kb = cg >> 3, c8 = cg & 7;
-        float loc[8][8];
-        float acc[8];
+        float loc[4][8], acc[8], gam[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) acc[u] = 0.f;
         const float* gt = reinterpret_cast<const float*>(sm + S::GR);
 #pragma unroll
-        for (int rr = 0; rr < 8; ++rr) {
-            const int r = 8 * rb + rr;
+        for (int rr = 0; rr < 4; ++rr) {
+            const int r = 4 * rb + rr;
             const float4 g0 = *reinterpret_cast<const float4*>(gt + r * D + 8 * cg);
             const float4 g1 = *reinterpret_cast<const float4*>(gt + r * D + 8 * cg + 4);
             const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
@@ -245,18 +258,23 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 loc[rr][u] = acc[u];
             }
         }
+        float other[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) sX[rb * D + 8 * cg + u] = acc[u];
+        for (int u = 0; u < 8; ++u) other[u] = __shfl_xor_sync(0xffffffffu, acc[u], 16);
+        if (half == 0) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sX[warp * D + 8 * cg + u] = acc[u] + other[u];
+        }
         __syncthreads();
-        float base[8], gam[8];
+        float base[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            float b = 0.f, t = 0.f;
+            float b = half ? other[u] : 0.f, t = 0.f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float x = sX[j * D + 8 * cg + u];
+            for (int w = 0; w < 8; ++w) {
+                const float x = sX[w * D + 8 * cg + u];
                 t += x;
-                if (j < rb) b += x;
+                if (w < warp) b += x;
             }
             base[u] = b;
             gam[u] = __expf(t);
@@ -267,8 +285,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             gdst[1] = make_float4(gam[4], gam[5], gam[6], gam[7]);
         }
 #pragma unroll
-        for (int rr = 0; rr < 8; ++rr) {
-            const int r = 8 * rb + rr;
+        for (int rr = 0; rr < 4; ++rr) {
+            const int r = 4 * rb + rr;
             const uint32_t o = kb * S::BLK + sw128_off(r, c8);
             float qv[8], kv[8], qd[8], kd[8], ki[8];
             unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + o), qv);
@@ -288,6 +306,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         fence_proxy_async_smem();
         __syncthreads();
+        KDA_TRACE_POINT(ptr_, 8192 + 2);
 
         // ---- (2) [K_dec ; Q_dec] K_inv^T -> TMEM [0, 64) ----
         if (tid == 0) {
@@ -306,42 +325,41 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tc_fence_after();
         if (!prep_sync_ok(ok, tid)) goto done;
         {
-            float d0[32], d1[32];
-            const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
-            tmem_ld32(ta, d0);
-            tmem_ld32(ta + 32, d1);
+            float d[32];
+            tmem_ld32(tl + 32 * wh, d);
             tmem_wait_ld();
-            if (warp < 2) {  // L row r = beta_r (K_dec K_inv^T)[r, s], s < r
-                const int r = 32 * warp + lane;
+            if (wq < 2) {   // L[r][s] = beta_r (K_dec K_inv^T)[r][s] for s < r (fp32, pitch 65)
+                const int r = 32 * wq + lane;
                 const float br = sBeta[r];
 #pragma unroll
-                for (int s4 = 0; s4 < C / 4; ++s4) {
+                for (int u4 = 0; u4 < 8; ++u4) {
                     float e[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const int s = 4 * s4 + u;
-                        e[u] = s < r ? br * (s < 32 ? d0[s & 31] : d1[s & 31]) : 0.f;
+                        const int s = 32 * wh + 4 * u4 + u;
+                        e[u] = s < r ? br * d[4 * u4 + u] : 0.f;
                     }
-                    *reinterpret_cast<float4*>(sL + r * C + 4 * s4) = make_float4(e[0], e[1], e[2], e[3]);
+                    *reinterpret_cast<float4*>(sLI + r * kLP + 32 * wh + 4 * u4) =
+                        make_float4(e[0], e[1], e[2], e[3]);
                 }
-            } else {         // Aqk row r = (Q_dec K_inv^T)[r, s], s <= r
-                const int r = 32 * (warp - 2) + lane;
+            } else {        // Aqk[r][s] = (Q_dec K_inv^T)[r][s] for s <= r (bf16 image)
+                const int r = 32 * (wq - 2) + lane;
 #pragma unroll
-                for (int cb = 0; cb < C / 8; ++cb) {
+                for (int qq = 0; qq < 4; ++qq) {
                     float e[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        const int s = 8 * cb + u;
-                        e[u] = s <= r ? (s < 32 ? d0[s & 31] : d1[s & 31]) : 0.f;
+                        const int s = 32 * wh + 8 * qq + u;
+                        e[u] = s <= r ? d[8 * qq + u] : 0.f;
                     }
-                    *reinterpret_cast<uint4*>(sm + S::AQK + sw128_off(r, cb)) = pack_bf16x8(e);
+                    *reinterpret_cast<uint4*>(sm + S::AQK + sw128_off(r, 4 * wh + qq)) = pack_bf16x8(e);
                 }
             }
         }
         // K_res = K_inv gamma, in place (the first MMA has finished reading K_inv)
 #pragma unroll
-        for (int rr = 0; rr < 8; ++rr) {
-            const uint32_t o = S::KI0 + kb * S::BLK + sw128_off(8 * rb + rr, c8);
+        for (int rr = 0; rr < 4; ++rr) {
+            const uint32_t o = S::KI0 + kb * S::BLK + sw128_off(4 * rb + rr, c8);
             float ki[8];
             unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + o), ki);
 #pragma unroll
@@ -352,33 +370,97 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tc_fence_before();
     fence_proxy_async_smem();
     __syncthreads();
+    KDA_TRACE_POINT(ptr_, 8192 + 3);
 
-    // ---- (3) UT transform: INV = (I + L)^{-1}; Abar = INV diag(beta), column j per thread ----
-    if (tid < C) {
-        const int j = tid;
-        float x[C];
+    // ---- (3) UT transform INV = (I + L)^{-1}, in place over L ----
+    // Every entry above the diagonal of the buffer is 0 (L is strictly lower triangular and
+    // the inverse is lower triangular), so the block products below need no masks.
+    {
+        float* sT = sX;
+        // 16x16 diagonal blocks D_b by forward substitution: thread (block b, column j)
+        float x[16];
+        const int b = tid >> 4, j = tid & 15;
+        if (tid < 64) {
 #pragma unroll
-        for (int r = 0; r < C; ++r) {
-            float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+            for (int r = 0; r < 16; ++r) {
+                float acc = (r == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int s4 = 0; s4 < (r + 3) / 4; ++s4) {
-                const float4 l = *reinterpret_cast<const float4*>(sL + r * C + 4 * s4);
-                if (4 * s4 + 0 < r) acc0 -= l.x * x[4 * s4 + 0];
-                if (4 * s4 + 1 < r) acc1 -= l.y * x[4 * s4 + 1];
-                if (4 * s4 + 2 < r) acc2 -= l.z * x[4 * s4 + 2];
-                if (4 * s4 + 3 < r) acc3 -= l.w * x[4 * s4 + 3];
+                for (int s2 = 0; s2 < r; ++s2) acc -= sLI[(16 * b + r) * kLP + 16 * b + s2] * x[s2];
+                x[r] = acc;
             }
-            x[r] = (acc0 + acc1) + (acc2 + acc3);
         }
-        const float bj = sBeta[j];
+        __syncthreads();
+        if (tid < 64) {
 #pragma unroll
-        for (int r = 0; r < C; ++r) x[r] *= bj;
+            for (int r = 0; r < 16; ++r) sLI[(16 * b + r) * kLP + 16 * b + j] = x[r];
+        }
+        __syncthreads();
+        // 16 -> 32, block pairs (0,1) and (2,3): X = -D_hi (L_lo D_lo); 1x4 tiles per thread
+        if (tid < 128) {
+            const int p = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
+            const int R = 16 * (2 * p + 1), Cc = 32 * p;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int cb = 0; cb < C / 8; ++cb)
-            *reinterpret_cast<uint4*>(sm + S::ABAR + sw128_off(j, cb)) = pack_bf16x8(&x[8 * cb]);
+            for (int s2 = 0; s2 < 16; ++s2) {
+                const float l = sLI[(R + r) * kLP + Cc + s2];
+                const float4 dv = *reinterpret_cast<const float4*>(sLI + (Cc + s2) * kLP + Cc + c4);
+                acc.x += l * dv.x; acc.y += l * dv.y; acc.z += l * dv.z; acc.w += l * dv.w;
+            }
+            *reinterpret_cast<float4*>(sT + (16 * p + r) * kTP + c4) = acc;
+        }
+        __syncthreads();
+        if (tid < 128) {
+            const int p = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
+            const int R = 16 * (2 * p + 1), Cc = 32 * p;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int s2 = 0; s2 < 16; ++s2) {
+                const float dh = sLI[(R + r) * kLP + R + s2];
+                const float4 tv = *reinterpret_cast<const float4*>(sT + (16 * p + s2) * kTP + c4);
+                acc.x -= dh * tv.x; acc.y -= dh * tv.y; acc.z -= dh * tv.z; acc.w -= dh * tv.w;
+            }
+            *reinterpret_cast<float4*>(sLI + (R + r) * kLP + Cc + c4) = acc;
+        }
+        __syncthreads();
+        // 32 -> 64: X = -B^{-1} (L[32:64, 0:32] A^{-1}); thread (row r, 4 columns)
+        {
+            const int r = tid >> 3, c4 = 4 * (tid & 7);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+            for (int s2 = 0; s2 < 32; ++s2) {
+                const float l = sLI[(32 + r) * kLP + s2];
+                const float4 av = *reinterpret_cast<const float4*>(sLI + s2 * kLP + c4);
+                acc.x += l * av.x; acc.y += l * av.y; acc.z += l * av.z; acc.w += l * av.w;
+            }
+            *reinterpret_cast<float4*>(sT + r * kTP + c4) = acc;
+            __syncthreads();
+            float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+            for (int s2 = 0; s2 < 32; ++s2) {
+                const float bi = sLI[(32 + r) * kLP + 32 + s2];
+                const float4 tv = *reinterpret_cast<const float4*>(sT + s2 * kTP + c4);
+                xo.x -= bi * tv.x; xo.y -= bi * tv.y; xo.z -= bi * tv.z; xo.w -= bi * tv.w;
+            }
+            *reinterpret_cast<float4*>(sLI + (32 + r) * kLP + c4) = xo;
+        }
+        __syncthreads();
+        // Abar = INV diag(beta) as MN-major A image: row s = beta_s * column s of INV
+        {
+            const int jj = tid >> 2;
+            const float bj = sBeta[jj];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int chnk = 2 * (tid & 3) + h2;
+                float e[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) e[u] = bj * sLI[(8 * chnk + u) * kLP + jj];
+                *reinterpret_cast<uint4*>(sm + S::ABAR + sw128_off(jj, chnk)) = pack_bf16x8(e);
+            }
+        }
     }
     fence_proxy_async_smem();
     __syncthreads();
+    KDA_TRACE_POINT(ptr_, 8192 + 4);
 
     // ---- (4) [W | U] = Abar [K_dec | V] -> TMEM [0, 256) (lanes 0-63 meaningful) ----
     if (tid == 0) {
@@ -394,24 +476,25 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     phase ^= 1;
     tc_fence_after();
     if (!prep_sync_ok(ok, tid)) goto done;
-    if (warp < 2) {  // W, U rows r -> bf16 B image in place of K_dec, V (MN-major, rows r)
-        const int r = tid;
-        const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
+    if (wq < 2) {  // rows r of W (column half 0) / U (column half 1) -> bf16 B image in place
+        const int r = 32 * wq + lane;
 #pragma unroll
-        for (int cb = 0; cb < 8; ++cb) {
+        for (int cb = 0; cb < 4; ++cb) {
             float d[32];
-            tmem_ld32(ta + 32 * cb, d);
+            const int col = 128 * wh + 32 * cb;
+            tmem_ld32(tl + col, d);
             tmem_wait_ld();
-            const uint32_t blk = S::KD0 + (cb >> 1) * S::BLK;
+            const uint32_t blk = S::KD0 + (col >> 6) * S::BLK;
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq)
-                *reinterpret_cast<uint4*>(sm + blk + sw128_off(r, (cb & 1) * 4 + qq)) =
+                *reinterpret_cast<uint4*>(sm + blk + sw128_off(r, ((col & 63) >> 3) + qq)) =
                     pack_bf16x8(&d[8 * qq]);
         }
     }
     tc_fence_before();
     fence_proxy_async_smem();
     __syncthreads();
+    KDA_TRACE_POINT(ptr_, 8192 + 5);
 
     // ---- (5) [-M | B] = K_res^T [W | U] -> TMEM [0, 256) ----
     if (tid == 0) {
@@ -428,29 +511,32 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tc_fence_after();
     if (!prep_sync_ok(ok, tid)) goto done;
     {
-        const int i = tid;  // TMEM lane = key channel
-        const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
+        const int i = 32 * wq + lane;  // TMEM lane = key channel
 #pragma unroll
-        for (int cb = 0; cb < 8; ++cb) {
+        for (int cb = 0; cb < 4; ++cb) {
             float d[32];
-            tmem_ld32(ta + 32 * cb, d);
+            const int col = 128 * wh + 32 * cb;
+            tmem_ld32(tl + col, d);
             tmem_wait_ld();
-            if (cb < 4) {   // M = -K_res^T W, K-major rows i
+            if (wh == 0) {   // M = -K_res^T W: K-major rows i, K blocks of 64 channels
 #pragma unroll
                 for (int u = 0; u < 32; ++u) d[u] = -d[u];
-                uint8_t* mdst = rec + kRecM0 + (cb >> 1) * kRecKB;
+                uint8_t* mdst = rec + kRecM0 + (col >> 6) * 16384;
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq)
-                    *reinterpret_cast<uint4*>(mdst + sw128_off(i, (cb & 1) * 4 + qq)) = pack_bf16x8(&d[8 * qq]);
-            } else {        // B = K_res^T U, value-channel slice cb-4
-                uint4* bdst = reinterpret_cast<uint4*>(rec + kRecB + (cb - 4) * 8192 + i * 64);
+                    *reinterpret_cast<uint4*>(mdst + sw128_off(i, ((col & 63) >> 3) + qq)) = pack_bf16x8(&d[8 * qq]);
+            } else {         // B = K_res^T U: value-channel slice (col-128)/64, rows i swizzled
+                const int j0 = col - 128;
+                uint8_t* bdst = rec + kRecB + (j0 >> 6) * 16384;
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) bdst[qq] = pack_bf16x8(&d[8 * qq]);
+                for (int qq = 0; qq < 4; ++qq)
+                    *reinterpret_cast<uint4*>(bdst + sw128_off(i, ((j0 & 63) >> 3) + qq)) = pack_bf16x8(&d[8 * qq]);
             }
         }
     }
     tc_fence_before();
     __syncthreads();
+    KDA_TRACE_POINT(ptr_, 8192 + 6);
 
     // ---- (6) [Aqk W | Aqk U] -> TMEM [0, 256) (lanes 0-63); P = Q_dec - Aqk W, R = Aqk U ----
     if (tid == 0) {
@@ -466,20 +552,20 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     phase ^= 1;
     tc_fence_after();
     if (!prep_sync_ok(ok, tid)) goto done;
-    if (warp < 2) {
-        const int r = tid;
-        const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
+    if (wq < 2) {
+        const int r = 32 * wq + lane;
 #pragma unroll
-        for (int cb = 0; cb < 8; ++cb) {
+        for (int cb = 0; cb < 4; ++cb) {
             float d[32];
-            tmem_ld32(ta + 32 * cb, d);
+            const int col = 128 * wh + 32 * cb;
+            tmem_ld32(tl + col, d);
             tmem_wait_ld();
-            if (cb < 4) {
-                const int kb = cb >> 1;
-                uint8_t* pdst = rec + kRecP0 + kb * kRecKB;
+            if (wh == 0) {
+                const int kb = col >> 6;
+                uint8_t* pdst = rec + kRecP0 + kb * 8192;
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
-                    const int ch = (cb & 1) * 4 + qq;
+                    const int ch = ((col & 63) >> 3) + qq;
                     float qv[8];
                     unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + kb * S::BLK + sw128_off(r, ch)), qv);
 #pragma unroll
@@ -487,15 +573,18 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     *reinterpret_cast<uint4*>(pdst + sw128_off(r, ch)) = pack_bf16x8(qv);
                 }
             } else {
-                uint4* rdst = reinterpret_cast<uint4*>(rec + kRecR + (cb - 4) * 4096 + r * 64);
+                const int j0 = col - 128;
+                uint8_t* rdst = rec + kRecR + (j0 >> 6) * 8192;
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) rdst[qq] = pack_bf16x8(&d[8 * qq]);
+                for (int qq = 0; qq < 4; ++qq)
+                    *reinterpret_cast<uint4*>(rdst + sw128_off(r, ((j0 & 63) >> 3) + qq)) = pack_bf16x8(&d[8 * qq]);
             }
         }
     }
 done:
     tc_fence_before();
     __syncthreads();
+    KDA_TRACE_POINT(ptr_, 8192 + 7);
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, kPrepTmemCols);
@@ -503,27 +592,26 @@ done:
 }
 
 // ------------------------------------------------------------------ chunk recurrence
-constexpr int kRecThreads = 160;      // warps 0-3: state rows / TMEM lanes; warp 4: loader
+constexpr int kRecThreads = 192;      // warps 0-3: state rows / TMEM lanes; 4: loader; 5: MMA issuer
 constexpr int kStages = 3;
-constexpr uint32_t kStA = 0;          // [P0 | M0 | P1 | M1]  48 KB
-constexpr uint32_t kStB = 49152;      // B slice [128][32] bf16
-constexpr uint32_t kStR = 57344;      // R slice [64][32] bf16
-constexpr uint32_t kStG = 61440;      // gamma [128]
-constexpr uint32_t kStageLoad = 61952;
-constexpr uint32_t kStageBytes = 62464;
+constexpr uint32_t kStM = 0;          // M, both K blocks (32 KB)
+constexpr uint32_t kStB = 32768;      // B slice [128][64] bf16 (rows swizzled)
+constexpr uint32_t kStG = 49152;      // gamma [128]
+constexpr uint32_t kStageLoad = 49664;
+constexpr uint32_t kStageBytes = 50176;
 struct RecSmem {
-    static constexpr uint32_t SB = kStages * kStageBytes;   // S (bf16) B images, 2 x 8 KB
-    static constexpr uint32_t BAR = SB + 2 * 8192;          // full[3] empty[3] mma_s mma_o[2]
+    static constexpr uint32_t SB = kStages * kStageBytes;   // S (bf16) B images, 2 x 16 KB
+    static constexpr uint32_t BAR = SB + 2 * 16384;         // full[3] empty[3] mma_s sb_ready[2]
     static constexpr uint32_t TMEM = BAR + 9 * 8;
     static constexpr uint32_t FLAG = TMEM + 4;
     static constexpr uint32_t BYTES = FLAG + 4 + 1024;
 };
-constexpr uint32_t kRecTmemCols = 128;  // D_S [0,32), D_O[0] [32,64), D_O[1] [64,96)
+constexpr uint32_t kRecTmemCols = 64;   // D_S
 
 __global__ void __launch_bounds__(kRecThreads, 1)
 rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* __restrict__ off,
-           const uint8_t* __restrict__ records, const float* initial_state, float* final_state,
-           __nv_bfloat16* __restrict__ out) {
+           const uint8_t* __restrict__ records, uint8_t* __restrict__ states,
+           const float* initial_state, float* final_state) {
     using S = RecSmem;
     const int sl = blockIdx.x % NSL;
     const int h = (blockIdx.x / NSL) % H;
@@ -533,59 +621,89 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     const uint32_t sb = smem_u32(sm);
-    // mma_o[b] tracks the output product of the chunks with kk % 2 == b, so a waiter can
-    // never fall two phases behind (the next use of the same barrier is after a CTA sync).
-    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 24, mma_s = full0 + 48, mma_o0 = full0 + 56;
+    // Each barrier's waiters can never fall two phases behind: its next phase needs an
+    // arrival that every waiter of the current phase precedes.
+    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 24, mma_s = full0 + 48, sbr0 = full0 + 56;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + S::FLAG);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (warp == 0) tmem_alloc(sb + S::TMEM, kRecTmemCols);
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(full0 + 8 * s, 1);
-            mbar_init(empty0 + 8 * s, 1);
+        for (int st = 0; st < kStages; ++st) {
+            mbar_init(full0 + 8 * st, 1);
+            mbar_init(empty0 + 8 * st, 4);
         }
         mbar_init(mma_s, 1);
-        mbar_init(mma_o0, 1);
-        mbar_init(mma_o0 + 8, 1);
+        mbar_init(sbr0, 4);
+        mbar_init(sbr0 + 8, 4);
         fence_mbar_init();
         *abort_flag = 0;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
-    const uint32_t tS = tmem, tO = tmem + 32;
+    const uint32_t tS = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
 
     if (warp == 4) {
-        // ---------------- loader ----------------------------------------------------------
+        // ---------------- loader: M, this slice of B, gamma of every chunk -----------------
         if (lane == 0) {
             int issued = 0;
-            for (int kk = 0; kk < nchunks; ++kk) {
+            for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
                 const int st = kk % kStages, use = kk / kStages;
+                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 0);
                 if (use > 0 && !mbar_wait(empty0 + 8 * st, (use - 1) & 1)) {
                     kda_set_status(KDA_ERR_TIMEOUT);
                     *abort_flag = 1;
                     break;
                 }
-                if (*abort_flag) break;
                 const uint8_t* rec = records + ((size_t)(c_begin + kk) * H + h) * kRecBytes;
                 const uint32_t dst = sb + st * kStageBytes;
                 const uint32_t fb = full0 + 8 * st;
                 mbar_arrive_expect_tx(fb, kStageLoad);
-                bulk_g2s(dst + kStA, rec, 24576, fb);
-                bulk_g2s(dst + kStA + 24576, rec + 24576, 24576, fb);
-                bulk_g2s(dst + kStB, rec + kRecB + sl * 8192, 8192, fb);
-                bulk_g2s(dst + kStR, rec + kRecR + sl * 4096, 4096, fb);
+                bulk_g2s(dst + kStM, rec + kRecM0, 16384, fb);
+                bulk_g2s(dst + kStM + 16384, rec + kRecM0 + 16384, 16384, fb);
+                bulk_g2s(dst + kStB, rec + kRecB + sl * 16384, 16384, fb);
                 bulk_g2s(dst + kStG, rec + kRecGamma, 512, fb);
+                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 1);
                 ++issued;
             }
             // never leave with copies in flight: wait (bounded) for the last stages filled
             for (int kk = max(0, issued - kStages); kk < issued; ++kk)
                 mbar_wait(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
         }
+    } else if (warp == 5) {
+        // ---------------- MMA issuer: D_S = M S_in once the stage and S_in are ready --------
+        if (lane == 0) {
+            constexpr uint32_t id = idesc_bf16(128, NV, false, true);
+            for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
+                const int st = kk % kStages;
+                if (!mbar_wait(full0 + 8 * st, (kk / kStages) & 1) ||
+                    !mbar_wait(sbr0 + 8 * (kk & 1), (kk >> 1) & 1)) {
+                    kda_set_status(KDA_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t stage = sb + st * kStageBytes;
+                const uint32_t sbuf = sb + S::SB + (kk & 1) * 16384;
+                // the other S buffer is rewritten after this chunk's product completes: its
+                // copy to the workspace (issued one chunk ago) must have read it by then
+                bulk_wait_read<0>();
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t ko = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    umma_bf16(tS, smem_desc(stage + kStM + ko, 16, 1024, kSwizzle128),
+                              smem_desc(sbuf + ks * 2048, 16, 1024, kSwizzle128), id, ks > 0);
+                }
+                umma_commit(mma_s);
+                // the state entering chunk kk, for the output kernel
+                bulk_s2g(states + ((size_t)(c_begin + kk) * H + h) * kStateImgBytes + sl * 16384,
+                         sbuf, 16384);
+            }
+            bulk_wait_all();
+        }
     } else {
-        // ---------------- state rows i = tid ------------------------------------------------
+        // ---------------- state rows i = tid (warps 0-3) ------------------------------------
         const int i = tid;
         const uint32_t taw = (uint32_t)(32 * warp) << 16;
         const size_t sbase = (((size_t)n * H + h) * D + i) * D + (size_t)sl * NV;
@@ -600,107 +718,66 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
 #pragma unroll
             for (int j = 0; j < NV; ++j) Sr[j] = 0.f;
         }
+        // bf16 image of the state entering the next chunk (B operand of its product; the
+        // issuer also copies it to the workspace for the output kernel)
+        auto put_state = [&](uint32_t buf) {
 #pragma unroll
-        for (int cb = 0; cb < NV / 8; ++cb)
-            *reinterpret_cast<uint4*>(sm + S::SB + sw64_off(i, cb)) = pack_bf16x8(&Sr[8 * cb]);
-        fence_proxy_async_smem();
-        named_bar(1, 128);
-
-        const int t_seq = nchunks > 0 ? cu[n] : 0;
-        const int t_end = nchunks > 0 ? cu[n + 1] : 0;
-        bool ok = true;
-        // Output of chunk kk-1 (O = D_O + R): warps 0-1 (TMEM lanes = token rows).
-        auto emit_output = [&](int kk) {
-            if (warp < 2 && ok) {
-                ok = __all_sync(0xffffffffu, mbar_wait(mma_o0 + 8 * (kk & 1), (kk >> 1) & 1));
-                tc_fence_after();
-                if (!ok) return;
-                float ov[32];
-                tmem_ld32(tO + 32 * (kk & 1) + taw, ov);
-                tmem_wait_ld();
-                const int r = i;
-                const int t0 = t_seq + kk * C;
-                if (r < min(C, t_end - t0)) {
-                    const uint8_t* st_p = sm + (kk % kStages) * kStageBytes;
-                    const uint4* rs = reinterpret_cast<const uint4*>(st_p + kStR + r * 64);
-                    uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * H + h) * D + sl * NV);
-#pragma unroll
-                    for (int cb = 0; cb < 4; ++cb) {
-                        float rv[8];
-                        unpack_bf16x8(rs[cb], rv);
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) rv[u] += ov[8 * cb + u];
-                        dst[cb] = pack_bf16x8(rv);
-                    }
-                }
-            }
+            for (int cb = 0; cb < NV / 8; ++cb)
+                *reinterpret_cast<uint4*>(sm + buf + sw128_off(i, cb)) = pack_bf16x8(&Sr[8 * cb]);
         };
+        if (nchunks > 0) put_state(S::SB);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sbr0);
+
+        bool ok = true;
         for (int kk = 0; kk < nchunks; ++kk) {
             const int st = kk % kStages;
-            const uint32_t stage = sb + st * kStageBytes;
             const uint8_t* stage_p = sm + st * kStageBytes;
-            const uint32_t sbuf = sb + S::SB + (kk & 1) * 8192;
-            ok = __all_sync(0xffffffffu, ok && mbar_wait(full0 + 8 * st, (kk / kStages) & 1));
-            if (!ok) *abort_flag = 1;
-            if (tid == 0 && ok) {
-                tc_fence_after();
-                constexpr uint32_t id = idesc_bf16(128, NV, false, true);
-                // D_S = M S_in (the serial product), then D_O = [P ; *] S_in
+            const bool tr = blockIdx.x == 0 && tid == 0 && kk < 256;
+            (void)tr;
+            KDA_TRACE_POINT(tr, kk * 8 + 0);
+            ok = __all_sync(0xffffffffu, mbar_wait(full0 + 8 * st, (kk / kStages) & 1));
+            if (!ok || *abort_flag) { ok = false; break; }
+            KDA_TRACE_POINT(tr, kk * 8 + 1);
+            // this chunk's gamma and B row, before the serial product lands
+            const float gam = reinterpret_cast<const float*>(stage_p + kStG)[i];
+            uint4 bq[NV / 8];
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t ko = (ks >> 2) * kRecKB + (ks & 3) * 32;
-                    umma_bf16(tS, smem_desc(stage + kRecM0 + ko, 16, 1024, kSwizzle128),
-                              smem_desc(sbuf + ks * 1024, 16, 512, kSwizzle64), id, ks > 0);
-                }
-                umma_commit(mma_s);
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t ko = (ks >> 2) * kRecKB + (ks & 3) * 32;
-                    umma_bf16(tO + 32 * (kk & 1), smem_desc(stage + kRecP0 + ko, 16, 1024, kSwizzle128),
-                              smem_desc(sbuf + ks * 1024, 16, 512, kSwizzle64), id, ks > 0);
-                }
-                umma_commit(mma_o0 + 8 * (kk & 1));
-            }
-            // previous chunk's output overlaps this chunk's serial product
-            if (kk > 0) emit_output(kk - 1);
-            ok = __all_sync(0xffffffffu, ok && mbar_wait(mma_s, kk & 1));
-            if (!ok) *abort_flag = 1;
+            for (int cb = 0; cb < NV / 8; ++cb)
+                bq[cb] = *reinterpret_cast<const uint4*>(stage_p + kStB + sw128_off(i, cb));
+            KDA_TRACE_POINT(tr, kk * 8 + 2);
+            ok = __all_sync(0xffffffffu, mbar_wait(mma_s, kk & 1));
+            if (!ok) break;
+            KDA_TRACE_POINT(tr, kk * 8 + 3);
             tc_fence_after();
-            if (ok) {
-                float dsv[32];
-                tmem_ld32(tS + taw, dsv);
-                tmem_wait_ld();
-                const float gam = reinterpret_cast<const float*>(stage_p + kStG)[i];
-                const uint4* bs = reinterpret_cast<const uint4*>(stage_p + kStB + i * 64);
+            float dsv[NV];
+            tmem_ld32(tS + taw, *reinterpret_cast<float(*)[32]>(&dsv[0]));
+            tmem_ld32(tS + taw + 32, *reinterpret_cast<float(*)[32]>(&dsv[32]));
+            tmem_wait_ld();
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    float bv[8];
-                    unpack_bf16x8(bs[cb], bv);
+            for (int cb = 0; cb < NV / 8; ++cb) {
+                float bv[8];
+                unpack_bf16x8(bq[cb], bv);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int j = 8 * cb + u;
-                        Sr[j] = fmaf(gam, Sr[j], dsv[j] + bv[u]);
-                    }
+                for (int u = 0; u < 8; ++u) {
+                    const int j = 8 * cb + u;
+                    Sr[j] = fmaf(gam, Sr[j], dsv[j] + bv[u]);
                 }
-                // the other S buffer was last read by chunk kk-1's products: both completed
-                // (mma_s waited above in chunk kk-1, mma_o waited by emit_output / below)
-                if (warp >= 2 && kk > 0)
-                    ok = __all_sync(0xffffffffu, mbar_wait(mma_o0 + 8 * ((kk - 1) & 1), ((kk - 1) >> 1) & 1));
-                if (!ok) *abort_flag = 1;
-                const uint32_t nb = S::SB + ((kk + 1) & 1) * 8192;
-#pragma unroll
-                for (int cb = 0; cb < NV / 8; ++cb)
-                    *reinterpret_cast<uint4*>(sm + nb + sw64_off(i, cb)) = pack_bf16x8(&Sr[8 * cb]);
             }
+            KDA_TRACE_POINT(tr, kk * 8 + 4);
+            if (kk + 1 < nchunks) put_state(S::SB + ((kk + 1) & 1) * 16384);
             tc_fence_before();
             fence_proxy_async_smem();
-            named_bar(1, 128);
-            if (tid == 0 && kk > 0) mbar_arrive(empty0 + 8 * ((kk - 1) % kStages));
-            if (*abort_flag) { ok = false; break; }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(sbr0 + 8 * ((kk + 1) & 1));
+                mbar_arrive(empty0 + 8 * st);
+            }
+            KDA_TRACE_POINT(tr, kk * 8 + 5);
         }
-        if (ok && nchunks > 0) emit_output(nchunks - 1);
-        if (!ok || *abort_flag) {
-            if (tid == 0) kda_set_status(KDA_ERR_TIMEOUT);
+        if (!ok) {
+            if (lane == 0) kda_set_status(KDA_ERR_TIMEOUT);
             *abort_flag = 1;
         } else if (final_state) {
 #pragma unroll
@@ -713,7 +790,99 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kRecTmemCols);
+        tmem_dealloc(tS, kRecTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ chunk outputs
+// One CTA per (chunk, head), fully parallel: O = [P ; *] S_in + R from the record and the
+// state image the recurrence left for this chunk.
+constexpr int kOutThreads = 128;
+struct OutSmem {
+    static constexpr uint32_t A = 0;         // P0 | P1 | 8 KB of filler rows (never read back)
+    static constexpr uint32_t SI = 24576;    // state image, 2 slices (32 KB)
+    static constexpr uint32_t RR = 57344;    // R, 2 slices (16 KB)
+    static constexpr uint32_t BAR = 73728;
+    static constexpr uint32_t TMEM = BAR + 8;
+    static constexpr uint32_t BYTES = TMEM + 8 + 1024;
+};
+constexpr uint32_t kOutTmemCols = 128;
+constexpr uint32_t kOutTx = 16384 + kStateImgBytes + 16384;
+
+__global__ void __launch_bounds__(kOutThreads)
+out_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* __restrict__ off,
+           const uint8_t* __restrict__ records, const uint8_t* __restrict__ states,
+           __nv_bfloat16* __restrict__ out) {
+    using S = OutSmem;
+    const int c = blockIdx.x, h = blockIdx.y;
+    const int total_chunks = off[num_seqs];
+    if (c >= total_chunks) return;
+    const int n = find_seq(off, num_seqs, c);
+    const int t0 = cu[n] + (c - off[n]) * C;
+    const int nrow = min(C, cu[n + 1] - t0);
+    const uint8_t* rec = records + ((size_t)c * H + h) * kRecBytes;
+    const uint8_t* simg = states + ((size_t)c * H + h) * kStateImgBytes;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+    const uint32_t sb = smem_u32(sm);
+    const uint32_t bar = sb + S::BAR;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (warp == 0) tmem_alloc(sb + S::TMEM, kOutTmemCols);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(bar, kOutTx);
+        bulk_g2s(sb + S::A, rec + kRecP0, 16384, bar);
+        bulk_g2s(sb + S::SI, simg, kStateImgBytes, bar);
+        bulk_g2s(sb + S::RR, rec + kRecR, 16384, bar);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
+    bool ok = mbar_wait(bar, 0);
+    if (tid == 0 && ok) {
+        constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+            umma_bf16(tmem, smem_desc(sb + S::A + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128),
+                      smem_desc(sb + S::SI + ks * 2048, 16384, 1024, kSwizzle128), id, ks > 0);
+        umma_commit(bar);
+    }
+    ok = ok && mbar_wait(bar, 1);
+    tc_fence_after();
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) kda_set_status(KDA_ERR_TIMEOUT);
+    } else if (warp < 2) {
+        const int r = tid;
+        const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+            float d[32];
+            tmem_ld32(ta + 32 * cb, d);
+            tmem_wait_ld();
+            if (r < nrow) {
+                const int slc = cb >> 1;
+                uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * H + h) * D + 32 * cb);
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    float rv[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4*>(
+                                      sm + S::RR + slc * 8192 + sw128_off(r, (cb & 1) * 4 + qq)), rv);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) rv[u] += d[8 * qq + u];
+                    dst[qq] = pack_bf16x8(rv);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kOutTmemCols);
     }
 }
 
@@ -756,11 +925,15 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
                                   void* workspace, cudaStream_t stream) {
     int32_t* off = static_cast<int32_t*>(workspace);
     uint8_t* records = static_cast<uint8_t*>(workspace) + ws_records_offset(num_seqs);
+    uint8_t* states = static_cast<uint8_t*>(workspace) + ws_states_offset(total, num_seqs, H);
     cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepSmem::BYTES);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(rec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)RecSmem::BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)OutSmem::BYTES);
     if (e != cudaSuccess) return e;
     chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, off);
     const int64_t mc = max_chunks(total, num_seqs);
@@ -776,7 +949,12 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
                                                                      num_seqs, H, off, records);
     }
     rec_kernel<<<(unsigned)num_seqs * H * NSL, kRecThreads, RecSmem::BYTES, stream>>>(
-        cu, num_seqs, H, off, records, s0, sf, static_cast<__nv_bfloat16*>(out));
+        cu, num_seqs, H, off, records, states, s0, sf);
+    if (total > 0) {
+        dim3 grid((unsigned)mc, (unsigned)H);
+        out_kernel<<<grid, kOutThreads, OutSmem::BYTES, stream>>>(
+            cu, num_seqs, H, off, records, states, static_cast<__nv_bfloat16*>(out));
+    }
     return cudaGetLastError();
 }
 

@@ -128,6 +128,14 @@ kda_status kda_decode(const void* q, const void* k, const void* v, const float* 
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+#ifdef KDA_TRACE
+// Trace builds only: copy the first n clock stamps to host memory.
+int kda_debug_read_trace(unsigned long long* host, int n) {
+    if (n > kTraceSlots) n = kTraceSlots;
+    return cudaMemcpyFromSymbol(host, g_kda_trace, sizeof(unsigned long long) * n) == cudaSuccess ? n : -1;
+}
+#endif
+
 kda_status kda_get_device_status(kda_stream_t stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) return KDA_ERR_CUDA;

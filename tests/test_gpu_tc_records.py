@@ -13,7 +13,6 @@ from tests.gpu_helpers import to_device
 pytestmark = pytest.mark.gpu
 
 REC_BYTES = 98816
-KB = 24576
 
 
 def _bf16(u8: np.ndarray) -> np.ndarray:
@@ -54,12 +53,12 @@ def test_prep_record_matches_chunked_oracle(nrow):
     B_ref = T["K_res"].T @ T["U"]
     P_ref = T["Q_dec"] - T["Aqk"] @ T["W"]
     R_ref = T["Aqk"] @ T["U"]
-    P = np.concatenate([_sw128(rec[kb * KB:kb * KB + 8192], 64) for kb in range(2)], axis=1)
-    M = np.concatenate([_sw128(rec[8192 + kb * KB:8192 + kb * KB + 16384], 128) for kb in range(2)], axis=1)
-    B = np.concatenate([_bf16(rec[49152 + s * 8192:49152 + (s + 1) * 8192].reshape(128, 64))
-                        for s in range(4)], axis=1)
-    R = np.concatenate([_bf16(rec[81920 + s * 4096:81920 + (s + 1) * 4096].reshape(64, 64))
-                        for s in range(4)], axis=1)
+    P = np.concatenate([_sw128(rec[kb * 8192:(kb + 1) * 8192], 64) for kb in range(2)], axis=1)
+    M = np.concatenate([_sw128(rec[16384 + kb * 16384:16384 + (kb + 1) * 16384], 128) for kb in range(2)], axis=1)
+    B = np.concatenate([_sw128(rec[49152 + s * 16384:49152 + (s + 1) * 16384], 128)
+                        for s in range(2)], axis=1)
+    R = np.concatenate([_sw128(rec[81920 + s * 8192:81920 + (s + 1) * 8192], 64)
+                        for s in range(2)], axis=1)
     gam = rec[98304:98816].copy().view(np.float32).astype(np.float64)
 
     def rel(a, b):
