@@ -180,6 +180,13 @@ __device__ __forceinline__ bool prep_sync_ok(bool ok, int tid) {
     return true;
 }
 
+// 4 KB staging slot of warp w for the record drains; all of them lie in operand space that
+// is dead by then (K_res after its product, the Abar image, the L / INV buffer).
+__device__ __forceinline__ uint32_t stage_slot(int w) {
+    const uint32_t base = w < 2 ? PrepSmem::KI0 : w < 4 ? PrepSmem::KI1 : w < 6 ? PrepSmem::ABAR : PrepSmem::LI;
+    return base + (w & 1) * 4096;
+}
+
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -511,27 +518,32 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tc_fence_after();
     if (!prep_sync_ok(ok, tid)) goto done;
     {
-        const int i = 32 * wq + lane;  // TMEM lane = key channel
+        // Drain: each warp turns its 32 TMEM lanes x 128 columns into two 4 KB pieces of the
+        // record (32 complete swizzled rows each) staged in a private, now unused 4 KB slot,
+        // and copies each piece out with one bulk copy.
+        //   column half 0 -> M = -K_res^T W rows i, K block 0 / 1
+        //   column half 1 -> B = K_res^T U rows i, value slice 0 / 1
+        uint8_t* slot = sm + stage_slot(warp);
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            float d[32];
-            const int col = 128 * wh + 32 * cb;
-            tmem_ld32(tl + col, d);
+        for (int pc = 0; pc < 2; ++pc) {
+            const uint32_t col0 = 128 * wh + 64 * pc;
+            float d[64];
+            tmem_ld32(tl + col0, *reinterpret_cast<float(*)[32]>(&d[0]));
+            tmem_ld32(tl + col0 + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
             tmem_wait_ld();
-            if (wh == 0) {   // M = -K_res^T W: K-major rows i, K blocks of 64 channels
+            if (wh == 0) {
 #pragma unroll
-                for (int u = 0; u < 32; ++u) d[u] = -d[u];
-                uint8_t* mdst = rec + kRecM0 + (col >> 6) * 16384;
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq)
-                    *reinterpret_cast<uint4*>(mdst + sw128_off(i, ((col & 63) >> 3) + qq)) = pack_bf16x8(&d[8 * qq]);
-            } else {         // B = K_res^T U: value-channel slice (col-128)/64, rows i swizzled
-                const int j0 = col - 128;
-                uint8_t* bdst = rec + kRecB + (j0 >> 6) * 16384;
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq)
-                    *reinterpret_cast<uint4*>(bdst + sw128_off(i, ((j0 & 63) >> 3) + qq)) = pack_bf16x8(&d[8 * qq]);
+                for (int u = 0; u < 64; ++u) d[u] = -d[u];
             }
+            if (pc == 1 && lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+#pragma unroll
+            for (int cb = 0; cb < 8; ++cb)
+                *reinterpret_cast<uint4*>(slot + sw128_off(lane, cb)) = pack_bf16x8(&d[8 * cb]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                bulk_s2g(rec + (wh == 0 ? kRecM0 : kRecB) + pc * 16384 + wq * 4096, smem_u32(slot), 4096);
         }
     }
     tc_fence_before();
@@ -553,35 +565,39 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tc_fence_after();
     if (!prep_sync_ok(ok, tid)) goto done;
     if (wq < 2) {
+        //   column half 0 -> P = Q_dec - Aqk W rows r, K block 0 / 1
+        //   column half 1 -> R = Aqk U rows r, value slice 0 / 1
         const int r = 32 * wq + lane;
+        uint8_t* slot = sm + stage_slot(warp);
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            float d[32];
-            const int col = 128 * wh + 32 * cb;
-            tmem_ld32(tl + col, d);
+        for (int pc = 0; pc < 2; ++pc) {
+            const uint32_t col0 = 128 * wh + 64 * pc;
+            float d[64];
+            tmem_ld32(tl + col0, *reinterpret_cast<float(*)[32]>(&d[0]));
+            tmem_ld32(tl + col0 + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
             tmem_wait_ld();
             if (wh == 0) {
-                const int kb = col >> 6;
-                uint8_t* pdst = rec + kRecP0 + kb * 8192;
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int ch = ((col & 63) >> 3) + qq;
+                for (int cb = 0; cb < 8; ++cb) {
                     float qv[8];
-                    unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + kb * S::BLK + sw128_off(r, ch)), qv);
+                    unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + pc * S::BLK + sw128_off(r, cb)), qv);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) qv[u] -= d[8 * qq + u];
-                    *reinterpret_cast<uint4*>(pdst + sw128_off(r, ch)) = pack_bf16x8(qv);
+                    for (int u = 0; u < 8; ++u) d[8 * cb + u] = qv[u] - d[8 * cb + u];
                 }
-            } else {
-                const int j0 = col - 128;
-                uint8_t* rdst = rec + kRecR + (j0 >> 6) * 8192;
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq)
-                    *reinterpret_cast<uint4*>(rdst + sw128_off(r, ((j0 & 63) >> 3) + qq)) = pack_bf16x8(&d[8 * qq]);
             }
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+#pragma unroll
+            for (int cb = 0; cb < 8; ++cb)
+                *reinterpret_cast<uint4*>(slot + sw128_off(lane, cb)) = pack_bf16x8(&d[8 * cb]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                bulk_s2g(rec + (wh == 0 ? kRecP0 : kRecR) + pc * 8192 + wq * 4096, smem_u32(slot), 4096);
         }
     }
 done:
+    if (lane == 0) bulk_wait_all();   // no copy may still read shared memory at exit
     tc_fence_before();
     __syncthreads();
     KDA_TRACE_POINT(ptr_, 8192 + 7);
