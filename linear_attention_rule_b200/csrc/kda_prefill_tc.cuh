@@ -272,20 +272,29 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
             for (int u = 0; u < 8; ++u) sX[warp * D + 8 * cg + u] = acc[u] + other[u];
         }
+        KDA_TRACE_POINT(ptr_, 8192 + 20);
         __syncthreads();
-        float base[8];
+        KDA_TRACE_POINT(ptr_, 8192 + 21);
+        float base[8], tot[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            float b = half ? other[u] : 0.f, t = 0.f;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                const float x = sX[w * D + 8 * cg + u];
-                t += x;
-                if (w < warp) b += x;
-            }
-            base[u] = b;
-            gam[u] = __expf(t);
+            base[u] = half ? other[u] : 0.f;
+            tot[u] = 0.f;
         }
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            const float4 x0 = *reinterpret_cast<const float4*>(sX + w * D + 8 * cg);
+            const float4 x1 = *reinterpret_cast<const float4*>(sX + w * D + 8 * cg + 4);
+            const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                tot[u] += xv[u];
+                if (w < warp) base[u] += xv[u];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) gam[u] = __expf(tot[u]);
+        KDA_TRACE_POINT(ptr_, 8192 + 22);
         if (rb == 0) {
             float4* gdst = reinterpret_cast<float4*>(rec + kRecGamma + 32 * cg);
             gdst[0] = make_float4(gam[0], gam[1], gam[2], gam[3]);
@@ -397,11 +406,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         }
         __syncthreads();
+        KDA_TRACE_POINT(ptr_, 8192 + 16);
         if (tid < 64) {
 #pragma unroll
             for (int r = 0; r < 16; ++r) sLI[(16 * b + r) * kLP + 16 * b + j] = x[r];
         }
         __syncthreads();
+        KDA_TRACE_POINT(ptr_, 8192 + 17);
         // 16 -> 32, block pairs (0,1) and (2,3): X = -D_hi (L_lo D_lo); 1x4 tiles per thread
         if (tid < 128) {
             const int p = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
@@ -429,6 +440,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             *reinterpret_cast<float4*>(sLI + (R + r) * kLP + Cc + c4) = acc;
         }
         __syncthreads();
+        KDA_TRACE_POINT(ptr_, 8192 + 18);
         // 32 -> 64: X = -B^{-1} (L[32:64, 0:32] A^{-1}); thread (row r, 4 columns)
         {
             const int r = tid >> 3, c4 = 4 * (tid & 7);
@@ -451,6 +463,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             *reinterpret_cast<float4*>(sLI + (32 + r) * kLP + c4) = xo;
         }
         __syncthreads();
+        KDA_TRACE_POINT(ptr_, 8192 + 19);
         // Abar = INV diag(beta) as MN-major A image: row s = beta_s * column s of INV
         {
             const int jj = tid >> 2;
@@ -608,7 +621,11 @@ done:
 }
 
 // ------------------------------------------------------------------ chunk recurrence
-constexpr int kRecThreads = 192;      // warps 0-3: state rows / TMEM lanes; 4: loader; 5: MMA issuer
+// warps 0-7: state (warp w: rows 32 (w % 4) .. +31 = its TMEM lanes, columns 32 (w / 4) .. +31
+// of the slice); warp 8: loader; warp 9: MMA issuer
+constexpr int kRecThreads = 320;
+constexpr int kRecComputeWarps = 8;
+constexpr int kLoaderWarp = 8, kIssuerWarp = 9;
 constexpr int kStages = 3;
 constexpr uint32_t kStM = 0;          // M, both K blocks (32 KB)
 constexpr uint32_t kStB = 32768;      // B slice [128][64] bf16 (rows swizzled)
@@ -647,11 +664,11 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
     if (tid == 0) {
         for (int st = 0; st < kStages; ++st) {
             mbar_init(full0 + 8 * st, 1);
-            mbar_init(empty0 + 8 * st, 4);
+            mbar_init(empty0 + 8 * st, kRecComputeWarps);
         }
         mbar_init(mma_s, 1);
-        mbar_init(sbr0, 4);
-        mbar_init(sbr0 + 8, 4);
+        mbar_init(sbr0, kRecComputeWarps);
+        mbar_init(sbr0 + 8, kRecComputeWarps);
         fence_mbar_init();
         *abort_flag = 0;
     }
@@ -660,7 +677,7 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
     tc_fence_after();
     const uint32_t tS = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
 
-    if (warp == 4) {
+    if (warp == kLoaderWarp) {
         // ---------------- loader: M, this slice of B, gamma of every chunk -----------------
         if (lane == 0) {
             int issued = 0;
@@ -687,7 +704,7 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
             for (int kk = max(0, issued - kStages); kk < issued; ++kk)
                 mbar_wait(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
         }
-    } else if (warp == 5) {
+    } else if (warp == kIssuerWarp) {
         // ---------------- MMA issuer: D_S = M S_in once the stage and S_in are ready --------
         if (lane == 0) {
             constexpr uint32_t id = idesc_bf16(128, NV, false, true);
@@ -719,27 +736,28 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
             bulk_wait_all();
         }
     } else {
-        // ---------------- state rows i = tid (warps 0-3) ------------------------------------
-        const int i = tid;
-        const uint32_t taw = (uint32_t)(32 * warp) << 16;
-        const size_t sbase = (((size_t)n * H + h) * D + i) * D + (size_t)sl * NV;
-        float Sr[NV];
+        // ---------------- state: row i, columns 32 cw .. 32 cw + 31 of the slice -----------
+        constexpr int NC = NV / 2;   // columns per thread
+        const int i = 32 * (warp & 3) + lane, cw = warp >> 2;
+        const uint32_t taw = (uint32_t)(32 * (warp & 3)) << 16;
+        const size_t sbase = (((size_t)n * H + h) * D + i) * D + (size_t)sl * NV + NC * cw;
+        float Sr[NC];
         if (initial_state) {
 #pragma unroll
-            for (int j4 = 0; j4 < NV / 4; ++j4) {
+            for (int j4 = 0; j4 < NC / 4; ++j4) {
                 const float4 t = reinterpret_cast<const float4*>(initial_state + sbase)[j4];
                 Sr[4 * j4] = t.x; Sr[4 * j4 + 1] = t.y; Sr[4 * j4 + 2] = t.z; Sr[4 * j4 + 3] = t.w;
             }
         } else {
 #pragma unroll
-            for (int j = 0; j < NV; ++j) Sr[j] = 0.f;
+            for (int j = 0; j < NC; ++j) Sr[j] = 0.f;
         }
         // bf16 image of the state entering the next chunk (B operand of its product; the
         // issuer also copies it to the workspace for the output kernel)
         auto put_state = [&](uint32_t buf) {
 #pragma unroll
-            for (int cb = 0; cb < NV / 8; ++cb)
-                *reinterpret_cast<uint4*>(sm + buf + sw128_off(i, cb)) = pack_bf16x8(&Sr[8 * cb]);
+            for (int cb = 0; cb < NC / 8; ++cb)
+                *reinterpret_cast<uint4*>(sm + buf + sw128_off(i, 4 * cw + cb)) = pack_bf16x8(&Sr[8 * cb]);
         };
         if (nchunks > 0) put_state(S::SB);
         fence_proxy_async_smem();
@@ -758,21 +776,20 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
             KDA_TRACE_POINT(tr, kk * 8 + 1);
             // this chunk's gamma and B row, before the serial product lands
             const float gam = reinterpret_cast<const float*>(stage_p + kStG)[i];
-            uint4 bq[NV / 8];
+            uint4 bq[NC / 8];
 #pragma unroll
-            for (int cb = 0; cb < NV / 8; ++cb)
-                bq[cb] = *reinterpret_cast<const uint4*>(stage_p + kStB + sw128_off(i, cb));
+            for (int cb = 0; cb < NC / 8; ++cb)
+                bq[cb] = *reinterpret_cast<const uint4*>(stage_p + kStB + sw128_off(i, 4 * cw + cb));
             KDA_TRACE_POINT(tr, kk * 8 + 2);
             ok = __all_sync(0xffffffffu, mbar_wait(mma_s, kk & 1));
             if (!ok) break;
             KDA_TRACE_POINT(tr, kk * 8 + 3);
             tc_fence_after();
-            float dsv[NV];
-            tmem_ld32(tS + taw, *reinterpret_cast<float(*)[32]>(&dsv[0]));
-            tmem_ld32(tS + taw + 32, *reinterpret_cast<float(*)[32]>(&dsv[32]));
+            float dsv[NC];
+            tmem_ld32(tS + taw + NC * cw, dsv);
             tmem_wait_ld();
 #pragma unroll
-            for (int cb = 0; cb < NV / 8; ++cb) {
+            for (int cb = 0; cb < NC / 8; ++cb) {
                 float bv[8];
                 unpack_bf16x8(bq[cb], bv);
 #pragma unroll
@@ -797,7 +814,7 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
             *abort_flag = 1;
         } else if (final_state) {
 #pragma unroll
-            for (int j4 = 0; j4 < NV / 4; ++j4)
+            for (int j4 = 0; j4 < NC / 4; ++j4)
                 reinterpret_cast<float4*>(final_state + sbase)[j4] =
                     make_float4(Sr[4 * j4], Sr[4 * j4 + 1], Sr[4 * j4 + 2], Sr[4 * j4 + 3]);
         }
