@@ -431,8 +431,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int p = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
             const int R = 16 * (2 * p + 1), Cc = 32 * p;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int smax = ((tid >> 2) & 15) | 7;   // last row of this warp's rows (upper zeros)
 #pragma unroll
             for (int s2 = 0; s2 < 16; ++s2) {
+                if (s2 > smax) break;
                 const float dh = sLI[(R + r) * kLP + R + s2];
                 const float4 tv = *reinterpret_cast<const float4*>(sT + (16 * p + s2) * kTP + c4);
                 acc.x -= dh * tv.x; acc.y -= dh * tv.y; acc.z -= dh * tv.z; acc.w -= dh * tv.w;
@@ -454,8 +456,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             *reinterpret_cast<float4*>(sT + r * kTP + c4) = acc;
             __syncthreads();
             float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
+            const int smax = r | 3;   // rows r of a warp are 4 w .. 4 w + 3; B^{-1}[r][s] = 0 for s > r
+#pragma unroll 4
             for (int s2 = 0; s2 < 32; ++s2) {
+                if (s2 > smax) break;
                 const float bi = sLI[(32 + r) * kLP + 32 + s2];
                 const float4 tv = *reinterpret_cast<const float4*>(sT + s2 * kTP + c4);
                 xo.x -= bi * tv.x; xo.y -= bi * tv.y; xo.z -= bi * tv.z; xo.w -= bi * tv.w;
@@ -464,17 +468,19 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         __syncthreads();
         KDA_TRACE_POINT(ptr_, 8192 + 19);
-        // Abar = INV diag(beta) as MN-major A image: row s = beta_s * column s of INV
+        // Abar = INV diag(beta) as a K-major A image: row r = INV[r][.] scaled by beta
         {
-            const int jj = tid >> 2;
-            const float bj = sBeta[jj];
+            const int r = tid >> 2;
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 const int chnk = 2 * (tid & 3) + h2;
-                float e[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) e[u] = bj * sLI[(8 * chnk + u) * kLP + jj];
-                *reinterpret_cast<uint4*>(sm + S::ABAR + sw128_off(jj, chnk)) = pack_bf16x8(e);
+                const float4 i0 = *reinterpret_cast<const float4*>(sLI + r * kLP + 8 * chnk);
+                const float4 i1 = *reinterpret_cast<const float4*>(sLI + r * kLP + 8 * chnk + 4);
+                const float4 b0 = *reinterpret_cast<const float4*>(sBeta + 8 * chnk);
+                const float4 b1 = *reinterpret_cast<const float4*>(sBeta + 8 * chnk + 4);
+                const float e[8] = {i0.x * b0.x, i0.y * b0.y, i0.z * b0.z, i0.w * b0.w,
+                                    i1.x * b1.x, i1.y * b1.y, i1.z * b1.z, i1.w * b1.w};
+                *reinterpret_cast<uint4*>(sm + S::ABAR + sw128_off(r, chnk)) = pack_bf16x8(e);
             }
         }
     }
@@ -485,10 +491,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // ---- (4) [W | U] = Abar [K_dec | V] -> TMEM [0, 256) (lanes 0-63 meaningful) ----
     if (tid == 0) {
         tc_fence_after();
-        constexpr uint32_t id = idesc_bf16(128, 256, true, true);
+        constexpr uint32_t id = idesc_bf16(128, 256, false, true);
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
-            umma_bf16(tmem, smem_desc(sb + S::ABAR + ks * 2048, 8192, 1024, kSwizzle128),
+            umma_bf16(tmem, smem_desc(sb + S::ABAR + ks * 32, 16, 1024, kSwizzle128),
                       smem_desc(sb + S::KD0 + ks * 2048, S::BLK, 1024, kSwizzle128), id, ks > 0);
         umma_commit(bar);
     }
