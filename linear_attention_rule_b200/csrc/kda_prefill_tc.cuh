@@ -866,7 +866,7 @@ out_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
     uint8_t* sm = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     const uint32_t sb = smem_u32(sm);
     const uint32_t bar = sb + S::BAR;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
 
     if (warp == 0) tmem_alloc(sb + S::TMEM, kOutTmemCols);
     if (tid == 0) {
@@ -958,24 +958,26 @@ inline bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, 
                sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* g,
-                                  const float* beta, const float* s0, const int32_t* cu,
-                                  int num_seqs, int64_t total, int H, void* out, float* sf,
-                                  void* workspace, cudaStream_t stream) {
-    int32_t* off = static_cast<int32_t*>(workspace);
-    uint8_t* records = static_cast<uint8_t*>(workspace) + ws_records_offset(num_seqs);
-    uint8_t* states = static_cast<uint8_t*>(workspace) + ws_states_offset(total, num_seqs, H);
+struct Workspace {
+    int32_t* off;
+    uint8_t* records;
+    uint8_t* states;
+};
+inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs, int H) {
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    return {reinterpret_cast<int32_t*>(base), base + ws_records_offset(num_seqs),
+            base + ws_states_offset(total, num_seqs, H)};
+}
+
+// Chunk table + chunk-parallel preparation.
+inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const int32_t* cu, int num_seqs,
+                                  int64_t total, int H, void* workspace, cudaStream_t stream) {
+    const Workspace w = split_workspace(workspace, total, num_seqs, H);
     cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepSmem::BYTES);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(rec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)RecSmem::BYTES);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)OutSmem::BYTES);
-    if (e != cudaSuccess) return e;
-    chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, off);
-    const int64_t mc = max_chunks(total, num_seqs);
+    chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off);
     if (total > 0) {
         CUtensorMap tq, tk, tv, tg;
         if (!make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -983,18 +985,58 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
             !make_tmap(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_tmap(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
-        dim3 grid((unsigned)mc, (unsigned)H);
+        dim3 grid((unsigned)max_chunks(total, num_seqs), (unsigned)H);
         prep_kernel<<<grid, kPrepThreads, PrepSmem::BYTES, stream>>>(tq, tk, tv, tg, beta, cu,
-                                                                     num_seqs, H, off, records);
-    }
-    rec_kernel<<<(unsigned)num_seqs * H * NSL, kRecThreads, RecSmem::BYTES, stream>>>(
-        cu, num_seqs, H, off, records, states, s0, sf);
-    if (total > 0) {
-        dim3 grid((unsigned)mc, (unsigned)H);
-        out_kernel<<<grid, kOutThreads, OutSmem::BYTES, stream>>>(
-            cu, num_seqs, H, off, records, states, static_cast<__nv_bfloat16*>(out));
+                                                                     num_seqs, H, w.off, w.records);
     }
     return cudaGetLastError();
+}
+
+// Chunk-serial recurrence over every (sequence, head, value slice).
+inline cudaError_t launch_scan(const float* s0, float* sf, const int32_t* cu, int num_seqs,
+                               int64_t total, int H, void* workspace, cudaStream_t stream) {
+    const Workspace w = split_workspace(workspace, total, num_seqs, H);
+    cudaError_t e = cudaFuncSetAttribute(rec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)RecSmem::BYTES);
+    if (e != cudaSuccess) return e;
+    rec_kernel<<<(unsigned)num_seqs * H * NSL, kRecThreads, RecSmem::BYTES, stream>>>(
+        cu, num_seqs, H, w.off, w.records, w.states, s0, sf);
+    return cudaGetLastError();
+}
+
+// Chunk-parallel outputs.
+inline cudaError_t launch_output(void* out, const int32_t* cu, int num_seqs, int64_t total, int H,
+                                 void* workspace, cudaStream_t stream) {
+    if (total == 0) return cudaSuccess;
+    const Workspace w = split_workspace(workspace, total, num_seqs, H);
+    cudaError_t e = cudaFuncSetAttribute(out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)OutSmem::BYTES);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)max_chunks(total, num_seqs), (unsigned)H);
+    out_kernel<<<grid, kOutThreads, OutSmem::BYTES, stream>>>(cu, num_seqs, H, w.off, w.records,
+                                                               w.states, static_cast<__nv_bfloat16*>(out));
+    return cudaGetLastError();
+}
+
+inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const float* s0, const int32_t* cu,
+                                  int num_seqs, int64_t total, int H, void* out, float* sf,
+                                  void* workspace, cudaStream_t stream) {
+    cudaError_t e = launch_prepare(q, k, v, g, beta, cu, num_seqs, total, H, workspace, stream);
+    if (e == cudaSuccess) e = launch_scan(s0, sf, cu, num_seqs, total, H, workspace, stream);
+    if (e == cudaSuccess) e = launch_output(out, cu, num_seqs, total, H, workspace, stream);
+    return e;
+}
+
+// One thread waits (bounded) on a barrier nothing arrives on and reports the expiry.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar_storage;
+    if (threadIdx.x == 0) {
+        const uint32_t bar = smem_u32(&bar_storage);
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        if (!mbar_wait(bar, 0, limit_ns)) kda_set_status(KDA_ERR_TIMEOUT);
+    }
 }
 
 }  // namespace tc

@@ -104,6 +104,70 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+// Checks shared by the staged tensor-core entry points.
+static kda_status check_staged(const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                               int32_t H, int32_t dk, int32_t dv, kda_dtype dt, int32_t C,
+                               const void* workspace, size_t ws_bytes) {
+    if (num_seqs < 0 || total_tokens < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (total_tokens > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    if (!tensor_core_path(dt, dk) || !supported_dim(dk, dv) || !valid_chunk(dt, C))
+        return KDA_ERR_UNSUPPORTED;
+    if (num_seqs > 0 && (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0))
+        return KDA_ERR_INVALID_ARG;
+    const size_t need = kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, dt);
+    if (ws_bytes < need || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+
+kda_status kda_prefill_prepare(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const int32_t* cu_seqlens, int32_t num_seqs,
+                               int64_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                               kda_dtype dt, int32_t C, void* workspace, size_t ws_bytes,
+                               kda_stream_t stream) {
+    kda_status st = check_staged(cu_seqlens, num_seqs, total_tokens, H, dk, dv, dt, C, workspace, ws_bytes);
+    if (st != KDA_OK || num_seqs == 0) return st;
+    if (total_tokens > 0 && (!q || !k || !v || !g || !beta)) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, beta};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    return kda::tc::launch_prepare(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, H, workspace,
+                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_prefill_scan(const float* initial_state, float* final_state,
+                            const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                            int32_t H, int32_t dk, int32_t dv, kda_dtype dt, int32_t C,
+                            void* workspace, size_t ws_bytes, kda_stream_t stream) {
+    kda_status st = check_staged(cu_seqlens, num_seqs, total_tokens, H, dk, dv, dt, C, workspace, ws_bytes);
+    if (st != KDA_OK || num_seqs == 0) return st;
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return KDA_ERR_INVALID_ARG;
+    return kda::tc::launch_scan(initial_state, final_state, cu_seqlens, num_seqs, total_tokens, H,
+                                workspace, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_prefill_output(void* out, const int32_t* cu_seqlens, int32_t num_seqs,
+                              int64_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                              kda_dtype dt, int32_t C, void* workspace, size_t ws_bytes,
+                              kda_stream_t stream) {
+    kda_status st = check_staged(cu_seqlens, num_seqs, total_tokens, H, dk, dv, dt, C, workspace, ws_bytes);
+    if (st != KDA_OK || num_seqs == 0) return st;
+    if (total_tokens > 0 && (!out || !aligned16(out))) return KDA_ERR_INVALID_ARG;
+    return kda::tc::launch_output(out, cu_seqlens, num_seqs, total_tokens, H, workspace,
+                                  reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_selftest_bounded_wait(uint64_t limit_ns, kda_stream_t stream) {
+    if (limit_ns < 1000ull || limit_ns > 2000000000ull) return KDA_ERR_INVALID_ARG;
+    kda::tc::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status kda_decode(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* state_inout, void* out, int32_t N, int32_t H,
                       int32_t dk, int32_t dv, kda_dtype dt, kda_stream_t stream) {

@@ -155,3 +155,38 @@ def make_decode_step_inputs(N: int, H: int, dk: int, dv: int, dtype: torch.dtype
     d = make_prefill_inputs([1] * N, H, dk, dv, dtype, g_mean, 0.0,
                             seed + STEP_SEED_STRIDE * (step + 1), heads=heads)
     return dict(q=d["q"], k=d["k"], v=d["v"], g=d["g"], beta=d["beta"])
+
+
+def make_prefill_inputs_device(lengths: Sequence[int], H: int, dk: int, dv: int,
+                               dtype: torch.dtype, g_mean: float, s0_std: float, seed: int,
+                               cpu_heads: Sequence[int] = (), device="cuda") -> dict:
+    """Large batches: draw every head with a seeded torch device generator (same recipe),
+    except `cpu_heads`, which are drawn from their per-head CPU streams exactly as
+    make_prefill_inputs does (so an oracle can be given those heads' identical bytes).
+    Returns device tensors plus `cpu` = the make_prefill_inputs(..., heads=cpu_heads) dict."""
+    T = int(sum(lengths))
+    N = len(lengths)
+    gen = torch.Generator(device=device).manual_seed(seed)
+    q = torch.empty(T, H, dk, dtype=dtype, device=device)
+    k = torch.empty(T, H, dk, dtype=dtype, device=device)
+    v = torch.empty(T, H, dv, dtype=dtype, device=device)
+    g = torch.empty(T, H, dk, dtype=torch.float32, device=device)
+    beta = torch.empty(T, H, dtype=torch.float32, device=device)
+    s0 = torch.empty(N, H, dk, dv, dtype=torch.float32, device=device) if s0_std > 0 else None
+    for h in range(H):
+        q[:, h] = _l2_normalise(torch.randn(T, dk, generator=gen, device=device)).to(dtype)
+        k[:, h] = _l2_normalise(torch.randn(T, dk, generator=gen, device=device)).to(dtype)
+        v[:, h] = torch.randn(T, dv, generator=gen, device=device).to(dtype)
+        beta[:, h] = torch.sigmoid(torch.randn(T, generator=gen, device=device))
+        g[:, h] = torch.nn.functional.logsigmoid(
+            g_mean + torch.randn(T, dk, generator=gen, device=device))
+        if s0 is not None:
+            s0[:, h] = s0_std * torch.randn(N, dk, dv, generator=gen, device=device)
+    cpu = make_prefill_inputs(lengths, H, dk, dv, dtype, g_mean, s0_std, seed, heads=cpu_heads)
+    for j, h in enumerate(cpu_heads):
+        for key, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
+            t[:, h] = cpu[key][:, j].to(device)
+        if s0 is not None:
+            s0[:, h] = cpu["s0"][:, j].to(device)
+    return dict(q=q, k=k, v=v, g=g, beta=beta, cu_seqlens=cu_seqlens_of(lengths).to(device),
+                s0=s0, cpu=cpu)

@@ -101,3 +101,25 @@ def test_decode_rejects_bad_arguments(lib):
     assert dec(g=P(4097)) == kda.KDA_ERR_INVALID_ARG
     assert dec(dt=5) == kda.KDA_ERR_INVALID_ARG
     assert dec(N=0) == kda.KDA_OK
+
+
+def test_staged_entry_points_reject_bad_arguments(lib):
+    P = ctypes.c_void_p
+    need = lib.kda_prefill_workspace_size(256, 1, 2, 128, 128, 64, kda.KDA_BF16)
+    ws = P(1 << 20)
+    # only the tensor-core problem is staged
+    assert lib.kda_prefill_prepare(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), 1, 256, 2,
+                                   64, 64, kda.KDA_F32, 64, ws, need, None) == kda.KDA_ERR_UNSUPPORTED
+    assert lib.kda_prefill_scan(None, None, P(4096), 1, 256, 2, 128, 128, kda.KDA_BF16, 64, ws,
+                                need - 1, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_prefill_output(None, P(4096), 1, 256, 2, 128, 128, kda.KDA_BF16, 64, ws, need,
+                                  None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_prefill_output(P(4096), P(4096), 1, 256, 2, 128, 128, kda.KDA_BF16, 64, P(4096 + 16),
+                                  need, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_prefill_scan(None, None, P(4096), 0, 0, 2, 128, 128, kda.KDA_BF16, 64, ws, need,
+                                None) == kda.KDA_OK
+
+
+def test_selftest_rejects_out_of_range_limits(lib):
+    assert lib.kda_selftest_bounded_wait(10, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_selftest_bounded_wait(3_000_000_000, None) == kda.KDA_ERR_INVALID_ARG

@@ -135,3 +135,37 @@ def test_bad_cu_seqlens_reported_by_device():
     kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], bad, out, C=64)
     assert kda.kda_get_device_status() == kda.KDA_ERR_BAD_SEQLENS
     assert kda.kda_get_device_status() == kda.KDA_OK   # cleared by the read
+
+
+@pytest.mark.slow
+def test_config4_long_context_full_size_sampled_heads():
+    """Config 4 at full size: T = 1,048,576, H = 32, D = 128, bf16, slow decay
+    g = logsigmoid(N(4, 1)), zero initial state, in the benchmark's launch configuration.
+    Heads 0 and 17 are drawn on the CPU and followed by the fp64 oracle over all 1M tokens
+    (every output row and the final state); the other heads are drawn on the device."""
+    import oracle
+    cfg = synthetic.CONFIGS[4]
+    lens = synthetic.draw_lengths(cfg)
+    heads = [0, 17]
+    d = synthetic.make_prefill_inputs_device(lens, cfg.H, cfg.D, cfg.D, cfg.dtype, cfg.g_mean,
+                                             cfg.s0_std, cfg.seed, cpu_heads=heads)
+    T = sum(lens)
+    out = torch.empty(T, cfg.H, cfg.D, dtype=cfg.dtype, device="cuda")
+    fin = torch.empty(1, cfg.H, cfg.D, cfg.D, device="cuda")
+    kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out,
+                    final_state=fin, C=cfg.C)
+    assert kda.kda_get_device_status() == kda.KDA_OK
+    o = out[:, heads].double().cpu().numpy()
+    f = fin[:, heads].double().cpu().numpy()
+    del d["q"], d["k"], d["v"], d["g"], out
+    c = d["cpu"]
+    o_ref, f_ref = oracle.prefill(c["q"], c["k"], c["v"], c["g"], c["beta"], c["cu_seqlens"],
+                                  nthreads=len(heads))
+    e_o = oracle.max_rel_frobenius_per_slice(o, o_ref, c["cu_seqlens"])
+    e_f = oracle.max_rel_frobenius_states(f, f_ref)
+    print("config4 max rel err out %.3g final %.3g" % (e_o, e_f))
+    assert e_o <= TOL[torch.bfloat16] and e_f <= TOL[torch.bfloat16]
+    # windows along the sequence (early, middle, end) stay within tolerance too
+    for a in (0, T // 2, T - 65536):
+        e_w = oracle.rel_frobenius(o[a:a + 65536], o_ref[a:a + 65536])
+        assert e_w <= TOL[torch.bfloat16], (a, e_w)
