@@ -84,6 +84,44 @@ def prefill_page_counts(lengths, H, D, C):
     return flops, bytes_
 
 
+def prefill_stage_page_bytes(lengths, H, D, C):
+    """The pages' byte count split by stage (FlashKDA section): the preparation reads
+    q, k, v (3 x 2CD) and writes the chunk tensors (3 x 2CD + 2 x 2C^2); the recurrence
+    reads them back and writes O (2 x 2CD), plus the 8 D^2 state bytes per head."""
+    chunks = sum((n + C - 1) // C for n in lengths)
+    ch = chunks * H
+    prep = ch * (3 * 2 * C * D + 3 * 2 * C * D + 2 * 2 * C * C)
+    rest = ch * (3 * 2 * C * D + 2 * 2 * C * C + 2 * 2 * C * D) + 8 * D * D * len(lengths) * H
+    return prep, rest
+
+
+def source_digest():
+    """Short hash of the CUDA sources, to tell whether recorded ncu counters still apply."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_rule_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` recorded from an ncu capture in profiles/
+    ('<kernel> traffic_bytes_per_launch <N> sources <digest>'), or None when absent or
+    taken on different sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        with open(path) as fh:
+            for line in fh:
+                f = line.split()
+                if len(f) >= 5 and f[0] == kernel and f[1] == "traffic_bytes_per_launch":
+                    return int(f[2]) if f[4] == source_digest() else None
+    except OSError:
+        pass
+    return None
+
+
 def prefill_strict_bytes(lengths, H, D, in_bytes, has_s0, has_final):
     """Bytes the method itself must move: q, k, v, out in the input dtype, g fp32 (dk per
     token-head), beta fp32, and the fp32 states read/written."""
@@ -197,16 +235,22 @@ def timed(stream, dev, world, steps, fn):
     return ms_local, max_over_ranks(ms_local, world, dev), clk.summary()
 
 
-def setup_prefill(dev, rank):
+def setup_prefill(dev, rank, cfg_id=PREFILL_CFG):
     import torch
     from linear_attention_rule_b200 import kda, synthetic
-    cfg = synthetic.CONFIGS[PREFILL_CFG]
+    cfg = synthetic.CONFIGS[cfg_id]
     lengths = synthetic.draw_lengths(cfg)
     D, H, C = cfg.D, cfg.H, cfg.C
-    inp = synthetic.make_prefill_inputs(lengths, H, D, D, cfg.dtype, cfg.g_mean, cfg.s0_std,
-                                        rank_seed(cfg.seed, rank))
-    T, N = inp["q"].shape[0], len(lengths)
-    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    if sum(lengths) * H > (1 << 24):   # large batches are drawn on the device (same recipe)
+        d = synthetic.make_prefill_inputs_device(lengths, H, D, D, cfg.dtype, cfg.g_mean,
+                                                 cfg.s0_std, rank_seed(cfg.seed, rank), device=dev)
+        d.pop("cpu")
+        inp = None
+    else:
+        inp = synthetic.make_prefill_inputs(lengths, H, D, D, cfg.dtype, cfg.g_mean, cfg.s0_std,
+                                            rank_seed(cfg.seed, rank))
+        d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    T, N = sum(lengths), len(lengths)
     out = torch.empty(T, H, D, dtype=cfg.dtype, device=dev)
     fin = torch.empty(N, H, D, D, dtype=torch.float32, device=dev)
     ws_bytes = kda.kda_prefill_workspace_size(T, N, H, D, D, C, cfg.dtype)
@@ -216,6 +260,7 @@ def setup_prefill(dev, rank):
 
 
 def bench_prefill(args, P, dev, stream, world, peaks):
+    import torch
     from linear_attention_rule_b200 import kda
     cfg, d, D, H, C, T = P["cfg"], P["d"], P["D"], P["H"], P["C"], P["T"]
 
@@ -231,22 +276,70 @@ def bench_prefill(args, P, dev, stream, world, peaks):
     assert kda.kda_get_device_status(stream) == kda.KDA_OK
     flops, page_bytes = prefill_page_counts(P["lengths"], H, D, C)
     strict = prefill_strict_bytes(P["lengths"], H, D, 2 if cfg.dtype.itemsize == 2 else 4,
-                                  P["inp"]["s0"] is not None, True)
+                                  d["s0"] is not None, True)
     t_s = ms_local * 1e-3
-    achieved = page_bytes / t_s / 1e9
-    roofline = {
-        "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-        "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
-        "kernel": "kda_prefill (whole path: chunk index + prep + recurrence)",
-        "bytes_per_launch": page_bytes,
-        "counts": "pages' 8C^2+22CD bytes per chunk-head + 8D^2 per head",
-        "peak_source": peaks["source"],
-        "tensor_frac": round(flops / t_s / 1e12 / peaks["bf16_tflops"], 4),
-        "strict_frac": round(strict / t_s / 1e9 / peaks["hbm_gbs"], 4),
-    }
-    return dict(value=world * T / (ms * 1e-3), ms=ms, ms_local=ms_local, roofline=roofline,
-                clocks=clocks, launches=kda.prefill_launches(cfg.dtype, D) * args.steps,
-                step=step)
+    res = dict(value=world * T / (ms * 1e-3), ms=ms, ms_local=ms_local, clocks=clocks,
+               launches=kda.prefill_launches(cfg.dtype, D) * args.steps, step=step,
+               whole_frac=page_bytes / t_s / 1e9 / peaks["hbm_gbs"],
+               tensor_frac=flops / t_s / 1e12 / peaks["bf16_tflops"],
+               strict_frac=strict / t_s / 1e9 / peaks["hbm_gbs"])
+
+    # Per kernel: the same work through the staged entry points, CUDA events between the
+    # stages on the launching stream.
+    stage_ms = None
+    if kda.prefill_launches(cfg.dtype, D) > 1:
+        ws = P["ws"]
+        stages = [
+            ("prep_kernel", lambda: kda.kda_prefill_prepare(d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                                            d["cu_seqlens"], ws, C=C, stream=stream)),
+            ("rec_kernel", lambda: kda.kda_prefill_scan(d["cu_seqlens"], T, H, D, ws,
+                                                        initial_state=d["s0"], final_state=P["fin"],
+                                                        C=C, stream=stream)),
+            ("out_kernel", lambda: kda.kda_prefill_output(P["out"], d["cu_seqlens"], ws, C=C,
+                                                          stream=stream)),
+        ]
+        for _ in range(args.warmup):
+            for _, f in stages:
+                f()
+        torch.cuda.synchronize(dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+              for _ in range(args.steps)]
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            for j, (_, f) in enumerate(stages):
+                f()
+                ev[i][j + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        assert kda.kda_get_device_status(stream) == kda.KDA_OK
+        stage_ms = {name: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)) / args.steps
+                    for j, (name, _) in enumerate(stages)}
+        prep_bytes, _ = prefill_stage_page_bytes(P["lengths"], H, D, C)
+        top = max(stage_ms, key=stage_ms.get)
+        per_launch = {"prep_kernel": prep_bytes}
+        if top in per_launch:
+            achieved = per_launch[top] / (stage_ms[top] * 1e-3) / 1e9
+            res["roofline"] = {
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": recorded_traffic(top), "kernel": "kda::tc::" + top,
+                "bytes_per_launch": per_launch[top],
+                "counts": "pages' preparation bytes 3x2CD + (3x2CD + 2x2C^2) per chunk-head",
+                "peak_source": peaks["source"], "ms_per_launch": round(stage_ms[top], 4),
+            }
+        res["stage_ms"] = {k: round(v, 4) for k, v in stage_ms.items()}
+    if "roofline" not in res:
+        achieved = page_bytes / t_s / 1e9
+        res["roofline"] = {
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+            "kernel": "kda_prefill (single kernel)", "bytes_per_launch": page_bytes,
+            "counts": "pages' 8C^2+22CD bytes per chunk-head + 8D^2 per head",
+            "peak_source": peaks["source"],
+        }
+    res["roofline"]["path_frac"] = round(res["whole_frac"], 4)
+    res["roofline"]["path_strict_frac"] = round(res["strict_frac"], 4)
+    res["roofline"]["path_tensor_frac"] = round(res["tensor_frac"], 4)
+    return res
 
 
 def bench_decode(args, dev, stream, rank, world, peaks):
@@ -327,13 +420,19 @@ def bench_gpu(args):
     stream = torch.cuda.current_stream(dev)
 
     line = {}
-    if args.workload in ("all", "prefill"):
+    if args.workload in ("config2", "config4"):
+        P = setup_prefill(dev, rank, int(args.workload[-1]))
+        pre = bench_prefill(args, P, dev, stream, world, peaks)
+        line = {"workload": P["cfg"].name, "value": round(pre["value"], 1), "unit": "tokens/s",
+                "ms_per_step": round(pre["ms"], 4), "roofline": pre["roofline"],
+                "stage_ms": pre.get("stage_ms"), "clocks": pre["clocks"], "n_gpus": world}
+    elif args.workload in ("all", "prefill"):
         P = setup_prefill(dev, rank)
         pre = bench_prefill(args, P, dev, stream, world, peaks)
         decode = bench_decode(args, dev, stream, rank, world, peaks) if args.workload == "all" else None
         e2e = None if args.no_e2e else bench_e2e(args, P, pre, dev, stream, world)
         cpu = None
-        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if rank == 0 and world == 1 and not args.no_cpu_baseline and P["inp"] is not None:
             tps, ts, secs, threads = oracle_sample_tokens_per_s(P["inp"], args.cpu_seconds)
             cpu = {"value": round(tps, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
                    "sample": "first %d tokens x all %d heads of the same workload (repeated), "
@@ -350,8 +449,9 @@ def bench_gpu(args):
                            sum(P["d"][k].numel() * P["d"][k].element_size()
                                for k in ("q", "k", "v", "g", "beta")) / 1e6),
                        "parallelism": "replicas" if world > 1 else "single GPU"},
-            "roofline": pre["roofline"], "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
-            "clocks": pre["clocks"], "gpu_launches": pre["launches"],
+            "roofline": pre["roofline"], "stage_ms": pre.get("stage_ms"), "decode": decode,
+            "e2e": e2e, "cpu_baseline": cpu, "clocks": pre["clocks"],
+            "gpu_launches": pre["launches"],
         }
     else:
         line = {"decode": bench_decode(args, dev, stream, rank, world, peaks)}
@@ -414,8 +514,10 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--workload", choices=["all", "prefill", "decode"], default="all",
-                    help="restrict the run (profiling); the JSON line needs 'all'")
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "config2", "config4"],
+                    default="all",
+                    help="restrict the run (profiling) or measure another prefill config; "
+                         "the driver's JSON line is 'all'")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
