@@ -61,27 +61,45 @@ constexpr uint32_t kStateImgBytes = 32768;
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline size_t ws_records_offset(int num_seqs) {
-    return align_up(sizeof(int32_t) * (size_t)(num_seqs + 1), 1024);
-}
 __host__ inline int64_t max_chunks(int64_t total_tokens, int num_seqs) {
     return total_tokens / C + num_seqs;
 }
-__host__ inline size_t ws_states_offset(int64_t total_tokens, int num_seqs, int H) {
-    return ws_records_offset(num_seqs) + (size_t)max_chunks(total_tokens, num_seqs) * H * kRecBytes;
+// Workspace: [chunk offsets int32 (N+1)] [chunk table int2 (max_chunks)] [records
+// (max_chunks x H)] [chunk states (max_chunks x H)]
+__host__ inline size_t ws_table_offset(int num_seqs) {
+    return align_up(sizeof(int32_t) * (size_t)(num_seqs + 1), 16);
 }
-// Workspace: [chunk offsets int32 (N+1)] [records (max_chunks x H)] [chunk states (max_chunks x H)]
+__host__ inline size_t ws_records_offset(int64_t total_tokens, int num_seqs) {
+    return align_up(ws_table_offset(num_seqs) + sizeof(int2) * (size_t)max_chunks(total_tokens, num_seqs),
+                    1024);
+}
+__host__ inline size_t ws_states_offset(int64_t total_tokens, int num_seqs, int H) {
+    return ws_records_offset(total_tokens, num_seqs) +
+           (size_t)max_chunks(total_tokens, num_seqs) * H * kRecBytes;
+}
 __host__ inline size_t workspace_bytes(int64_t total_tokens, int num_seqs, int H) {
     return ws_states_offset(total_tokens, num_seqs, H) +
            (size_t)max_chunks(total_tokens, num_seqs) * H * kStateImgBytes;
 }
 
 // ------------------------------------------------------------------ chunk index
-// Single CTA of 1024 threads: off[n] = sum_{m<n} ceil(len_m / C), off[N] = total chunks.
+// Sequence containing global chunk c: the largest n with off[n] <= c.
+__device__ __forceinline__ int find_seq(const int32_t* off, int num_seqs, int c) {
+    int lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= c) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Single CTA of 1024 threads: off[n] = sum_{m<n} ceil(len_m / C), off[N] = total chunks,
+// and the chunk table tab[c] = (first token, rows) of every chunk c < off[N], so that the
+// chunk-parallel kernels find their tokens with one load.
 // Inconsistent cu_seqlens -> KDA_ERR_BAD_SEQLENS and every count 0 (nothing downstream runs).
 __global__ void __launch_bounds__(1024)
 chunk_index_kernel(const int32_t* __restrict__ cu, int num_seqs, int64_t total,
-                   int32_t* __restrict__ off) {
+                   int32_t* __restrict__ off, int2* __restrict__ tab) {
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t carry;
     __shared__ int bad;
@@ -124,21 +142,18 @@ chunk_index_kernel(const int32_t* __restrict__ cu, int num_seqs, int64_t total,
         __syncthreads();
     }
     if (tid == 0) off[num_seqs] = carry;
-    __syncthreads();
+    __syncthreads();   // off[] (global, written by this CTA) is visible to all its threads
     if (bad) {
         if (tid == 0) kda_set_status(KDA_ERR_BAD_SEQLENS);
         for (int n = tid; n <= num_seqs; n += 1024) off[n] = 0;
+        return;
     }
-}
-
-// Sequence containing global chunk c: the largest n with off[n] <= c.
-__device__ __forceinline__ int find_seq(const int32_t* off, int num_seqs, int c) {
-    int lo = 0, hi = num_seqs - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (off[mid] <= c) lo = mid; else hi = mid - 1;
+    const int nch = carry;
+    for (int c = tid; c < nch; c += 1024) {
+        const int n = find_seq(off, num_seqs, c);
+        const int t0 = cu[n] + (c - off[n]) * C;
+        tab[c] = make_int2(t0, min(C, cu[n + 1] - t0));
     }
-    return lo;
 }
 
 // 2-D tiled TMA load (no multicast) of box (x, y) of `tmap` into shared memory.
@@ -187,18 +202,18 @@ __device__ __forceinline__ uint32_t stage_slot(int w) {
     return base + (w & 1) * 4096;
 }
 
+// One CTA per (chunk, head) unit, 2 CTAs per SM.
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-            const float* __restrict__ beta, const int32_t* __restrict__ cu, int num_seqs, int H,
-            const int32_t* __restrict__ off, uint8_t* __restrict__ records) {
+            const float* __restrict__ beta, int num_seqs, int H, const int32_t* __restrict__ off,
+            const int2* __restrict__ tab, uint8_t* __restrict__ records) {
     using S = PrepSmem;
     const int c = blockIdx.x, h = blockIdx.y;
     const int total_chunks = off[num_seqs];
+    const int2 e = tab[c];   // in bounds for every c < max_chunks; meaningful for c < total
     if (c >= total_chunks) return;
-    const int n = find_seq(off, num_seqs, c);
-    const int t0 = cu[n] + (c - off[n]) * C;
-    const int nrow = min(C, cu[n + 1] - t0);
+    const int t0 = e.x, nrow = e.y;
     uint8_t* rec = records + ((size_t)c * H + h) * kRecBytes;
 
     extern __shared__ uint8_t smem_raw[];
@@ -213,20 +228,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     bool ok = true;
     uint32_t phase = 0;
 
-    if (warp == 0) tmem_alloc(sb + S::TMEM, kPrepTmemCols);
+    // ---- (0) TMA: rows t0..t0+63 of q, k, v (two 64-channel boxes each) and g; the
+    // barrier is initialised and the copies issued by the same thread, before anything else
     if (tid == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
-    }
-    if (tid < C) sBeta[tid] = tid < nrow ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
-    const uint32_t tl = tmem + ((uint32_t)(32 * wq) << 16);   // this warp's TMEM lanes
-
-    // ---- (0) TMA: rows t0..t0+63 of q, k, v (two 64-channel boxes each) and g ----
-    if (tid == 0) {
         mbar_arrive_expect_tx(bar, kPrepTx);
         const int x0 = h * D;
         tma_load_2d(sb + S::QD0, &tm_q, x0, t0, bar);
@@ -237,6 +243,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tma_load_2d(sb + S::V1, &tm_v, x0 + 64, t0, bar);
         tma_load_2d(sb + S::GR, &tm_g, x0, t0, bar);
     }
+    if (warp == 1) tmem_alloc(sb + S::TMEM, kPrepTmemCols);
+    if (tid < C) sBeta[tid] = tid < nrow ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
+    const uint32_t tl = tmem + ((uint32_t)(32 * wq) << 16);   // this warp's TMEM lanes
     const bool ptr_ = blockIdx.x == 37 && blockIdx.y == 3 && tid == 0;
     (void)ptr_;
     KDA_TRACE_POINT(ptr_, 8192 + 0);
@@ -372,16 +385,42 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
         }
-        // K_res = K_inv gamma, in place (the first MMA has finished reading K_inv)
+        // First step of the UT transform INV = (I + L)^{-1}: the 16x16 diagonal blocks D_b,
+        // inverted in place by the warp that drained them (warp 0: blocks 0, 1 = rows and
+        // columns 0..31; warp 5: blocks 2, 3), lane = (block, column j).  Column-oriented
+        // forward substitution: once x[s] is final it is subtracted from every later row, so
+        // the dependent chain is 15 FMAs long.
+        if (warp == 0 || warp == 5) {
+            __syncwarp();
+            const int b = (warp == 5 ? 2 : 0) + (lane >> 4), j = lane & 15;
+            float x[16];
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            const uint32_t o = S::KI0 + kb * S::BLK + sw128_off(4 * rb + rr, c8);
-            float ki[8];
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + o), ki);
+            for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) ki[u] *= gam[u];
-            *reinterpret_cast<uint4*>(sm + o) = pack_bf16x8(ki);
+            for (int s2 = 0; s2 < 15; ++s2) {
+#pragma unroll
+                for (int r = s2 + 1; r < 16; ++r) x[r] -= sLI[(16 * b + r) * kLP + 16 * b + s2] * x[s2];
+            }
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < 16; ++r) sLI[(16 * b + r) * kLP + 16 * b + j] = x[r];
         }
+        // K_res = K_inv gamma, in place (the first MMA has finished reading K_inv); warps 1
+        // and 4 also take the rows of warps 0 and 5
+        auto kres_rows = [&](int wsrc) {
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const uint32_t o = S::KI0 + kb * S::BLK + sw128_off(4 * (2 * wsrc + half) + rr, c8);
+                float ki[8];
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + o), ki);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) ki[u] *= gam[u];
+                *reinterpret_cast<uint4*>(sm + o) = pack_bf16x8(ki);
+            }
+        };
+        if (warp != 0 && warp != 5) kres_rows(warp);
+        if (warp == 1) kres_rows(0);
+        if (warp == 4) kres_rows(5);
     }
     tc_fence_before();
     fence_proxy_async_smem();
@@ -393,26 +432,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // the inverse is lower triangular), so the block products below need no masks.
     {
         float* sT = sX;
-        // 16x16 diagonal blocks D_b by forward substitution: thread (block b, column j)
-        float x[16];
-        const int b = tid >> 4, j = tid & 15;
-        if (tid < 64) {
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = (r == j) ? 1.f : 0.f;
-#pragma unroll
-                for (int s2 = 0; s2 < r; ++s2) acc -= sLI[(16 * b + r) * kLP + 16 * b + s2] * x[s2];
-                x[r] = acc;
-            }
-        }
-        __syncthreads();
-        KDA_TRACE_POINT(ptr_, 8192 + 16);
-        if (tid < 64) {
-#pragma unroll
-            for (int r = 0; r < 16; ++r) sLI[(16 * b + r) * kLP + 16 * b + j] = x[r];
-        }
-        __syncthreads();
-        KDA_TRACE_POINT(ptr_, 8192 + 17);
         // 16 -> 32, block pairs (0,1) and (2,3): X = -D_hi (L_lo D_lo); 1x4 tiles per thread
         if (tid < 128) {
             const int p = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
@@ -464,25 +483,21 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const float4 tv = *reinterpret_cast<const float4*>(sT + s2 * kTP + c4);
                 xo.x -= bi * tv.x; xo.y -= bi * tv.y; xo.z -= bi * tv.z; xo.w -= bi * tv.w;
             }
-            *reinterpret_cast<float4*>(sLI + (32 + r) * kLP + c4) = xo;
+            // Abar = INV diag(beta) as a bf16 K-major A image.  This thread writes columns
+            // c4..c4+3 and 32+c4..32+c4+3 of rows r and 32 + r: the block just computed, and
+            // entries final since the 16 -> 32 step (INV[r][32..63] = 0 for r < 32).
+            const float4 b_lo = *reinterpret_cast<const float4*>(sBeta + c4);
+            const float4 b_hi = *reinterpret_cast<const float4*>(sBeta + 32 + c4);
+            auto put4 = [&](int row, int col, float4 x4, float4 b4) {
+                *reinterpret_cast<uint2*>(sm + S::ABAR + sw128_off(row, col >> 3) + (col & 4) * 2) =
+                    make_uint2(pack_bf16x2(x4.x * b4.x, x4.y * b4.y), pack_bf16x2(x4.z * b4.z, x4.w * b4.w));
+            };
+            put4(32 + r, c4, xo, b_lo);
+            put4(r, c4, *reinterpret_cast<const float4*>(sLI + r * kLP + c4), b_lo);
+            put4(r, 32 + c4, make_float4(0.f, 0.f, 0.f, 0.f), b_hi);
+            put4(32 + r, 32 + c4, *reinterpret_cast<const float4*>(sLI + (32 + r) * kLP + 32 + c4), b_hi);
         }
-        __syncthreads();
         KDA_TRACE_POINT(ptr_, 8192 + 19);
-        // Abar = INV diag(beta) as a K-major A image: row r = INV[r][.] scaled by beta
-        {
-            const int r = tid >> 2;
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const int chnk = 2 * (tid & 3) + h2;
-                const float4 i0 = *reinterpret_cast<const float4*>(sLI + r * kLP + 8 * chnk);
-                const float4 i1 = *reinterpret_cast<const float4*>(sLI + r * kLP + 8 * chnk + 4);
-                const float4 b0 = *reinterpret_cast<const float4*>(sBeta + 8 * chnk);
-                const float4 b1 = *reinterpret_cast<const float4*>(sBeta + 8 * chnk + 4);
-                const float e[8] = {i0.x * b0.x, i0.y * b0.y, i0.z * b0.z, i0.w * b0.w,
-                                    i1.x * b1.x, i1.y * b1.y, i1.z * b1.z, i1.w * b1.w};
-                *reinterpret_cast<uint4*>(sm + S::ABAR + sw128_off(r, chnk)) = pack_bf16x8(e);
-            }
-        }
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -620,7 +635,7 @@ done:
     tc_fence_before();
     __syncthreads();
     KDA_TRACE_POINT(ptr_, 8192 + 7);
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kPrepTmemCols);
     }
@@ -849,16 +864,15 @@ constexpr uint32_t kOutTmemCols = 128;
 constexpr uint32_t kOutTx = 16384 + kStateImgBytes + 16384;
 
 __global__ void __launch_bounds__(kOutThreads)
-out_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* __restrict__ off,
+out_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __restrict__ tab,
            const uint8_t* __restrict__ records, const uint8_t* __restrict__ states,
            __nv_bfloat16* __restrict__ out) {
     using S = OutSmem;
     const int c = blockIdx.x, h = blockIdx.y;
     const int total_chunks = off[num_seqs];
+    const int2 e = tab[c];   // in bounds for every c < max_chunks; meaningful for c < total
     if (c >= total_chunks) return;
-    const int n = find_seq(off, num_seqs, c);
-    const int t0 = cu[n] + (c - off[n]) * C;
-    const int nrow = min(C, cu[n + 1] - t0);
+    const int t0 = e.x, nrow = e.y;
     const uint8_t* rec = records + ((size_t)c * H + h) * kRecBytes;
     const uint8_t* simg = states + ((size_t)c * H + h) * kStateImgBytes;
 
@@ -960,13 +974,14 @@ inline bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, 
 
 struct Workspace {
     int32_t* off;
+    int2* tab;
     uint8_t* records;
     uint8_t* states;
 };
 inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs, int H) {
     uint8_t* base = static_cast<uint8_t*>(workspace);
-    return {reinterpret_cast<int32_t*>(base), base + ws_records_offset(num_seqs),
-            base + ws_states_offset(total, num_seqs, H)};
+    return {reinterpret_cast<int32_t*>(base), reinterpret_cast<int2*>(base + ws_table_offset(num_seqs)),
+            base + ws_records_offset(total, num_seqs), base + ws_states_offset(total, num_seqs, H)};
 }
 
 // Chunk table + chunk-parallel preparation.
@@ -977,7 +992,7 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
     cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepSmem::BYTES);
     if (e != cudaSuccess) return e;
-    chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off);
+    chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off, w.tab);
     if (total > 0) {
         CUtensorMap tq, tk, tv, tg;
         if (!make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -986,8 +1001,8 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
             !make_tmap(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
         dim3 grid((unsigned)max_chunks(total, num_seqs), (unsigned)H);
-        prep_kernel<<<grid, kPrepThreads, PrepSmem::BYTES, stream>>>(tq, tk, tv, tg, beta, cu,
-                                                                     num_seqs, H, w.off, w.records);
+        prep_kernel<<<grid, kPrepThreads, PrepSmem::BYTES, stream>>>(tq, tk, tv, tg, beta, num_seqs,
+                                                                     H, w.off, w.tab, w.records);
     }
     return cudaGetLastError();
 }
@@ -1013,7 +1028,7 @@ inline cudaError_t launch_output(void* out, const int32_t* cu, int num_seqs, int
                                          (int)OutSmem::BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)max_chunks(total, num_seqs), (unsigned)H);
-    out_kernel<<<grid, kOutThreads, OutSmem::BYTES, stream>>>(cu, num_seqs, H, w.off, w.records,
+    out_kernel<<<grid, kOutThreads, OutSmem::BYTES, stream>>>(num_seqs, H, w.off, w.tab, w.records,
                                                                w.states, static_cast<__nv_bfloat16*>(out));
     return cudaGetLastError();
 }
