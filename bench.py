@@ -292,11 +292,9 @@ def bench_prefill(args, P, dev, stream, world, peaks):
         stages = [
             ("prep_kernel", lambda: kda.kda_prefill_prepare(d["q"], d["k"], d["v"], d["g"], d["beta"],
                                                             d["cu_seqlens"], ws, C=C, stream=stream)),
-            ("rec_kernel", lambda: kda.kda_prefill_scan(d["cu_seqlens"], T, H, D, ws,
+            ("rec_kernel", lambda: kda.kda_prefill_scan(P["out"], d["cu_seqlens"], ws,
                                                         initial_state=d["s0"], final_state=P["fin"],
                                                         C=C, stream=stream)),
-            ("out_kernel", lambda: kda.kda_prefill_output(P["out"], d["cu_seqlens"], ws, C=C,
-                                                          stream=stream)),
         ]
         for _ in range(args.warmup):
             for _, f in stages:

@@ -12,8 +12,8 @@
 // so the serial chain carries ONE tensor-core product per chunk (M S_in), and the output
 // product (P S_in) runs beside it.
 //
-//   chunk_index_kernel  cu_seqlens -> first chunk of every sequence (device side, no host
-//                       sync); validates cu_seqlens.
+//   chunk_index_kernel  cu_seqlens -> first chunk of every sequence and the chunk table
+//                       (first token, rows) (device side, no host sync); validates cu_seqlens.
 //   prep_kernel         one CTA of 8 warps per (chunk, head), fully parallel, 2 CTAs per SM:
 //                         TMA: q, k, v tiles (128-byte swizzled) and g into shared memory
 //                         a, gamma, Q_dec = q e^a, K_dec = k e^a, K_inv = k e^-a      (FFMA/MUFU)
@@ -27,8 +27,9 @@
 //                       and writes one record per (chunk, head): the shared-memory
 //                       operand images of M and P, value-channel slices of B and R, gamma.
 //   rec_kernel          one CTA per (sequence, head, 64 value channels): the chunk chain
-//                       with the fp32 state slice in registers; a loader warp streams the
-//                       records in (2 stages of bulk copies) and an issuer warp launches the
+//                       with the fp32 state slice in registers and, beside it, the chunk
+//                       outputs O = P S_in + R; two loader warps stream the records in (bulk
+//                       copies into rings of 3 and 2 stages) and an issuer warp launches the
 //                       tensor-core products, hand-offs through mbarriers only.
 #pragma once
 
@@ -55,9 +56,6 @@ constexpr uint32_t kRecB = 49152;       // B  [slice][i 128][64] bf16, rows swiz
 constexpr uint32_t kRecR = 81920;       // R  [slice][r 64][64]  bf16, rows swizzled (2 x 8 KB)
 constexpr uint32_t kRecGamma = 98304;   // gamma fp32 [128]
 constexpr uint32_t kRecBytes = 98816;
-// bf16 state entering each (chunk, head): 2 slices of the MN-major image [i 128][64], 128-byte
-// swizzle, written by the recurrence and read by the output kernel.
-constexpr uint32_t kStateImgBytes = 32768;
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -65,7 +63,7 @@ __host__ inline int64_t max_chunks(int64_t total_tokens, int num_seqs) {
     return total_tokens / C + num_seqs;
 }
 // Workspace: [chunk offsets int32 (N+1)] [chunk table int2 (max_chunks)] [records
-// (max_chunks x H)] [chunk states (max_chunks x H)]
+// (max_chunks x H)]
 __host__ inline size_t ws_table_offset(int num_seqs) {
     return align_up(sizeof(int32_t) * (size_t)(num_seqs + 1), 16);
 }
@@ -73,13 +71,9 @@ __host__ inline size_t ws_records_offset(int64_t total_tokens, int num_seqs) {
     return align_up(ws_table_offset(num_seqs) + sizeof(int2) * (size_t)max_chunks(total_tokens, num_seqs),
                     1024);
 }
-__host__ inline size_t ws_states_offset(int64_t total_tokens, int num_seqs, int H) {
+__host__ inline size_t workspace_bytes(int64_t total_tokens, int num_seqs, int H) {
     return ws_records_offset(total_tokens, num_seqs) +
            (size_t)max_chunks(total_tokens, num_seqs) * H * kRecBytes;
-}
-__host__ inline size_t workspace_bytes(int64_t total_tokens, int num_seqs, int H) {
-    return ws_states_offset(total_tokens, num_seqs, H) +
-           (size_t)max_chunks(total_tokens, num_seqs) * H * kStateImgBytes;
 }
 
 // ------------------------------------------------------------------ chunk index
@@ -641,55 +635,76 @@ done:
     }
 }
 
-// ------------------------------------------------------------------ chunk recurrence
+// ------------------------------------------------------------------ chunk recurrence + outputs
+// One CTA per (sequence, head, 64 value channels).  Per chunk, the issuer launches two
+// tensor-core products reading the same bf16 image of S_in:
+//   D_S = M S_in   (128 x 64, K = 128)  -> S_out = gamma S_in + D_S + B  (the serial chain)
+//   D_O = P S_in   ( 64 x 64, K = 128)  -> O = D_O + R                   (beside the chain)
 // warps 0-7: state (warp w: rows 32 (w % 4) .. +31 = its TMEM lanes, columns 32 (w / 4) .. +31
-// of the slice); warp 8: loader; warp 9: MMA issuer
-constexpr int kRecThreads = 320;
+// of the slice), then this chunk's output rows 16 (w % 4) .. +15 (the M = 64 accumulator
+// puts row r in lane 32 (r / 16) + r % 16); warp 8: loader of M, B, gamma (3 stages);
+// warp 9: issuer of D_S; warp 10: loader of P, R (2 stages); warp 11: issuer of D_O.  The
+// two issuers are separate threads so that a late P never holds back the chain's product.
+constexpr int kRecThreads = 384;
 constexpr int kRecComputeWarps = 8;
-constexpr int kLoaderWarp = 8, kIssuerWarp = 9;
-constexpr int kStages = 3;
+constexpr int kLoaderWarp = 8, kIssuerWarp = 9, kLoaderOWarp = 10, kIssuerOWarp = 11;
+constexpr int kStagesA = 3, kStagesB = 2;
 constexpr uint32_t kStM = 0;          // M, both K blocks (32 KB)
 constexpr uint32_t kStB = 32768;      // B slice [128][64] bf16 (rows swizzled)
-constexpr uint32_t kStG = 49152;      // gamma [128]
-constexpr uint32_t kStageLoad = 49664;
-constexpr uint32_t kStageBytes = 50176;
+constexpr uint32_t kStageA = 49152;
+constexpr uint32_t kStP = 0;          // P, both K blocks (16 KB)
+constexpr uint32_t kStR = 16384;      // R slice [64][64] bf16 (rows swizzled)
+constexpr uint32_t kStageB = 24576;
 struct RecSmem {
-    static constexpr uint32_t SB = kStages * kStageBytes;   // S (bf16) B images, 2 x 16 KB
-    static constexpr uint32_t BAR = SB + 2 * 16384;         // full[3] empty[3] mma_s sb_ready[2]
-    static constexpr uint32_t TMEM = BAR + 9 * 8;
+    static constexpr uint32_t RB = kStagesA * kStageA;       // ring of P / R stages
+    static constexpr uint32_t SB = RB + kStagesB * kStageB;  // S (bf16) B images, 2 x 16 KB
+    static constexpr uint32_t GAM = SB + 2 * 16384;          // gamma [stage][128] fp32
+    // fullA[3] emptyA[3] fullB[2] emptyB[2] mma_s mma_o[2] ofree[2] sbr[2]
+    static constexpr uint32_t BAR = GAM + kStagesA * 512;
+    static constexpr uint32_t TMEM = BAR + 17 * 8;
     static constexpr uint32_t FLAG = TMEM + 4;
     static constexpr uint32_t BYTES = FLAG + 4 + 1024;
 };
-constexpr uint32_t kRecTmemCols = 64;   // D_S
+static_assert(RecSmem::BYTES <= 232448, "recurrence shared memory exceeds 227 KB");
+constexpr uint32_t kRecTmemCols = 256;  // D_S [0, 64), D_O buffers [64, 128), [128, 192)
+constexpr uint32_t kTxA = 32768 + 16384 + 512;
+constexpr uint32_t kTxB = 16384 + 8192;
 
 __global__ void __launch_bounds__(kRecThreads, 1)
-rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* __restrict__ off,
-           const uint8_t* __restrict__ records, uint8_t* __restrict__ states,
-           const float* initial_state, float* final_state) {
+rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __restrict__ tab,
+           const uint8_t* __restrict__ records, const float* initial_state, float* final_state,
+           __nv_bfloat16* __restrict__ out) {
     using S = RecSmem;
     const int sl = blockIdx.x % NSL;
     const int h = (blockIdx.x / NSL) % H;
     const int n = blockIdx.x / (NSL * H);
     const int c_begin = off[n], nchunks = off[n + 1] - c_begin;
+    (void)num_seqs;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     const uint32_t sb = smem_u32(sm);
     // Each barrier's waiters can never fall two phases behind: its next phase needs an
     // arrival that every waiter of the current phase precedes.
-    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 24, mma_s = full0 + 48, sbr0 = full0 + 56;
+    const uint32_t fullA = sb + S::BAR, emptyA = fullA + 24, fullB = fullA + 48, emptyB = fullA + 64;
+    const uint32_t mma_s = fullA + 80, mma_o = fullA + 88, ofree = fullA + 104, sbr0 = fullA + 120;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + S::FLAG);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (warp == 0) tmem_alloc(sb + S::TMEM, kRecTmemCols);
     if (tid == 0) {
-        for (int st = 0; st < kStages; ++st) {
-            mbar_init(full0 + 8 * st, 1);
-            mbar_init(empty0 + 8 * st, kRecComputeWarps);
+        for (int st = 0; st < kStagesA; ++st) {
+            mbar_init(fullA + 8 * st, 1);
+            mbar_init(emptyA + 8 * st, kRecComputeWarps);
+        }
+        for (int st = 0; st < kStagesB; ++st) {
+            mbar_init(fullB + 8 * st, 1);
+            mbar_init(emptyB + 8 * st, kRecComputeWarps);
+            mbar_init(mma_o + 8 * st, 1);
+            mbar_init(ofree + 8 * st, kRecComputeWarps);
+            mbar_init(sbr0 + 8 * st, kRecComputeWarps);
         }
         mbar_init(mma_s, 1);
-        mbar_init(sbr0, kRecComputeWarps);
-        mbar_init(sbr0 + 8, kRecComputeWarps);
         fence_mbar_init();
         *abort_flag = 0;
     }
@@ -698,69 +713,110 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
     tc_fence_after();
     const uint32_t tS = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
 
-    if (warp == kLoaderWarp) {
-        // ---------------- loader: M, this slice of B, gamma of every chunk -----------------
+    if (warp == kLoaderWarp || warp == kLoaderOWarp) {
+        // ---------------- loaders: ring A (M, B slice, gamma), ring B (P, R slice) ----------
         if (lane == 0) {
+            const bool ring_a = warp == kLoaderWarp;
+            const int nst = ring_a ? kStagesA : kStagesB;
+            const uint32_t full = ring_a ? fullA : fullB, empty = ring_a ? emptyA : emptyB;
             int issued = 0;
             for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
-                const int st = kk % kStages, use = kk / kStages;
-                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 0);
-                if (use > 0 && !mbar_wait(empty0 + 8 * st, (use - 1) & 1)) {
+                const int st = kk % nst, use = kk / nst;
+                KDA_TRACE_POINT(ring_a && blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 0);
+                if (use > 0 && !mbar_wait(empty + 8 * st, (use - 1) & 1)) {
                     kda_set_status(KDA_ERR_TIMEOUT);
                     *abort_flag = 1;
                     break;
                 }
                 const uint8_t* rec = records + ((size_t)(c_begin + kk) * H + h) * kRecBytes;
-                const uint32_t dst = sb + st * kStageBytes;
-                const uint32_t fb = full0 + 8 * st;
-                mbar_arrive_expect_tx(fb, kStageLoad);
-                bulk_g2s(dst + kStM, rec + kRecM0, 16384, fb);
-                bulk_g2s(dst + kStM + 16384, rec + kRecM0 + 16384, 16384, fb);
-                bulk_g2s(dst + kStB, rec + kRecB + sl * 16384, 16384, fb);
-                bulk_g2s(dst + kStG, rec + kRecGamma, 512, fb);
-                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 1);
+                const uint32_t fb = full + 8 * st;
+                if (ring_a) {
+                    const uint32_t dst = sb + st * kStageA;
+                    mbar_arrive_expect_tx(fb, kTxA);
+                    bulk_g2s(dst + kStM, rec + kRecM0, 32768, fb);
+                    bulk_g2s(dst + kStB, rec + kRecB + sl * 16384, 16384, fb);
+                    bulk_g2s(sb + S::GAM + st * 512, rec + kRecGamma, 512, fb);
+                    // everything this CTA will read of the record kStagesA chunks ahead goes to
+                    // L2 now, so that those copies are served from L2
+                    if (kk + kStagesA < nchunks) {
+                        const uint8_t* ahead = rec + (size_t)kStagesA * H * kRecBytes;
+                        bulk_prefetch_l2(ahead + kRecP0, 16384 + 32768);
+                        bulk_prefetch_l2(ahead + kRecB + sl * 16384, 16384);
+                        bulk_prefetch_l2(ahead + kRecR + sl * 8192, 8192);
+                        bulk_prefetch_l2(ahead + kRecGamma, 512);
+                    }
+                } else {
+                    const uint32_t dst = sb + S::RB + st * kStageB;
+                    mbar_arrive_expect_tx(fb, kTxB);
+                    bulk_g2s(dst + kStP, rec + kRecP0, 16384, fb);
+                    bulk_g2s(dst + kStR, rec + kRecR + sl * 8192, 8192, fb);
+                }
+                KDA_TRACE_POINT(ring_a && blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 1);
                 ++issued;
             }
             // never leave with copies in flight: wait (bounded) for the last stages filled
-            for (int kk = max(0, issued - kStages); kk < issued; ++kk)
-                mbar_wait(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
+            for (int kk = max(0, issued - nst); kk < issued; ++kk)
+                mbar_wait(full + 8 * (kk % nst), (kk / nst) & 1);
         }
     } else if (warp == kIssuerWarp) {
-        // ---------------- MMA issuer: D_S = M S_in once the stage and S_in are ready --------
+        // ---------------- issuer of D_S = M S_in, once the stage and S_in are ready --------
         if (lane == 0) {
-            constexpr uint32_t id = idesc_bf16(128, NV, false, true);
+            constexpr uint32_t idS = idesc_bf16(128, NV, false, true);
             for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
-                const int st = kk % kStages;
-                if (!mbar_wait(full0 + 8 * st, (kk / kStages) & 1) ||
+                const int st = kk % kStagesA;
+                const uint32_t sbuf = sb + S::SB + (kk & 1) * 16384;
+                if (!mbar_wait(fullA + 8 * st, (kk / kStagesA) & 1) ||
                     !mbar_wait(sbr0 + 8 * (kk & 1), (kk >> 1) & 1)) {
                     kda_set_status(KDA_ERR_TIMEOUT);
                     *abort_flag = 1;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t stage = sb + st * kStageBytes;
-                const uint32_t sbuf = sb + S::SB + (kk & 1) * 16384;
-                // the other S buffer is rewritten after this chunk's product completes: its
-                // copy to the workspace (issued one chunk ago) must have read it by then
-                bulk_wait_read<0>();
+                const uint32_t stage = sb + st * kStageA;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t ko = (ks >> 2) * 16384 + (ks & 3) * 32;
                     umma_bf16(tS, smem_desc(stage + kStM + ko, 16, 1024, kSwizzle128),
-                              smem_desc(sbuf + ks * 2048, 16, 1024, kSwizzle128), id, ks > 0);
+                              smem_desc(sbuf + ks * 2048, 16, 1024, kSwizzle128), idS, ks > 0);
                 }
                 umma_commit(mma_s);
-                // the state entering chunk kk, for the output kernel
-                bulk_s2g(states + ((size_t)(c_begin + kk) * H + h) * kStateImgBytes + sl * 16384,
-                         sbuf, 16384);
+                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 2);
             }
-            bulk_wait_all();
+        }
+    } else if (warp == kIssuerOWarp) {
+        // ---------------- issuer of D_O = P S_in into output buffer kk % 2, once P and S_in
+        // are in and the output rows of chunk kk - 2 have left that buffer.  S_in's image
+        // stays put until this product is done: the state warps overwrite it only after
+        // they have drained D_O.
+        if (lane == 0) {
+            constexpr uint32_t idO = idesc_bf16(64, NV, false, true);
+            for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
+                const int so = kk & 1;
+                const uint32_t sbuf = sb + S::SB + (kk & 1) * 16384;
+                if (!mbar_wait(fullB + 8 * so, (kk >> 1) & 1) ||
+                    !mbar_wait(sbr0 + 8 * (kk & 1), (kk >> 1) & 1) ||
+                    (kk >= 2 && !mbar_wait(ofree + 8 * so, ((kk - 2) >> 1) & 1))) {
+                    kda_set_status(KDA_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t pst = sb + S::RB + so * kStageB;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t ko = (ks >> 2) * 8192 + (ks & 3) * 32;
+                    umma_bf16(tS + 64 + 64 * so, smem_desc(pst + kStP + ko, 16, 1024, kSwizzle128),
+                              smem_desc(sbuf + ks * 2048, 16, 1024, kSwizzle128), idO, ks > 0);
+                }
+                umma_commit(mma_o + 8 * so);
+                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 3);
+            }
         }
     } else {
         // ---------------- state: row i, columns 32 cw .. 32 cw + 31 of the slice -----------
         constexpr int NC = NV / 2;   // columns per thread
-        const int i = 32 * (warp & 3) + lane, cw = warp >> 2;
-        const uint32_t taw = (uint32_t)(32 * (warp & 3)) << 16;
+        const int q4 = warp & 3, i = 32 * q4 + lane, cw = warp >> 2;
+        const uint32_t taw = (uint32_t)(32 * q4) << 16;
         const size_t sbase = (((size_t)n * H + h) * D + i) * D + (size_t)sl * NV + NC * cw;
         float Sr[NC];
         if (initial_state) {
@@ -773,8 +829,7 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
 #pragma unroll
             for (int j = 0; j < NC; ++j) Sr[j] = 0.f;
         }
-        // bf16 image of the state entering the next chunk (B operand of its product; the
-        // issuer also copies it to the workspace for the output kernel)
+        // bf16 image of the state entering the next chunk (B operand of both products)
         auto put_state = [&](uint32_t buf) {
 #pragma unroll
             for (int cb = 0; cb < NC / 8; ++cb)
@@ -786,17 +841,19 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
         if (lane == 0) mbar_arrive(sbr0);
 
         bool ok = true;
+        const int r_out = 16 * q4 + lane;   // output row of this lane (lanes 0-15)
         for (int kk = 0; kk < nchunks; ++kk) {
-            const int st = kk % kStages;
-            const uint8_t* stage_p = sm + st * kStageBytes;
+            const int st = kk % kStagesA, so = kk & 1;
             const bool tr = blockIdx.x == 0 && tid == 0 && kk < 256;
             (void)tr;
+            const int2 ce = tab[c_begin + kk];   // (first token, rows) of this chunk
             KDA_TRACE_POINT(tr, kk * 8 + 0);
-            ok = __all_sync(0xffffffffu, mbar_wait(full0 + 8 * st, (kk / kStages) & 1));
+            ok = __all_sync(0xffffffffu, mbar_wait(fullA + 8 * st, (kk / kStagesA) & 1));
             if (!ok || *abort_flag) { ok = false; break; }
             KDA_TRACE_POINT(tr, kk * 8 + 1);
             // this chunk's gamma and B row, before the serial product lands
-            const float gam = reinterpret_cast<const float*>(stage_p + kStG)[i];
+            const float gam = reinterpret_cast<const float*>(sm + S::GAM + st * 512)[i];
+            const uint8_t* stage_p = sm + st * kStageA;
             uint4 bq[NC / 8];
 #pragma unroll
             for (int cb = 0; cb < NC / 8; ++cb)
@@ -806,17 +863,19 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
             if (!ok) break;
             KDA_TRACE_POINT(tr, kk * 8 + 3);
             tc_fence_after();
-            float dsv[NC];
-            tmem_ld32(tS + taw + NC * cw, dsv);
-            tmem_wait_ld();
+            {
+                float dsv[NC];
+                tmem_ld32(tS + taw + NC * cw, dsv);
+                tmem_wait_ld();
 #pragma unroll
-            for (int cb = 0; cb < NC / 8; ++cb) {
-                float bv[8];
-                unpack_bf16x8(bq[cb], bv);
+                for (int cb = 0; cb < NC / 8; ++cb) {
+                    float bv[8];
+                    unpack_bf16x8(bq[cb], bv);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int j = 8 * cb + u;
-                    Sr[j] = fmaf(gam, Sr[j], dsv[j] + bv[u]);
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = 8 * cb + u;
+                        Sr[j] = fmaf(gam, Sr[j], dsv[j] + bv[u]);
+                    }
                 }
             }
             KDA_TRACE_POINT(tr, kk * 8 + 4);
@@ -826,9 +885,51 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(sbr0 + 8 * ((kk + 1) & 1));
-                mbar_arrive(empty0 + 8 * st);
+                mbar_arrive(emptyA + 8 * st);
             }
             KDA_TRACE_POINT(tr, kk * 8 + 5);
+            // output rows 16 q4 .. 16 q4 + 15, columns 32 cw .. +31 of the slice: O = D_O + R
+            // (the R slice is read after this warp has itself seen the stage's copies land)
+            ok = __all_sync(0xffffffffu, mbar_wait(fullB + 8 * so, (kk >> 1) & 1) &&
+                                             mbar_wait(mma_o + 8 * so, (kk >> 1) & 1));
+            if (!ok) break;
+            KDA_TRACE_POINT(tr, kk * 8 + 7);
+            tc_fence_after();
+            float dov[NC];
+            tmem_ld32(tS + taw + 64 + 64 * so + NC * cw, dov);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ofree + 8 * so);
+            // O = D_O + R in place of this warp's own R entries (rows 16 q4 .. +15, 16-byte
+            // chunks 4 cw .. 4 cw + 3 of the slice), then re-read so that four lanes store one
+            // row's 64 contiguous bytes: each store instruction covers 8 rows.
+            uint8_t* rs = sm + S::RB + so * kStageB + kStR;
+            if (lane < 16) {
+#pragma unroll
+                for (int qq = 0; qq < NC / 8; ++qq) {
+                    uint4* p = reinterpret_cast<uint4*>(rs + sw128_off(r_out, 4 * cw + qq));
+                    float rv[8];
+                    unpack_bf16x8(*p, rv);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) rv[u] += dov[8 * qq + u];
+                    *p = pack_bf16x8(rv);
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+                const int rr = 16 * q4 + 8 * g8 + (lane >> 2), cc = lane & 3;
+                if (rr < ce.y) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(rs + sw128_off(rr, 4 * cw + cc));
+                    *reinterpret_cast<uint4*>(out + ((size_t)(ce.x + rr) * H + h) * D + sl * NV + NC * cw +
+                                              8 * cc) = v;
+                }
+            }
+            fence_proxy_async_smem();   // the slot is next written by a bulk copy
+            __syncwarp();
+            if (lane == 0) mbar_arrive(emptyB + 8 * so);
+            KDA_TRACE_POINT(tr, kk * 8 + 6);
         }
         if (!ok) {
             if (lane == 0) kda_set_status(KDA_ERR_TIMEOUT);
@@ -845,97 +946,6 @@ rec_kernel(const int32_t* __restrict__ cu, int num_seqs, int H, const int32_t* _
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tS, kRecTmemCols);
-    }
-}
-
-// ------------------------------------------------------------------ chunk outputs
-// One CTA per (chunk, head), fully parallel: O = [P ; *] S_in + R from the record and the
-// state image the recurrence left for this chunk.
-constexpr int kOutThreads = 128;
-struct OutSmem {
-    static constexpr uint32_t A = 0;         // P0 | P1 | 8 KB of filler rows (never read back)
-    static constexpr uint32_t SI = 24576;    // state image, 2 slices (32 KB)
-    static constexpr uint32_t RR = 57344;    // R, 2 slices (16 KB)
-    static constexpr uint32_t BAR = 73728;
-    static constexpr uint32_t TMEM = BAR + 8;
-    static constexpr uint32_t BYTES = TMEM + 8 + 1024;
-};
-constexpr uint32_t kOutTmemCols = 128;
-constexpr uint32_t kOutTx = 16384 + kStateImgBytes + 16384;
-
-__global__ void __launch_bounds__(kOutThreads)
-out_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __restrict__ tab,
-           const uint8_t* __restrict__ records, const uint8_t* __restrict__ states,
-           __nv_bfloat16* __restrict__ out) {
-    using S = OutSmem;
-    const int c = blockIdx.x, h = blockIdx.y;
-    const int total_chunks = off[num_seqs];
-    const int2 e = tab[c];   // in bounds for every c < max_chunks; meaningful for c < total
-    if (c >= total_chunks) return;
-    const int t0 = e.x, nrow = e.y;
-    const uint8_t* rec = records + ((size_t)c * H + h) * kRecBytes;
-    const uint8_t* simg = states + ((size_t)c * H + h) * kStateImgBytes;
-
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
-    const uint32_t sb = smem_u32(sm);
-    const uint32_t bar = sb + S::BAR;
-    const int tid = threadIdx.x, warp = tid >> 5;
-
-    if (warp == 0) tmem_alloc(sb + S::TMEM, kOutTmemCols);
-    if (tid == 0) {
-        mbar_init(bar, 1);
-        fence_mbar_init();
-        mbar_arrive_expect_tx(bar, kOutTx);
-        bulk_g2s(sb + S::A, rec + kRecP0, 16384, bar);
-        bulk_g2s(sb + S::SI, simg, kStateImgBytes, bar);
-        bulk_g2s(sb + S::RR, rec + kRecR, 16384, bar);
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
-    bool ok = mbar_wait(bar, 0);
-    if (tid == 0 && ok) {
-        constexpr uint32_t id = idesc_bf16(128, 128, false, true);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-            umma_bf16(tmem, smem_desc(sb + S::A + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128),
-                      smem_desc(sb + S::SI + ks * 2048, 16384, 1024, kSwizzle128), id, ks > 0);
-        umma_commit(bar);
-    }
-    ok = ok && mbar_wait(bar, 1);
-    tc_fence_after();
-    if (__syncthreads_or(!ok)) {
-        if (tid == 0) kda_set_status(KDA_ERR_TIMEOUT);
-    } else if (warp < 2) {
-        const int r = tid;
-        const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            float d[32];
-            tmem_ld32(ta + 32 * cb, d);
-            tmem_wait_ld();
-            if (r < nrow) {
-                const int slc = cb >> 1;
-                uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * H + h) * D + 32 * cb);
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    float rv[8];
-                    unpack_bf16x8(*reinterpret_cast<const uint4*>(
-                                      sm + S::RR + slc * 8192 + sw128_off(r, (cb & 1) * 4 + qq)), rv);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) rv[u] += d[8 * qq + u];
-                    dst[qq] = pack_bf16x8(rv);
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, kOutTmemCols);
     }
 }
 
@@ -976,19 +986,18 @@ struct Workspace {
     int32_t* off;
     int2* tab;
     uint8_t* records;
-    uint8_t* states;
 };
-inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs, int H) {
+inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs) {
     uint8_t* base = static_cast<uint8_t*>(workspace);
     return {reinterpret_cast<int32_t*>(base), reinterpret_cast<int2*>(base + ws_table_offset(num_seqs)),
-            base + ws_records_offset(total, num_seqs), base + ws_states_offset(total, num_seqs, H)};
+            base + ws_records_offset(total, num_seqs)};
 }
 
 // Chunk table + chunk-parallel preparation.
 inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, const int32_t* cu, int num_seqs,
                                   int64_t total, int H, void* workspace, cudaStream_t stream) {
-    const Workspace w = split_workspace(workspace, total, num_seqs, H);
+    const Workspace w = split_workspace(workspace, total, num_seqs);
     cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepSmem::BYTES);
     if (e != cudaSuccess) return e;
@@ -1007,29 +1016,15 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
     return cudaGetLastError();
 }
 
-// Chunk-serial recurrence over every (sequence, head, value slice).
-inline cudaError_t launch_scan(const float* s0, float* sf, const int32_t* cu, int num_seqs,
-                               int64_t total, int H, void* workspace, cudaStream_t stream) {
-    const Workspace w = split_workspace(workspace, total, num_seqs, H);
+// Chunk-serial recurrence and the chunk outputs, over every (sequence, head, value slice).
+inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_seqs, int64_t total,
+                               int H, void* workspace, cudaStream_t stream) {
+    const Workspace w = split_workspace(workspace, total, num_seqs);
     cudaError_t e = cudaFuncSetAttribute(rec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)RecSmem::BYTES);
     if (e != cudaSuccess) return e;
     rec_kernel<<<(unsigned)num_seqs * H * NSL, kRecThreads, RecSmem::BYTES, stream>>>(
-        cu, num_seqs, H, w.off, w.records, w.states, s0, sf);
-    return cudaGetLastError();
-}
-
-// Chunk-parallel outputs.
-inline cudaError_t launch_output(void* out, const int32_t* cu, int num_seqs, int64_t total, int H,
-                                 void* workspace, cudaStream_t stream) {
-    if (total == 0) return cudaSuccess;
-    const Workspace w = split_workspace(workspace, total, num_seqs, H);
-    cudaError_t e = cudaFuncSetAttribute(out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)OutSmem::BYTES);
-    if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)max_chunks(total, num_seqs), (unsigned)H);
-    out_kernel<<<grid, kOutThreads, OutSmem::BYTES, stream>>>(num_seqs, H, w.off, w.tab, w.records,
-                                                               w.states, static_cast<__nv_bfloat16*>(out));
+        num_seqs, H, w.off, w.tab, w.records, s0, sf, static_cast<__nv_bfloat16*>(out));
     return cudaGetLastError();
 }
 
@@ -1038,8 +1033,7 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
                                   int num_seqs, int64_t total, int H, void* out, float* sf,
                                   void* workspace, cudaStream_t stream) {
     cudaError_t e = launch_prepare(q, k, v, g, beta, cu, num_seqs, total, H, workspace, stream);
-    if (e == cudaSuccess) e = launch_scan(s0, sf, cu, num_seqs, total, H, workspace, stream);
-    if (e == cudaSuccess) e = launch_output(out, cu, num_seqs, total, H, workspace, stream);
+    if (e == cudaSuccess) e = launch_scan(s0, sf, out, num_seqs, total, H, workspace, stream);
     return e;
 }
 

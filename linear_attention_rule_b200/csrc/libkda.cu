@@ -45,7 +45,7 @@ cudaError_t dispatch_simt(int32_t dk, int32_t C, const void* q, const void* k, c
 
 extern "C" {
 
-int32_t kda_abi_version(void) { return 1; }
+int32_t kda_abi_version(void) { return 2; }
 
 const char* kda_status_string(kda_status s) {
     switch (s) {
@@ -137,7 +137,7 @@ kda_status kda_prefill_prepare(const void* q, const void* k, const void* v, cons
                ? KDA_OK : KDA_ERR_CUDA;
 }
 
-kda_status kda_prefill_scan(const float* initial_state, float* final_state,
+kda_status kda_prefill_scan(const float* initial_state, float* final_state, void* out,
                             const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                             int32_t H, int32_t dk, int32_t dv, kda_dtype dt, int32_t C,
                             void* workspace, size_t ws_bytes, kda_stream_t stream) {
@@ -145,20 +145,9 @@ kda_status kda_prefill_scan(const float* initial_state, float* final_state,
     if (st != KDA_OK || num_seqs == 0) return st;
     if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
         return KDA_ERR_INVALID_ARG;
-    return kda::tc::launch_scan(initial_state, final_state, cu_seqlens, num_seqs, total_tokens, H,
-                                workspace, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? KDA_OK : KDA_ERR_CUDA;
-}
-
-kda_status kda_prefill_output(void* out, const int32_t* cu_seqlens, int32_t num_seqs,
-                              int64_t total_tokens, int32_t H, int32_t dk, int32_t dv,
-                              kda_dtype dt, int32_t C, void* workspace, size_t ws_bytes,
-                              kda_stream_t stream) {
-    kda_status st = check_staged(cu_seqlens, num_seqs, total_tokens, H, dk, dv, dt, C, workspace, ws_bytes);
-    if (st != KDA_OK || num_seqs == 0) return st;
     if (total_tokens > 0 && (!out || !aligned16(out))) return KDA_ERR_INVALID_ARG;
-    return kda::tc::launch_output(out, cu_seqlens, num_seqs, total_tokens, H, workspace,
-                                  reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+    return kda::tc::launch_scan(initial_state, final_state, out, num_seqs, total_tokens, H,
+                                workspace, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -28,8 +28,7 @@ KDA_BF16 = 1
 # Every symbol include/libkda.h declares (checked by the CPU tests).
 EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_status_string",
             "kda_get_device_status", "kda_abi_version", "kda_prefill_noalloc",
-            "kda_prefill_prepare", "kda_prefill_scan", "kda_prefill_output",
-            "kda_selftest_bounded_wait")
+            "kda_prefill_prepare", "kda_prefill_scan", "kda_selftest_bounded_wait")
 
 # Size of the library-owned scratch behind kda_prefill_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -71,10 +70,8 @@ def load() -> ctypes.CDLL:
     lib.kda_prefill_prepare.argtypes = [P, P, P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, I32,
                                         P, SZ, P]
     lib.kda_prefill_prepare.restype = ctypes.c_int
-    lib.kda_prefill_scan.argtypes = [P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, I32, P, SZ, P]
+    lib.kda_prefill_scan.argtypes = [P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, I32, P, SZ, P]
     lib.kda_prefill_scan.restype = ctypes.c_int
-    lib.kda_prefill_output.argtypes = [P, P, I32, I64, I32, I32, I32, ctypes.c_int, I32, P, SZ, P]
-    lib.kda_prefill_output.restype = ctypes.c_int
     lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P]
     lib.kda_selftest_bounded_wait.restype = ctypes.c_int
     _lib = lib
@@ -182,27 +179,18 @@ def kda_prefill_prepare(q, k, v, g, beta, cu_seqlens, workspace, C: int = 64, st
         raise KdaError("kda_prefill_prepare", st)
 
 
-def kda_prefill_scan(cu_seqlens, total_tokens, H, D, workspace, initial_state=None,
-                     final_state=None, C: int = 64, stream=None):
-    """Stage 2: the chunk recurrence; reads/writes the states, fills chunk states in `workspace`."""
-    lib = load()
-    N = cu_seqlens.shape[0] - 1
-    st = lib.kda_prefill_scan(_ptr(initial_state), _ptr(final_state), _ptr(cu_seqlens), N,
-                              total_tokens, H, D, D, KDA_BF16, C, _ptr(workspace), _ws(workspace),
-                              _stream(stream))
-    if st != KDA_OK:
-        raise KdaError("kda_prefill_scan", st)
-
-
-def kda_prefill_output(out, cu_seqlens, workspace, C: int = 64, stream=None):
-    """Stage 3: the chunk outputs into `out` [T, H, D] bf16."""
+def kda_prefill_scan(out, cu_seqlens, workspace, initial_state=None, final_state=None,
+                     C: int = 64, stream=None):
+    """Stage 2: the chunk recurrence with the chunk outputs beside it; reads initial_state,
+    writes `out` [T, H, D] bf16 and final_state."""
     lib = load()
     T, H, D = out.shape
     N = cu_seqlens.shape[0] - 1
-    st = lib.kda_prefill_output(_ptr(out), _ptr(cu_seqlens), N, T, H, D, D, _dtype_code(out), C,
-                                _ptr(workspace), _ws(workspace), _stream(stream))
+    st = lib.kda_prefill_scan(_ptr(initial_state), _ptr(final_state), _ptr(out), _ptr(cu_seqlens), N,
+                              T, H, D, D, _dtype_code(out), C, _ptr(workspace), _ws(workspace),
+                              _stream(stream))
     if st != KDA_OK:
-        raise KdaError("kda_prefill_output", st)
+        raise KdaError("kda_prefill_scan", st)
 
 
 def kda_selftest_bounded_wait(limit_ns: int, stream=None):

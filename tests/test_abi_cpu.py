@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert kda.kda_abi_version() == 1
+    assert kda.kda_abi_version() == 2
     for code in range(6):
         s = kda.kda_status_string(code)
         assert s and s != "unknown status"
@@ -110,14 +110,19 @@ def test_staged_entry_points_reject_bad_arguments(lib):
     # only the tensor-core problem is staged
     assert lib.kda_prefill_prepare(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), 1, 256, 2,
                                    64, 64, kda.KDA_F32, 64, ws, need, None) == kda.KDA_ERR_UNSUPPORTED
-    assert lib.kda_prefill_scan(None, None, P(4096), 1, 256, 2, 128, 128, kda.KDA_BF16, 64, ws,
+    out = P(8192)
+    assert lib.kda_prefill_scan(None, None, out, P(4096), 1, 256, 2, 128, 128, kda.KDA_BF16, 64, ws,
                                 need - 1, None) == kda.KDA_ERR_INVALID_ARG
-    assert lib.kda_prefill_output(None, P(4096), 1, 256, 2, 128, 128, kda.KDA_BF16, 64, ws, need,
-                                  None) == kda.KDA_ERR_INVALID_ARG
-    assert lib.kda_prefill_output(P(4096), P(4096), 1, 256, 2, 128, 128, kda.KDA_BF16, 64, P(4096 + 16),
-                                  need, None) == kda.KDA_ERR_INVALID_ARG
-    assert lib.kda_prefill_scan(None, None, P(4096), 0, 0, 2, 128, 128, kda.KDA_BF16, 64, ws, need,
-                                None) == kda.KDA_OK
+    # out is required once there are tokens, and must be 16-byte aligned
+    assert lib.kda_prefill_scan(None, None, None, P(4096), 1, 256, 2, 128, 128, kda.KDA_BF16, 64, ws,
+                                need, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_prefill_scan(None, None, P(8192 + 8), P(4096), 1, 256, 2, 128, 128, kda.KDA_BF16,
+                                64, ws, need, None) == kda.KDA_ERR_INVALID_ARG
+    # misaligned workspace
+    assert lib.kda_prefill_scan(None, None, out, P(4096), 1, 256, 2, 128, 128, kda.KDA_BF16, 64,
+                                P((1 << 20) + 16), need, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_prefill_scan(None, None, None, P(4096), 0, 0, 2, 128, 128, kda.KDA_BF16, 64, ws,
+                                need, None) == kda.KDA_OK
 
 
 def test_selftest_rejects_out_of_range_limits(lib):

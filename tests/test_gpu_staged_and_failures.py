@@ -21,8 +21,7 @@ def test_staged_prefill_equals_kda_prefill_bitwise():
     out = torch.empty(T, H, D, dtype=torch.bfloat16, device="cuda")
     fin = torch.empty(N, H, D, D, device="cuda")
     kda.kda_prefill_prepare(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], ws)
-    kda.kda_prefill_scan(d["cu_seqlens"], T, H, D, ws, initial_state=d["s0"], final_state=fin)
-    kda.kda_prefill_output(out, d["cu_seqlens"], ws)
+    kda.kda_prefill_scan(out, d["cu_seqlens"], ws, initial_state=d["s0"], final_state=fin)
     assert kda.kda_get_device_status() == kda.KDA_OK
     np.testing.assert_array_equal(out.double().cpu().numpy(), out_ref)
     np.testing.assert_array_equal(fin.double().cpu().numpy(), fin_ref)
