@@ -171,7 +171,7 @@ kda_status kda_selftest_bounded_wait(uint64_t limit_ns, kda_stream_t stream);
  *     kda_prefill with a NULL workspace instead).
  *   - A problem whose kda_prefill_workspace_size exceeds KDA_NOALLOC_SCRATCH_BYTES returns
  *     KDA_ERR_UNSUPPORTED before anything is launched (with H = 32 and one sequence that
- *     is anything beyond 1,343 tokens).
+ *     is anything beyond 1,471 tokens).
  *   - The first call on each device looks the scratch address up (cudaGetSymbolAddress,
  *     with that device current); make that first call before any stream capture begins.
  *   - All calls on a device share the one scratch array, which keeps whatever the last

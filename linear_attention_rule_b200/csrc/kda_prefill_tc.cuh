@@ -7,10 +7,11 @@
 //   U' = U - W S_in,   O = Q_dec S_in + Aqk U',   S_out = diag(gamma) S_in + K_res^T U'.
 // Substituting U' moves every product that does not involve S_in into the parallel
 // preparation:
-//   S_out = diag(gamma) S_in + M S_in + B,   M = -K_res^T W,   B = K_res^T U
-//   O     = P S_in + R,                      P = Q_dec - Aqk W, R = Aqk U
-// so the serial chain carries ONE tensor-core product per chunk (M S_in), and the output
-// product (P S_in) runs beside it.
+//   S_out = diag(gamma) S_in + M S_in + K_res^T U,   M = -K_res^T W
+//   O     = P S_in + Aqk U,                          P = Q_dec - Aqk W
+// so the serial chain carries ONE tensor-core product per chunk, [M | K_res^T] [S_in ; U]
+// (K = 128 + 64), and the output product [P | Aqk] [S_in ; U] runs beside it: the terms
+// without S_in ride in the same accumulators as extra K steps.
 //
 //   chunk_index_kernel  cu_seqlens -> first chunk of every sequence and the chunk table
 //                       (first token, rows) (device side, no host sync); validates cu_seqlens.
@@ -22,10 +23,10 @@
 //                         INV = (I + L)^-1: 16x16 diagonal blocks by forward substitution,
 //                                               then block doubling 16 -> 32 -> 64 (fp32)
 //                         [W | U] = INV diag(beta) [K_dec | V]                       (MMA 128x256x64)
-//                         [M | B] = [-K_res^T W | K_res^T U]                         (MMA 128x256x64)
-//                         [Aqk W | Aqk U] -> P, R                                    (MMA 128x256x64)
+//                         -M = K_res^T W                                             (MMA 128x128x64)
+//                         Aqk W -> P = Q_dec - Aqk W                                 (MMA 128x128x64)
 //                       and writes one record per (chunk, head): the shared-memory
-//                       operand images of M and P, value-channel slices of B and R, gamma.
+//                       operand images of P, M, K_res, U (2 value slices), Aqk, and gamma.
 //   rec_kernel          one CTA per (sequence, head, 64 value channels): the chunk chain
 //                       with the fp32 state slice in registers and, beside it, the chunk
 //                       outputs O = P S_in + R; two loader warps stream the records in (bulk
@@ -49,13 +50,16 @@ constexpr int NV = 64;   // value channels per recurrence CTA
 constexpr int NSL = D / NV;
 
 // ---- record of one (chunk, head) ---------------------------------------------------------
-// Shared-memory operand images (rows of 128 B, 128-byte swizzle) and value-channel slices:
-constexpr uint32_t kRecP0 = 0;          // P  K-major rows r (64), channels 0..63 / 64..127 (2 x 8 KB)
-constexpr uint32_t kRecM0 = 16384;      // M  K-major rows i (128), channels 0..63 / 64..127 (2 x 16 KB)
-constexpr uint32_t kRecB = 49152;       // B  [slice][i 128][64] bf16, rows swizzled (2 x 16 KB)
-constexpr uint32_t kRecR = 81920;       // R  [slice][r 64][64]  bf16, rows swizzled (2 x 8 KB)
-constexpr uint32_t kRecGamma = 98304;   // gamma fp32 [128]
-constexpr uint32_t kRecBytes = 98816;
+// Shared-memory operand images (rows of 128 B, 128-byte swizzle), each 1024-byte aligned:
+constexpr uint32_t kRecP0 = 0;          // P     K-major rows r (64), key channels 0..63 / 64..127 (2 x 8 KB)
+constexpr uint32_t kRecM0 = 16384;      // M     K-major rows i (128), key channels 0..63 / 64..127 (2 x 16 KB)
+constexpr uint32_t kRecKR = 49152;      // K_res rows t (64), key channels i 0..63 / 64..127 (2 x 8 KB);
+                                        //       the MN-major A operand K_res^T
+constexpr uint32_t kRecU = 65536;       // U     rows t (64), value channels 0..63 / 64..127 (2 x 8 KB);
+                                        //       an MN-major B operand per value slice
+constexpr uint32_t kRecAQ = 81920;      // Aqk   K-major rows r (64), tokens s (8 KB)
+constexpr uint32_t kRecGamma = 90112;   // gamma fp32 [128]
+constexpr uint32_t kRecBytes = 90624;
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -420,6 +424,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     fence_proxy_async_smem();
     __syncthreads();
     KDA_TRACE_POINT(ptr_, 8192 + 3);
+    // K_res and Aqk are final: their images go to the record as they are (thread 0 waits for
+    // these copies to have read K_res before the K_res space is reused for staging)
+    if (tid == 0) {
+        bulk_s2g(rec + kRecKR, sb + S::KI0, 8192);
+        bulk_s2g(rec + kRecKR + 8192, sb + S::KI1, 8192);
+        bulk_s2g(rec + kRecAQ, sb + S::AQK, 8192);
+    }
 
     // ---- (3) UT transform INV = (I + L)^{-1}, in place over L ----
     // Every entry above the diagonal of the buffer is 0 (L is strictly lower triangular and
@@ -531,57 +542,50 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     KDA_TRACE_POINT(ptr_, 8192 + 5);
 
-    // ---- (5) [-M | B] = K_res^T [W | U] -> TMEM [0, 256) ----
+    // ---- (5) -M = K_res^T W -> TMEM [0, 128) ----
     if (tid == 0) {
         tc_fence_after();
-        constexpr uint32_t id = idesc_bf16(128, 256, true, true);
+        // U is final: its image (two value slices) goes to the record as it is
+        bulk_s2g(rec + kRecU, sb + S::V0, 8192);
+        bulk_s2g(rec + kRecU + 8192, sb + S::V1, 8192);
+        constexpr uint32_t id = idesc_bf16(128, 128, true, true);
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
             umma_bf16(tmem, smem_desc(sb + S::KI0 + ks * 2048, S::BLK, 1024, kSwizzle128),
                       smem_desc(sb + S::KD0 + ks * 2048, S::BLK, 1024, kSwizzle128), id, ks > 0);
         umma_commit(bar);
+        bulk_wait_read<2>();   // the K_res / Aqk copies have read their sources
     }
     ok = mbar_wait(bar, phase);
     phase ^= 1;
     tc_fence_after();
     if (!prep_sync_ok(ok, tid)) goto done;
     {
-        // Drain: each warp turns its 32 TMEM lanes x 128 columns into two 4 KB pieces of the
-        // record (32 complete swizzled rows each) staged in a private, now unused 4 KB slot,
-        // and copies each piece out with one bulk copy.
-        //   column half 0 -> M = -K_res^T W rows i, K block 0 / 1
-        //   column half 1 -> B = K_res^T U rows i, value slice 0 / 1
+        // Drain: warp (wq, wh) turns its 32 TMEM lanes x 64 columns (K block wh of M, rows
+        // i = 32 wq ..) into a 4 KB piece of the record (32 complete swizzled rows) staged in a
+        // private, now unused 4 KB slot, and copies it out with one bulk copy.
         uint8_t* slot = sm + stage_slot(warp);
+        float d[64];
+        tmem_ld32(tl + 64 * wh, *reinterpret_cast<float(*)[32]>(&d[0]));
+        tmem_ld32(tl + 64 * wh + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
+        tmem_wait_ld();
 #pragma unroll
-        for (int pc = 0; pc < 2; ++pc) {
-            const uint32_t col0 = 128 * wh + 64 * pc;
-            float d[64];
-            tmem_ld32(tl + col0, *reinterpret_cast<float(*)[32]>(&d[0]));
-            tmem_ld32(tl + col0 + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
-            tmem_wait_ld();
-            if (wh == 0) {
+        for (int u = 0; u < 64; ++u) d[u] = -d[u];
 #pragma unroll
-                for (int u = 0; u < 64; ++u) d[u] = -d[u];
-            }
-            if (pc == 1 && lane == 0) bulk_wait_read<0>();
-            __syncwarp();
-#pragma unroll
-            for (int cb = 0; cb < 8; ++cb)
-                *reinterpret_cast<uint4*>(slot + sw128_off(lane, cb)) = pack_bf16x8(&d[8 * cb]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0)
-                bulk_s2g(rec + (wh == 0 ? kRecM0 : kRecB) + pc * 16384 + wq * 4096, smem_u32(slot), 4096);
-        }
+        for (int cb = 0; cb < 8; ++cb)
+            *reinterpret_cast<uint4*>(slot + sw128_off(lane, cb)) = pack_bf16x8(&d[8 * cb]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) bulk_s2g(rec + kRecM0 + wh * 16384 + wq * 4096, smem_u32(slot), 4096);
     }
     tc_fence_before();
     __syncthreads();
     KDA_TRACE_POINT(ptr_, 8192 + 6);
 
-    // ---- (6) [Aqk W | Aqk U] -> TMEM [0, 256) (lanes 0-63); P = Q_dec - Aqk W, R = Aqk U ----
+    // ---- (6) Aqk W -> TMEM [0, 128) (lanes 0-63); P = Q_dec - Aqk W ----
     if (tid == 0) {
         tc_fence_after();
-        constexpr uint32_t id = idesc_bf16(128, 256, false, true);
+        constexpr uint32_t id = idesc_bf16(128, 128, false, true);
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
             umma_bf16(tmem, smem_desc(sb + S::AQK + ks * 32, 16, 1024, kSwizzle128),
@@ -593,36 +597,28 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tc_fence_after();
     if (!prep_sync_ok(ok, tid)) goto done;
     if (wq < 2) {
-        //   column half 0 -> P = Q_dec - Aqk W rows r, K block 0 / 1
-        //   column half 1 -> R = Aqk U rows r, value slice 0 / 1
+        // rows r = 32 wq .., K block wh of P
         const int r = 32 * wq + lane;
         uint8_t* slot = sm + stage_slot(warp);
+        float d[64];
+        tmem_ld32(tl + 64 * wh, *reinterpret_cast<float(*)[32]>(&d[0]));
+        tmem_ld32(tl + 64 * wh + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
+        tmem_wait_ld();
 #pragma unroll
-        for (int pc = 0; pc < 2; ++pc) {
-            const uint32_t col0 = 128 * wh + 64 * pc;
-            float d[64];
-            tmem_ld32(tl + col0, *reinterpret_cast<float(*)[32]>(&d[0]));
-            tmem_ld32(tl + col0 + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
-            tmem_wait_ld();
-            if (wh == 0) {
+        for (int cb = 0; cb < 8; ++cb) {
+            float qv[8];
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + wh * S::BLK + sw128_off(r, cb)), qv);
 #pragma unroll
-                for (int cb = 0; cb < 8; ++cb) {
-                    float qv[8];
-                    unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + pc * S::BLK + sw128_off(r, cb)), qv);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) d[8 * cb + u] = qv[u] - d[8 * cb + u];
-                }
-            }
-            if (lane == 0) bulk_wait_read<0>();
-            __syncwarp();
-#pragma unroll
-            for (int cb = 0; cb < 8; ++cb)
-                *reinterpret_cast<uint4*>(slot + sw128_off(lane, cb)) = pack_bf16x8(&d[8 * cb]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0)
-                bulk_s2g(rec + (wh == 0 ? kRecP0 : kRecR) + pc * 8192 + wq * 4096, smem_u32(slot), 4096);
+            for (int u = 0; u < 8; ++u) d[8 * cb + u] = qv[u] - d[8 * cb + u];
         }
+        if (lane == 0) bulk_wait_read<0>();   // this warp's M piece has left the slot
+        __syncwarp();
+#pragma unroll
+        for (int cb = 0; cb < 8; ++cb)
+            *reinterpret_cast<uint4*>(slot + sw128_off(lane, cb)) = pack_bf16x8(&d[8 * cb]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) bulk_s2g(rec + kRecP0 + wh * 8192 + wq * 4096, smem_u32(slot), 4096);
     }
 done:
     if (lane == 0) bulk_wait_all();   // no copy may still read shared memory at exit
@@ -636,39 +632,35 @@ done:
 }
 
 // ------------------------------------------------------------------ chunk recurrence + outputs
-// One CTA per (sequence, head, 64 value channels).  Per chunk, the issuer launches two
-// tensor-core products reading the same bf16 image of S_in:
-//   D_S = M S_in   (128 x 64, K = 128)  -> S_out = gamma S_in + D_S + B  (the serial chain)
-//   D_O = P S_in   ( 64 x 64, K = 128)  -> O = D_O + R                   (beside the chain)
+// One CTA per (sequence, head, 64 value channels).  Per chunk, two tensor-core products read
+// the same bf16 image of S_in and this slice of U:
+//   D_S = [M | K_res^T] [S_in ; U]   (128 x 64, K = 128 + 64)  -> S_out = gamma S_in + D_S
+//   D_O = [P | Aqk]     [S_in ; U]   ( 64 x 64, K = 128 + 64)  -> O = D_O
+// so the state warps only scale, add and convert; the chain is D_S -> state update -> the
+// next S_in image -> the next D_S.
 // warps 0-7: state (warp w: rows 32 (w % 4) .. +31 = its TMEM lanes, columns 32 (w / 4) .. +31
 // of the slice), then this chunk's output rows 16 (w % 4) .. +15 (the M = 64 accumulator
-// puts row r in lane 32 (r / 16) + r % 16); warp 8: loader of M, B, gamma (3 stages);
-// warp 9: issuer of D_S; warp 10: loader of P, R (2 stages); warp 11: issuer of D_O.  The
-// two issuers are separate threads so that a late P never holds back the chain's product.
-constexpr int kRecThreads = 384;
+// puts row r in lane 32 (r / 16) + r % 16); warp 8: loader (2 stages of P, M, K_res, the U
+// slice and Aqk); warp 9: issuer of D_S; warp 10: issuer of D_O.  The two issuers are
+// separate threads, so that the output product never holds back the chain's.
+constexpr int kRecThreads = 352;
 constexpr int kRecComputeWarps = 8;
-constexpr int kLoaderWarp = 8, kIssuerWarp = 9, kLoaderOWarp = 10, kIssuerOWarp = 11;
-constexpr int kStagesA = 3, kStagesB = 2;
-constexpr uint32_t kStM = 0;          // M, both K blocks (32 KB)
-constexpr uint32_t kStB = 32768;      // B slice [128][64] bf16 (rows swizzled)
-constexpr uint32_t kStageA = 49152;
-constexpr uint32_t kStP = 0;          // P, both K blocks (16 KB)
-constexpr uint32_t kStR = 16384;      // R slice [64][64] bf16 (rows swizzled)
-constexpr uint32_t kStageB = 24576;
+constexpr int kLoaderWarp = 8, kIssuerWarp = 9, kIssuerOWarp = 10;
+constexpr int kStages = 2, kPrefetchAhead = 4;
+// stage: the record's first 64 KB (P, M, K_res) as they are, then the U slice and Aqk
+constexpr uint32_t kStP = 0, kStM = 16384, kStKR = 49152, kStU = 65536, kStAQ = 73728;
+constexpr uint32_t kStageBytes = 81920;
 struct RecSmem {
-    static constexpr uint32_t RB = kStagesA * kStageA;       // ring of P / R stages
-    static constexpr uint32_t SB = RB + kStagesB * kStageB;  // S (bf16) B images, 2 x 16 KB
-    static constexpr uint32_t GAM = SB + 2 * 16384;          // gamma [stage][128] fp32
-    // fullA[3] emptyA[3] fullB[2] emptyB[2] mma_s mma_o[2] ofree[2] sbr[2]
-    static constexpr uint32_t BAR = GAM + kStagesA * 512;
-    static constexpr uint32_t TMEM = BAR + 17 * 8;
+    static constexpr uint32_t SB = kStages * kStageBytes;   // S (bf16) B images, 2 x 16 KB
+    static constexpr uint32_t OST = SB + 2 * 16384;          // output staging [64][128 B]
+    // full[2] empty[2] mma_s mma_o[2] ofree[2] sbr[2]
+    static constexpr uint32_t BAR = OST + 8192;
+    static constexpr uint32_t TMEM = BAR + 11 * 8;
     static constexpr uint32_t FLAG = TMEM + 4;
     static constexpr uint32_t BYTES = FLAG + 4 + 1024;
 };
 static_assert(RecSmem::BYTES <= 232448, "recurrence shared memory exceeds 227 KB");
 constexpr uint32_t kRecTmemCols = 256;  // D_S [0, 64), D_O buffers [64, 128), [128, 192)
-constexpr uint32_t kTxA = 32768 + 16384 + 512;
-constexpr uint32_t kTxB = 16384 + 8192;
 
 __global__ void __launch_bounds__(kRecThreads, 1)
 rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __restrict__ tab,
@@ -680,29 +672,26 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
     const int n = blockIdx.x / (NSL * H);
     const int c_begin = off[n], nchunks = off[n + 1] - c_begin;
     (void)num_seqs;
+    auto record = [&](int kk) { return records + ((size_t)(c_begin + kk) * H + h) * kRecBytes; };
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     const uint32_t sb = smem_u32(sm);
     // Each barrier's waiters can never fall two phases behind: its next phase needs an
     // arrival that every waiter of the current phase precedes.
-    const uint32_t fullA = sb + S::BAR, emptyA = fullA + 24, fullB = fullA + 48, emptyB = fullA + 64;
-    const uint32_t mma_s = fullA + 80, mma_o = fullA + 88, ofree = fullA + 104, sbr0 = fullA + 120;
+    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 16, mma_s = full0 + 32, mma_o = full0 + 40;
+    const uint32_t ofree = full0 + 56, sbr0 = full0 + 72;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + S::FLAG);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (warp == 0) tmem_alloc(sb + S::TMEM, kRecTmemCols);
     if (tid == 0) {
-        for (int st = 0; st < kStagesA; ++st) {
-            mbar_init(fullA + 8 * st, 1);
-            mbar_init(emptyA + 8 * st, kRecComputeWarps);
-        }
-        for (int st = 0; st < kStagesB; ++st) {
-            mbar_init(fullB + 8 * st, 1);
-            mbar_init(emptyB + 8 * st, kRecComputeWarps);
-            mbar_init(mma_o + 8 * st, 1);
-            mbar_init(ofree + 8 * st, kRecComputeWarps);
-            mbar_init(sbr0 + 8 * st, kRecComputeWarps);
+        for (int b2 = 0; b2 < 2; ++b2) {
+            mbar_init(full0 + 8 * b2, 1);
+            mbar_init(empty0 + 8 * b2, 2);    // tcgen05.commit of both products that read it
+            mbar_init(mma_o + 8 * b2, 1);
+            mbar_init(ofree + 8 * b2, kRecComputeWarps);
+            mbar_init(sbr0 + 8 * b2, kRecComputeWarps);
         }
         mbar_init(mma_s, 1);
         fence_mbar_init();
@@ -713,111 +702,98 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
     tc_fence_after();
     const uint32_t tS = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
 
-    if (warp == kLoaderWarp || warp == kLoaderOWarp) {
-        // ---------------- loaders: ring A (M, B slice, gamma), ring B (P, R slice) ----------
+    if (warp == kLoaderWarp) {
+        // ---------------- loader ------------------------------------------------------------
         if (lane == 0) {
-            const bool ring_a = warp == kLoaderWarp;
-            const int nst = ring_a ? kStagesA : kStagesB;
-            const uint32_t full = ring_a ? fullA : fullB, empty = ring_a ? emptyA : emptyB;
+            // everything this CTA reads of a record goes to L2 kPrefetchAhead chunks early
+            auto prefetch = [&](int kk) {
+                const uint8_t* rec = record(kk);
+                bulk_prefetch_l2(rec, 65536);
+                bulk_prefetch_l2(rec + kRecU + sl * 8192, 8192);
+                bulk_prefetch_l2(rec + kRecAQ, 8192 + 512);
+            };
+            for (int kk = 0; kk < nchunks && kk < kPrefetchAhead; ++kk) prefetch(kk);
             int issued = 0;
             for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
-                const int st = kk % nst, use = kk / nst;
-                KDA_TRACE_POINT(ring_a && blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 0);
-                if (use > 0 && !mbar_wait(empty + 8 * st, (use - 1) & 1)) {
+                const int st = kk % kStages, use = kk / kStages;
+                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 0);
+                if (use > 0 && !mbar_wait(empty0 + 8 * st, (use - 1) & 1)) {
                     kda_set_status(KDA_ERR_TIMEOUT);
                     *abort_flag = 1;
                     break;
                 }
-                const uint8_t* rec = records + ((size_t)(c_begin + kk) * H + h) * kRecBytes;
-                const uint32_t fb = full + 8 * st;
-                if (ring_a) {
-                    const uint32_t dst = sb + st * kStageA;
-                    mbar_arrive_expect_tx(fb, kTxA);
-                    bulk_g2s(dst + kStM, rec + kRecM0, 32768, fb);
-                    bulk_g2s(dst + kStB, rec + kRecB + sl * 16384, 16384, fb);
-                    bulk_g2s(sb + S::GAM + st * 512, rec + kRecGamma, 512, fb);
-                    // everything this CTA will read of the record kStagesA chunks ahead goes to
-                    // L2 now, so that those copies are served from L2
-                    if (kk + kStagesA < nchunks) {
-                        const uint8_t* ahead = rec + (size_t)kStagesA * H * kRecBytes;
-                        bulk_prefetch_l2(ahead + kRecP0, 16384 + 32768);
-                        bulk_prefetch_l2(ahead + kRecB + sl * 16384, 16384);
-                        bulk_prefetch_l2(ahead + kRecR + sl * 8192, 8192);
-                        bulk_prefetch_l2(ahead + kRecGamma, 512);
-                    }
-                } else {
-                    const uint32_t dst = sb + S::RB + st * kStageB;
-                    mbar_arrive_expect_tx(fb, kTxB);
-                    bulk_g2s(dst + kStP, rec + kRecP0, 16384, fb);
-                    bulk_g2s(dst + kStR, rec + kRecR + sl * 8192, 8192, fb);
-                }
-                KDA_TRACE_POINT(ring_a && blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 1);
+                const uint8_t* rec = record(kk);
+                const uint32_t dst = sb + st * kStageBytes, fb = full0 + 8 * st;
+                mbar_arrive_expect_tx(fb, kStageBytes);
+#pragma unroll
+                for (int part = 0; part < 4; ++part)   // P, M, K_res: the record's first 64 KB
+                    bulk_g2s(dst + part * 16384, rec + part * 16384, 16384, fb);
+                bulk_g2s(dst + kStU, rec + kRecU + sl * 8192, 8192, fb);
+                bulk_g2s(dst + kStAQ, rec + kRecAQ, 8192, fb);
+                if (kk + kPrefetchAhead < nchunks) prefetch(kk + kPrefetchAhead);
+                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 1);
                 ++issued;
             }
             // never leave with copies in flight: wait (bounded) for the last stages filled
-            for (int kk = max(0, issued - nst); kk < issued; ++kk)
-                mbar_wait(full + 8 * (kk % nst), (kk / nst) & 1);
+            for (int kk = max(0, issued - kStages); kk < issued; ++kk)
+                mbar_wait(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
         }
-    } else if (warp == kIssuerWarp) {
-        // ---------------- issuer of D_S = M S_in, once the stage and S_in are ready --------
-        if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16(128, NV, false, true);
-            for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
-                const int st = kk % kStagesA;
-                const uint32_t sbuf = sb + S::SB + (kk & 1) * 16384;
-                if (!mbar_wait(fullA + 8 * st, (kk / kStagesA) & 1) ||
-                    !mbar_wait(sbr0 + 8 * (kk & 1), (kk >> 1) & 1)) {
-                    kda_set_status(KDA_ERR_TIMEOUT);
-                    *abort_flag = 1;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t stage = sb + st * kStageA;
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t ko = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    umma_bf16(tS, smem_desc(stage + kStM + ko, 16, 1024, kSwizzle128),
-                              smem_desc(sbuf + ks * 2048, 16, 1024, kSwizzle128), idS, ks > 0);
-                }
-                umma_commit(mma_s);
-                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 2);
-            }
-        }
-    } else if (warp == kIssuerOWarp) {
-        // ---------------- issuer of D_O = P S_in into output buffer kk % 2, once P and S_in
-        // are in and the output rows of chunk kk - 2 have left that buffer.  S_in's image
-        // stays put until this product is done: the state warps overwrite it only after
+    } else if (warp == kIssuerWarp || warp == kIssuerOWarp) {
+        // ---------------- issuers: D_S (warp 9) and D_O into buffer kk % 2 (warp 10) -------
+        // D_O(kk) also waits until the output rows of chunk kk - 2 have left its buffer.  The
+        // image of S_in stays put until D_O is done: the state warps overwrite it only after
         // they have drained D_O.
         if (lane == 0) {
+            const bool is_s = warp == kIssuerWarp;
+            constexpr uint32_t idS = idesc_bf16(128, NV, false, true);
+            constexpr uint32_t idSx = idesc_bf16(128, NV, true, true);    // A = K_res^T (MN-major)
             constexpr uint32_t idO = idesc_bf16(64, NV, false, true);
             for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
-                const int so = kk & 1;
+                const int st = kk % kStages, so = kk & 1;
                 const uint32_t sbuf = sb + S::SB + (kk & 1) * 16384;
-                if (!mbar_wait(fullB + 8 * so, (kk >> 1) & 1) ||
+                if (!mbar_wait(full0 + 8 * st, (kk / kStages) & 1) ||
                     !mbar_wait(sbr0 + 8 * (kk & 1), (kk >> 1) & 1) ||
-                    (kk >= 2 && !mbar_wait(ofree + 8 * so, ((kk - 2) >> 1) & 1))) {
+                    (!is_s && kk >= 2 && !mbar_wait(ofree + 8 * so, ((kk - 2) >> 1) & 1))) {
                     kda_set_status(KDA_ERR_TIMEOUT);
                     *abort_flag = 1;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t pst = sb + S::RB + so * kStageB;
+                const uint32_t stage = sb + st * kStageBytes;
+                if (is_s) {
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t ko = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    umma_bf16(tS + 64 + 64 * so, smem_desc(pst + kStP + ko, 16, 1024, kSwizzle128),
-                              smem_desc(sbuf + ks * 2048, 16, 1024, kSwizzle128), idO, ks > 0);
+                    for (int ks = 0; ks < D / 16; ++ks)
+                        umma_bf16(tS, smem_desc(stage + kStM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128),
+                                  smem_desc(sbuf + ks * 2048, 16, 1024, kSwizzle128), idS, ks > 0);
+#pragma unroll
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        umma_bf16(tS, smem_desc(stage + kStKR + ks * 2048, 8192, 1024, kSwizzle128),
+                                  smem_desc(stage + kStU + ks * 2048, 16, 1024, kSwizzle128), idSx, 1);
+                    umma_commit(mma_s);
+                    KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 2);
+                } else {
+                    const uint32_t tO = tS + 64 + 64 * so;
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks)
+                        umma_bf16(tO, smem_desc(stage + kStP + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128),
+                                  smem_desc(sbuf + ks * 2048, 16, 1024, kSwizzle128), idO, ks > 0);
+#pragma unroll
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        umma_bf16(tO, smem_desc(stage + kStAQ + ks * 32, 16, 1024, kSwizzle128),
+                                  smem_desc(stage + kStU + ks * 2048, 16, 1024, kSwizzle128), idO, 1);
+                    umma_commit(mma_o + 8 * so);
+                    KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 3);
                 }
-                umma_commit(mma_o + 8 * so);
-                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 3);
+                umma_commit(empty0 + 8 * st);
             }
         }
-    } else {
+    } else if (warp < kRecComputeWarps) {
         // ---------------- state: row i, columns 32 cw .. 32 cw + 31 of the slice -----------
         constexpr int NC = NV / 2;   // columns per thread
         const int q4 = warp & 3, i = 32 * q4 + lane, cw = warp >> 2;
         const uint32_t taw = (uint32_t)(32 * q4) << 16;
         const size_t sbase = (((size_t)n * H + h) * D + i) * D + (size_t)sl * NV + NC * cw;
+        const int r_out = 16 * q4 + lane;   // output row of this lane (lanes 0-15)
         float Sr[NC];
         if (initial_state) {
 #pragma unroll
@@ -835,32 +811,27 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
             for (int cb = 0; cb < NC / 8; ++cb)
                 *reinterpret_cast<uint4*>(sm + buf + sw128_off(i, 4 * cw + cb)) = pack_bf16x8(&Sr[8 * cb]);
         };
-        if (nchunks > 0) put_state(S::SB);
+        // gamma of row i and the (first token, rows) of a chunk, loaded one chunk ahead
+        float gam = 0.f;
+        int2 ce = make_int2(0, 0);
+        if (nchunks > 0) {
+            gam = __ldg(reinterpret_cast<const float*>(record(0) + kRecGamma) + i);
+            ce = tab[c_begin];
+            put_state(S::SB);
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(sbr0);
 
         bool ok = true;
-        const int r_out = 16 * q4 + lane;   // output row of this lane (lanes 0-15)
         for (int kk = 0; kk < nchunks; ++kk) {
-            const int st = kk % kStagesA, so = kk & 1;
+            const int so = kk & 1;
+            const bool more = kk + 1 < nchunks;
             const bool tr = blockIdx.x == 0 && tid == 0 && kk < 256;
             (void)tr;
-            const int2 ce = tab[c_begin + kk];   // (first token, rows) of this chunk
             KDA_TRACE_POINT(tr, kk * 8 + 0);
-            ok = __all_sync(0xffffffffu, mbar_wait(fullA + 8 * st, (kk / kStagesA) & 1));
-            if (!ok || *abort_flag) { ok = false; break; }
-            KDA_TRACE_POINT(tr, kk * 8 + 1);
-            // this chunk's gamma and B row, before the serial product lands
-            const float gam = reinterpret_cast<const float*>(sm + S::GAM + st * 512)[i];
-            const uint8_t* stage_p = sm + st * kStageA;
-            uint4 bq[NC / 8];
-#pragma unroll
-            for (int cb = 0; cb < NC / 8; ++cb)
-                bq[cb] = *reinterpret_cast<const uint4*>(stage_p + kStB + sw128_off(i, 4 * cw + cb));
-            KDA_TRACE_POINT(tr, kk * 8 + 2);
             ok = __all_sync(0xffffffffu, mbar_wait(mma_s, kk & 1));
-            if (!ok) break;
+            if (!ok || *abort_flag) { ok = false; break; }
             KDA_TRACE_POINT(tr, kk * 8 + 3);
             tc_fence_after();
             {
@@ -868,30 +839,24 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
                 tmem_ld32(tS + taw + NC * cw, dsv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int cb = 0; cb < NC / 8; ++cb) {
-                    float bv[8];
-                    unpack_bf16x8(bq[cb], bv);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int j = 8 * cb + u;
-                        Sr[j] = fmaf(gam, Sr[j], dsv[j] + bv[u]);
-                    }
-                }
+                for (int j = 0; j < NC; ++j) Sr[j] = fmaf(gam, Sr[j], dsv[j]);
             }
             KDA_TRACE_POINT(tr, kk * 8 + 4);
-            if (kk + 1 < nchunks) put_state(S::SB + ((kk + 1) & 1) * 16384);
+            // the image of S_{kk+1} replaces that of S_{kk-1}, whose products (D_S(kk-1), and
+            // D_O(kk-1), drained below in the previous pass) are complete
+            if (more) put_state(S::SB + ((kk + 1) & 1) * 16384);
             tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(sbr0 + 8 * ((kk + 1) & 1));
-                mbar_arrive(emptyA + 8 * st);
+            if (lane == 0) mbar_arrive(sbr0 + 8 * ((kk + 1) & 1));
+            const int t0 = ce.x, nrow = ce.y;
+            if (more) {
+                gam = __ldg(reinterpret_cast<const float*>(record(kk + 1) + kRecGamma) + i);
+                ce = tab[c_begin + kk + 1];
             }
             KDA_TRACE_POINT(tr, kk * 8 + 5);
-            // output rows 16 q4 .. 16 q4 + 15, columns 32 cw .. +31 of the slice: O = D_O + R
-            // (the R slice is read after this warp has itself seen the stage's copies land)
-            ok = __all_sync(0xffffffffu, mbar_wait(fullB + 8 * so, (kk >> 1) & 1) &&
-                                             mbar_wait(mma_o + 8 * so, (kk >> 1) & 1));
+            // output rows 16 q4 .. 16 q4 + 15, columns 32 cw .. +31 of the slice
+            ok = __all_sync(0xffffffffu, mbar_wait(mma_o + 8 * so, (kk >> 1) & 1));
             if (!ok) break;
             KDA_TRACE_POINT(tr, kk * 8 + 7);
             tc_fence_after();
@@ -901,34 +866,28 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(ofree + 8 * so);
-            // O = D_O + R in place of this warp's own R entries (rows 16 q4 .. +15, 16-byte
-            // chunks 4 cw .. 4 cw + 3 of the slice), then re-read so that four lanes store one
-            // row's 64 contiguous bytes: each store instruction covers 8 rows.
-            uint8_t* rs = sm + S::RB + so * kStageB + kStR;
+            // lane l (< 16) holds row 16 q4 + l: stage the bf16 rows, then re-read them so that
+            // four lanes store one row's 64 contiguous bytes (8 rows per store instruction)
+            uint8_t* os = sm + S::OST;
             if (lane < 16) {
 #pragma unroll
-                for (int qq = 0; qq < NC / 8; ++qq) {
-                    uint4* p = reinterpret_cast<uint4*>(rs + sw128_off(r_out, 4 * cw + qq));
-                    float rv[8];
-                    unpack_bf16x8(*p, rv);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) rv[u] += dov[8 * qq + u];
-                    *p = pack_bf16x8(rv);
-                }
+                for (int cb = 0; cb < NC / 8; ++cb)
+                    *reinterpret_cast<uint4*>(os + sw128_off(r_out, 4 * cw + cb)) = pack_bf16x8(&dov[8 * cb]);
             }
             __syncwarp();
+            uint4 ov[2];
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8)
+                ov[g8] = *reinterpret_cast<const uint4*>(
+                    os + sw128_off(16 * q4 + 8 * g8 + (lane >> 2), 4 * cw + (lane & 3)));
 #pragma unroll
             for (int g8 = 0; g8 < 2; ++g8) {
-                const int rr = 16 * q4 + 8 * g8 + (lane >> 2), cc = lane & 3;
-                if (rr < ce.y) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(rs + sw128_off(rr, 4 * cw + cc));
-                    *reinterpret_cast<uint4*>(out + ((size_t)(ce.x + rr) * H + h) * D + sl * NV + NC * cw +
-                                              8 * cc) = v;
-                }
+                const int rr = 16 * q4 + 8 * g8 + (lane >> 2);
+                if (rr < nrow)
+                    *reinterpret_cast<uint4*>(out + ((size_t)(t0 + rr) * H + h) * D + sl * NV + NC * cw +
+                                              8 * (lane & 3)) = ov[g8];
             }
-            fence_proxy_async_smem();   // the slot is next written by a bulk copy
-            __syncwarp();
-            if (lane == 0) mbar_arrive(emptyB + 8 * so);
+            __syncwarp();   // the staging rows are rewritten by the next chunk
             KDA_TRACE_POINT(tr, kk * 8 + 6);
         }
         if (!ok) {

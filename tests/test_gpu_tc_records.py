@@ -1,7 +1,8 @@
 """White-box check of the tensor-core preparation kernel: decode the per-(chunk, head)
-workspace record (shared-memory operand images with a 128-byte swizzle, and value-channel
-slices) and compare every chunk tensor with the fp64 chunked form of the oracle:
-M = -K_res^T W, B = K_res^T U, P = Q_dec - Aqk W, R = Aqk U, gamma."""
+workspace record (shared-memory operand images with a 128-byte swizzle) and compare every
+chunk tensor with the fp64 chunked form of the oracle: P = Q_dec - Aqk W, M = -K_res^T W,
+K_res, U, Aqk, gamma.  The recurrence adds K_res^T U and Aqk U to its products, so the
+derived B = K_res^T U and R = Aqk U are checked too."""
 import numpy as np
 import pytest
 import torch
@@ -12,7 +13,7 @@ from tests.gpu_helpers import to_device
 
 pytestmark = pytest.mark.gpu
 
-REC_BYTES = 98816
+REC_BYTES = 90624
 
 
 def _bf16(u8: np.ndarray) -> np.ndarray:
@@ -50,23 +51,23 @@ def test_prep_record_matches_chunked_oracle(nrow):
                               inp["beta"][:, 0].double().numpy())
     n = nrow
     M_ref = -T["K_res"].T @ T["W"]
-    B_ref = T["K_res"].T @ T["U"]
     P_ref = T["Q_dec"] - T["Aqk"] @ T["W"]
-    R_ref = T["Aqk"] @ T["U"]
     P = np.concatenate([_sw128(rec[kb * 8192:(kb + 1) * 8192], 64) for kb in range(2)], axis=1)
     M = np.concatenate([_sw128(rec[16384 + kb * 16384:16384 + (kb + 1) * 16384], 128) for kb in range(2)], axis=1)
-    B = np.concatenate([_sw128(rec[49152 + s * 16384:49152 + (s + 1) * 16384], 128)
-                        for s in range(2)], axis=1)
-    R = np.concatenate([_sw128(rec[81920 + s * 8192:81920 + (s + 1) * 8192], 64)
-                        for s in range(2)], axis=1)
-    gam = rec[98304:98816].copy().view(np.float32).astype(np.float64)
+    K_res = np.concatenate([_sw128(rec[49152 + b * 8192:49152 + (b + 1) * 8192], 64) for b in range(2)], axis=1)
+    U = np.concatenate([_sw128(rec[65536 + s * 8192:65536 + (s + 1) * 8192], 64) for s in range(2)], axis=1)
+    Aqk = _sw128(rec[81920:90112], 64)
+    gam = rec[90112:90624].copy().view(np.float32).astype(np.float64)
 
     def rel(a, b):
         return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
 
-    errs = {"M": rel(M, M_ref), "B": rel(B, B_ref), "P": rel(P[:n], P_ref), "R": rel(R[:n], R_ref),
-            "gamma": rel(gam, T["gamma"])}
+    errs = {"M": rel(M, M_ref), "P": rel(P[:n], P_ref), "K_res": rel(K_res[:n], T["K_res"]),
+            "U": rel(U[:n], T["U"]), "Aqk": rel(Aqk[:n, :n], T["Aqk"]),
+            "B": rel(K_res[:n].T @ U[:n], T["K_res"].T @ T["U"]),
+            "R": rel(Aqk[:n, :n] @ U[:n], T["Aqk"] @ T["U"]), "gamma": rel(gam, T["gamma"])}
     print(nrow, {k: "%.2e" % v for k, v in errs.items()})
     for k, e in errs.items():
         assert e < 2e-2, (k, e)
-    assert np.all(P[n:] == 0) and np.all(R[n:] == 0)
+    for x in (P[n:], K_res[n:], U[n:], Aqk[n:], Aqk[:, n:]):
+        assert np.all(x == 0)

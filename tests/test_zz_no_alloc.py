@@ -51,7 +51,7 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     args = lambda T, H, dt, dk: (P(4096), P(4096), P(4096), P(4096), P(4096), None, P(4096), 1,
                                  T, H, dk, dk, dt, P(4096), None, 64, None)
     need = lambda T, H: kda.kda_prefill_workspace_size(T, 1, H, 128, 128, 64, torch.bfloat16)
-    assert need(1343, 32) <= kda.NOALLOC_SCRATCH_BYTES < need(1344, 32)
-    assert lib.kda_prefill_noalloc(*args(1344, 32, kda.KDA_BF16, 128)) == kda.KDA_ERR_UNSUPPORTED
+    assert need(1471, 32) <= kda.NOALLOC_SCRATCH_BYTES < need(1472, 32)
+    assert lib.kda_prefill_noalloc(*args(1472, 32, kda.KDA_BF16, 128)) == kda.KDA_ERR_UNSUPPORTED
     assert lib.kda_prefill_noalloc(*args(1 << 20, 32, kda.KDA_BF16, 128)) == kda.KDA_ERR_UNSUPPORTED
     assert lib.kda_prefill_noalloc(*args(256, 2, kda.KDA_F32, 64)) == kda.KDA_ERR_UNSUPPORTED
