@@ -46,8 +46,6 @@ using namespace kda::sm100;
 
 constexpr int D = 128;   // d_k = d_v
 constexpr int C = 64;    // chunk
-constexpr int NV = 64;   // value channels per recurrence CTA
-constexpr int NSL = D / NV;
 
 // ---- record of one (chunk, head) ---------------------------------------------------------
 // Shared-memory operand images (rows of 128 B, 128-byte swizzle), each 1024-byte aligned:
@@ -55,8 +53,9 @@ constexpr uint32_t kRecP0 = 0;          // P     K-major rows r (64), key channe
 constexpr uint32_t kRecM0 = 16384;      // M     K-major rows i (128), key channels 0..63 / 64..127 (2 x 16 KB)
 constexpr uint32_t kRecKR = 49152;      // K_res rows t (64), key channels i 0..63 / 64..127 (2 x 8 KB);
                                         //       the MN-major A operand K_res^T
-constexpr uint32_t kRecU = 65536;       // U     rows t (64), value channels 0..63 / 64..127 (2 x 8 KB);
-                                        //       an MN-major B operand per value slice
+constexpr uint32_t kRecU = 65536;       // U     rows t (64), value channels 32 s .. 32 s + 31 for the 4
+                                        //       value slices s (4 x 4 KB, rows of 64 B, 64-byte
+                                        //       swizzle): an MN-major B operand per slice
 constexpr uint32_t kRecAQ = 81920;      // Aqk   K-major rows r (64), tokens s (8 KB)
 constexpr uint32_t kRecGamma = 90112;   // gamma fp32 [128]
 constexpr uint32_t kRecBytes = 90624;
@@ -522,7 +521,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     phase ^= 1;
     tc_fence_after();
     if (!prep_sync_ok(ok, tid)) goto done;
-    if (wq < 2) {  // rows r of W (column half 0) / U (column half 1) -> bf16 B image in place
+    if (wq < 2) {
+        // rows r of W (column half 0) -> bf16 B image in place of K_dec (two 64-column blocks,
+        // 128-byte swizzle); rows r of U (column half 1) -> four 32-column slices with a
+        // 64-byte swizzle, slices 0, 1 in place of V's first block and 2, 3 of its second
         const int r = 32 * wq + lane;
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
@@ -530,11 +532,18 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int col = 128 * wh + 32 * cb;
             tmem_ld32(tl + col, d);
             tmem_wait_ld();
-            const uint32_t blk = S::KD0 + (col >> 6) * S::BLK;
+            if (wh == 0) {
+                const uint32_t blk = S::KD0 + (col >> 6) * S::BLK;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq)
-                *reinterpret_cast<uint4*>(sm + blk + sw128_off(r, ((col & 63) >> 3) + qq)) =
-                    pack_bf16x8(&d[8 * qq]);
+                for (int qq = 0; qq < 4; ++qq)
+                    *reinterpret_cast<uint4*>(sm + blk + sw128_off(r, ((col & 63) >> 3) + qq)) =
+                        pack_bf16x8(&d[8 * qq]);
+            } else {
+                const uint32_t slice = (cb < 2 ? S::V0 : S::V1) + (cb & 1) * 4096;
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq)
+                    *reinterpret_cast<uint4*>(sm + slice + sw64_off(r, qq)) = pack_bf16x8(&d[8 * qq]);
+            }
         }
     }
     tc_fence_before();
@@ -545,7 +554,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // ---- (5) -M = K_res^T W -> TMEM [0, 128) ----
     if (tid == 0) {
         tc_fence_after();
-        // U is final: its image (two value slices) goes to the record as it is
+        // U is final: its image (four value slices) goes to the record as it is
         bulk_s2g(rec + kRecU, sb + S::V0, 8192);
         bulk_s2g(rec + kRecU + 8192, sb + S::V1, 8192);
         constexpr uint32_t id = idesc_bf16(128, 128, true, true);
@@ -632,13 +641,15 @@ done:
 }
 
 // ------------------------------------------------------------------ chunk recurrence + outputs
-// One CTA per (sequence, head, 64 value channels).  Per chunk, two tensor-core products read
-// the same bf16 image of S_in and this slice of U:
-//   D_S = [M | K_res^T] [S_in ; U]   (128 x 64, K = 128 + 64)  -> S_out = gamma S_in + D_S
-//   D_O = [P | Aqk]     [S_in ; U]   ( 64 x 64, K = 128 + 64)  -> O = D_O
+// One CTA per (sequence, head, NV value channels), NV = 32 or 64.  Per chunk, two tensor-core
+// products read the same bf16 image of S_in and this slice of U:
+//   D_S = [M | K_res^T] [S_in ; U]   (128 x NV, K = 128 + 64)  -> S_out = gamma S_in + D_S
+//   D_O = [P | Aqk]     [S_in ; U]   ( 64 x NV, K = 128 + 64)  -> O = D_O
 // so the state warps only scale, add and convert; the chain is D_S -> state update -> the
-// next S_in image -> the next D_S.
-// warps 0-7: state (warp w: rows 32 (w % 4) .. +31 = its TMEM lanes, columns 32 (w / 4) .. +31
+// next S_in image -> the next D_S.  Narrow slices shorten each chain step (half the columns
+// per thread, half the product) at the price of loading P, M, K_res and Aqk once per slice:
+// the launch takes NV = 32 while four CTAs per (sequence, head) still fit on the SMs at once.
+// warps 0-7: state (warp w: rows 32 (w % 4) .. +31 = its TMEM lanes, columns NV/2 (w / 4) ..
 // of the slice), then this chunk's output rows 16 (w % 4) .. +15 (the M = 64 accumulator
 // puts row r in lane 32 (r / 16) + r % 16); warp 8: loader (2 stages of P, M, K_res, the U
 // slice and Aqk); warp 9: issuer of D_S; warp 10: issuer of D_O.  The two issuers are
@@ -647,26 +658,44 @@ constexpr int kRecThreads = 352;
 constexpr int kRecComputeWarps = 8;
 constexpr int kLoaderWarp = 8, kIssuerWarp = 9, kIssuerOWarp = 10;
 constexpr int kStages = 2, kPrefetchAhead = 4;
-// stage: the record's first 64 KB (P, M, K_res) as they are, then the U slice and Aqk
-constexpr uint32_t kStP = 0, kStM = 16384, kStKR = 49152, kStU = 65536, kStAQ = 73728;
-constexpr uint32_t kStageBytes = 81920;
-struct RecSmem {
-    static constexpr uint32_t SB = kStages * kStageBytes;   // S (bf16) B images, 2 x 16 KB
-    static constexpr uint32_t OST = SB + 2 * 16384;          // output staging [64][128 B]
+constexpr uint32_t kUSlice = 4096;    // one 32-column U slice: 64 token rows of 64 B
+
+template <int NV_>
+struct RecCfg {
+    static constexpr int NV = NV_, NSL = D / NV, NC = NV / 2;   // NC: columns per thread
+    // stage: the record's first 64 KB (P, M, K_res) as they are, then the U slices and Aqk
+    static constexpr uint32_t kStP = 0, kStM = 16384, kStKR = 49152, kStU = 65536;
+    static constexpr uint32_t kUBytes = (NV / 32) * kUSlice;
+    static constexpr uint32_t kStAQ = kStU + kUBytes;
+    static constexpr uint32_t kStageBytes = kStAQ + 8192;
+    // S image (MN-major B operand): 128 key rows of 2 NV bytes, 128- or 64-byte swizzle
+    static constexpr uint32_t kSRow = 2 * NV, kSImg = 128 * kSRow, kSSbo = 8 * kSRow;
+    static constexpr uint32_t kSSwz = NV == 64 ? kSwizzle128 : kSwizzle64;
+    static constexpr uint32_t SB = kStages * kStageBytes;   // S images, 2 buffers
+    static constexpr uint32_t OST = SB + 2 * kSImg;          // output staging [64 rows][2 NV B]
     // full[2] empty[2] mma_s mma_o[2] ofree[2] sbr[2]
-    static constexpr uint32_t BAR = OST + 8192;
+    static constexpr uint32_t BAR = OST + 64 * kSRow;
     static constexpr uint32_t TMEM = BAR + 11 * 8;
     static constexpr uint32_t FLAG = TMEM + 4;
     static constexpr uint32_t BYTES = FLAG + 4 + 1024;
+    // D_S [0, NV), D_O buffers [NV, 2 NV), [2 NV, 3 NV)
+    static constexpr uint32_t kTmemCols = NV == 64 ? 256 : 128;
+    static_assert(kStAQ % 1024 == 0 && kStageBytes % 1024 == 0, "stage images must stay 1 KB aligned");
+    static_assert(BYTES <= 232448, "recurrence shared memory exceeds 227 KB");
+    // byte offset of 16-byte chunk `ch` of row `row` in an S image / the output staging
+    __device__ static __forceinline__ uint32_t s_off(uint32_t row, uint32_t ch) {
+        if constexpr (NV == 64) return sw128_off(row, ch);
+        else return sw64_off(row, ch);
+    }
 };
-static_assert(RecSmem::BYTES <= 232448, "recurrence shared memory exceeds 227 KB");
-constexpr uint32_t kRecTmemCols = 256;  // D_S [0, 64), D_O buffers [64, 128), [128, 192)
 
+template <int NV>
 __global__ void __launch_bounds__(kRecThreads, 1)
 rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __restrict__ tab,
            const uint8_t* __restrict__ records, const float* initial_state, float* final_state,
            __nv_bfloat16* __restrict__ out) {
-    using S = RecSmem;
+    using S = RecCfg<NV>;
+    constexpr int NSL = S::NSL;
     const int sl = blockIdx.x % NSL;
     const int h = (blockIdx.x / NSL) % H;
     const int n = blockIdx.x / (NSL * H);
@@ -684,7 +713,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + S::FLAG);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    if (warp == 0) tmem_alloc(sb + S::TMEM, kRecTmemCols);
+    if (warp == 0) tmem_alloc(sb + S::TMEM, S::kTmemCols);
     if (tid == 0) {
         for (int b2 = 0; b2 < 2; ++b2) {
             mbar_init(full0 + 8 * b2, 1);
@@ -709,7 +738,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
             auto prefetch = [&](int kk) {
                 const uint8_t* rec = record(kk);
                 bulk_prefetch_l2(rec, 65536);
-                bulk_prefetch_l2(rec + kRecU + sl * 8192, 8192);
+                bulk_prefetch_l2(rec + kRecU + sl * S::kUBytes, S::kUBytes);
                 bulk_prefetch_l2(rec + kRecAQ, 8192 + 512);
             };
             for (int kk = 0; kk < nchunks && kk < kPrefetchAhead; ++kk) prefetch(kk);
@@ -723,13 +752,13 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
                     break;
                 }
                 const uint8_t* rec = record(kk);
-                const uint32_t dst = sb + st * kStageBytes, fb = full0 + 8 * st;
-                mbar_arrive_expect_tx(fb, kStageBytes);
+                const uint32_t dst = sb + st * S::kStageBytes, fb = full0 + 8 * st;
+                mbar_arrive_expect_tx(fb, S::kStageBytes);
 #pragma unroll
                 for (int part = 0; part < 4; ++part)   // P, M, K_res: the record's first 64 KB
                     bulk_g2s(dst + part * 16384, rec + part * 16384, 16384, fb);
-                bulk_g2s(dst + kStU, rec + kRecU + sl * 8192, 8192, fb);
-                bulk_g2s(dst + kStAQ, rec + kRecAQ, 8192, fb);
+                bulk_g2s(dst + S::kStU, rec + kRecU + sl * S::kUBytes, S::kUBytes, fb);
+                bulk_g2s(dst + S::kStAQ, rec + kRecAQ, 8192, fb);
                 if (kk + kPrefetchAhead < nchunks) prefetch(kk + kPrefetchAhead);
                 KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 1);
                 ++issued;
@@ -750,7 +779,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
             constexpr uint32_t idO = idesc_bf16(64, NV, false, true);
             for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
                 const int st = kk % kStages, so = kk & 1;
-                const uint32_t sbuf = sb + S::SB + (kk & 1) * 16384;
+                const uint32_t sbuf = sb + S::SB + (kk & 1) * S::kSImg;
                 if (!mbar_wait(full0 + 8 * st, (kk / kStages) & 1) ||
                     !mbar_wait(sbr0 + 8 * (kk & 1), (kk >> 1) & 1) ||
                     (!is_s && kk >= 2 && !mbar_wait(ofree + 8 * so, ((kk - 2) >> 1) & 1))) {
@@ -759,28 +788,28 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
                     break;
                 }
                 tc_fence_after();
-                const uint32_t stage = sb + st * kStageBytes;
+                const uint32_t stage = sb + st * S::kStageBytes;
                 if (is_s) {
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks)
-                        umma_bf16(tS, smem_desc(stage + kStM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128),
-                                  smem_desc(sbuf + ks * 2048, 16, 1024, kSwizzle128), idS, ks > 0);
+                        umma_bf16(tS, smem_desc(stage + S::kStM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128),
+                                  smem_desc(sbuf + ks * 2 * S::kSSbo, 16, S::kSSbo, S::kSSwz), idS, ks > 0);
 #pragma unroll
                     for (int ks = 0; ks < C / 16; ++ks)
-                        umma_bf16(tS, smem_desc(stage + kStKR + ks * 2048, 8192, 1024, kSwizzle128),
-                                  smem_desc(stage + kStU + ks * 2048, 16, 1024, kSwizzle128), idSx, 1);
+                        umma_bf16(tS, smem_desc(stage + S::kStKR + ks * 2048, 8192, 1024, kSwizzle128),
+                                  smem_desc(stage + S::kStU + ks * 1024, kUSlice, 512, kSwizzle64), idSx, 1);
                     umma_commit(mma_s);
                     KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 2);
                 } else {
-                    const uint32_t tO = tS + 64 + 64 * so;
+                    const uint32_t tO = tS + NV + NV * so;
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks)
-                        umma_bf16(tO, smem_desc(stage + kStP + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128),
-                                  smem_desc(sbuf + ks * 2048, 16, 1024, kSwizzle128), idO, ks > 0);
+                        umma_bf16(tO, smem_desc(stage + S::kStP + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128),
+                                  smem_desc(sbuf + ks * 2 * S::kSSbo, 16, S::kSSbo, S::kSSwz), idO, ks > 0);
 #pragma unroll
                     for (int ks = 0; ks < C / 16; ++ks)
-                        umma_bf16(tO, smem_desc(stage + kStAQ + ks * 32, 16, 1024, kSwizzle128),
-                                  smem_desc(stage + kStU + ks * 2048, 16, 1024, kSwizzle128), idO, 1);
+                        umma_bf16(tO, smem_desc(stage + S::kStAQ + ks * 32, 16, 1024, kSwizzle128),
+                                  smem_desc(stage + S::kStU + ks * 1024, kUSlice, 512, kSwizzle64), idO, 1);
                     umma_commit(mma_o + 8 * so);
                     KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 3);
                 }
@@ -788,8 +817,8 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
             }
         }
     } else if (warp < kRecComputeWarps) {
-        // ---------------- state: row i, columns 32 cw .. 32 cw + 31 of the slice -----------
-        constexpr int NC = NV / 2;   // columns per thread
+        // ---------------- state: row i, columns NC cw .. NC cw + NC - 1 of the slice -------
+        constexpr int NC = S::NC;
         const int q4 = warp & 3, i = 32 * q4 + lane, cw = warp >> 2;
         const uint32_t taw = (uint32_t)(32 * q4) << 16;
         const size_t sbase = (((size_t)n * H + h) * D + i) * D + (size_t)sl * NV + NC * cw;
@@ -809,7 +838,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
         auto put_state = [&](uint32_t buf) {
 #pragma unroll
             for (int cb = 0; cb < NC / 8; ++cb)
-                *reinterpret_cast<uint4*>(sm + buf + sw128_off(i, 4 * cw + cb)) = pack_bf16x8(&Sr[8 * cb]);
+                *reinterpret_cast<uint4*>(sm + buf + S::s_off(i, (NC / 8) * cw + cb)) = pack_bf16x8(&Sr[8 * cb]);
         };
         // gamma of row i and the (first token, rows) of a chunk, loaded one chunk ahead
         float gam = 0.f;
@@ -836,7 +865,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
             tc_fence_after();
             {
                 float dsv[NC];
-                tmem_ld32(tS + taw + NC * cw, dsv);
+                tmem_ld_cols(tS + taw + NC * cw, dsv);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < NC; ++j) Sr[j] = fmaf(gam, Sr[j], dsv[j]);
@@ -844,7 +873,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
             KDA_TRACE_POINT(tr, kk * 8 + 4);
             // the image of S_{kk+1} replaces that of S_{kk-1}, whose products (D_S(kk-1), and
             // D_O(kk-1), drained below in the previous pass) are complete
-            if (more) put_state(S::SB + ((kk + 1) & 1) * 16384);
+            if (more) put_state(S::SB + ((kk + 1) & 1) * S::kSImg);
             tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
@@ -855,37 +884,40 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
                 ce = tab[c_begin + kk + 1];
             }
             KDA_TRACE_POINT(tr, kk * 8 + 5);
-            // output rows 16 q4 .. 16 q4 + 15, columns 32 cw .. +31 of the slice
+            // output rows 16 q4 .. 16 q4 + 15, columns NC cw .. of the slice
             ok = __all_sync(0xffffffffu, mbar_wait(mma_o + 8 * so, (kk >> 1) & 1));
             if (!ok) break;
             KDA_TRACE_POINT(tr, kk * 8 + 7);
             tc_fence_after();
             float dov[NC];
-            tmem_ld32(tS + taw + 64 + 64 * so + NC * cw, dov);
+            tmem_ld_cols(tS + taw + NV + NV * so + NC * cw, dov);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(ofree + 8 * so);
             // lane l (< 16) holds row 16 q4 + l: stage the bf16 rows, then re-read them so that
-            // four lanes store one row's 64 contiguous bytes (8 rows per store instruction)
+            // NC / 8 lanes store one row's 2 NC contiguous bytes
             uint8_t* os = sm + S::OST;
             if (lane < 16) {
 #pragma unroll
                 for (int cb = 0; cb < NC / 8; ++cb)
-                    *reinterpret_cast<uint4*>(os + sw128_off(r_out, 4 * cw + cb)) = pack_bf16x8(&dov[8 * cb]);
+                    *reinterpret_cast<uint4*>(os + S::s_off(r_out, (NC / 8) * cw + cb)) = pack_bf16x8(&dov[8 * cb]);
             }
             __syncwarp();
-            uint4 ov[2];
+            {
+                constexpr int LPR = NC / 8, RPI = 32 / LPR;   // lanes per row, rows per instruction
+                uint4 ov[16 / RPI];
 #pragma unroll
-            for (int g8 = 0; g8 < 2; ++g8)
-                ov[g8] = *reinterpret_cast<const uint4*>(
-                    os + sw128_off(16 * q4 + 8 * g8 + (lane >> 2), 4 * cw + (lane & 3)));
+                for (int g = 0; g < 16 / RPI; ++g)
+                    ov[g] = *reinterpret_cast<const uint4*>(
+                        os + S::s_off(16 * q4 + RPI * g + lane / LPR, LPR * cw + lane % LPR));
 #pragma unroll
-            for (int g8 = 0; g8 < 2; ++g8) {
-                const int rr = 16 * q4 + 8 * g8 + (lane >> 2);
-                if (rr < nrow)
-                    *reinterpret_cast<uint4*>(out + ((size_t)(t0 + rr) * H + h) * D + sl * NV + NC * cw +
-                                              8 * (lane & 3)) = ov[g8];
+                for (int g = 0; g < 16 / RPI; ++g) {
+                    const int rr = 16 * q4 + RPI * g + lane / LPR;
+                    if (rr < nrow)
+                        *reinterpret_cast<uint4*>(out + ((size_t)(t0 + rr) * H + h) * D + sl * NV + NC * cw +
+                                                  8 * (lane % LPR)) = ov[g];
+                }
             }
             __syncwarp();   // the staging rows are rewritten by the next chunk
             KDA_TRACE_POINT(tr, kk * 8 + 6);
@@ -904,7 +936,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tS, kRecTmemCols);
+        tmem_dealloc(tS, S::kTmemCols);
     }
 }
 
@@ -975,16 +1007,38 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
     return cudaGetLastError();
 }
 
-// Chunk-serial recurrence and the chunk outputs, over every (sequence, head, value slice).
+// SMs of the current device (cached per device; 0 when the query fails).
+inline int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cached[dev] == 0 &&
+        cudaDeviceGetAttribute(&cached[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cached[dev] = 0;
+    return cached[dev];
+}
+
+template <int NV>
+inline cudaError_t launch_scan_nv(const float* s0, float* sf, void* out, int num_seqs, const Workspace& w,
+                                  int H, cudaStream_t stream) {
+    using R = RecCfg<NV>;
+    cudaError_t e = cudaFuncSetAttribute(rec_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)R::BYTES);
+    if (e != cudaSuccess) return e;
+    rec_kernel<NV><<<(unsigned)num_seqs * H * R::NSL, kRecThreads, R::BYTES, stream>>>(
+        num_seqs, H, w.off, w.tab, w.records, s0, sf, static_cast<__nv_bfloat16*>(out));
+    return cudaGetLastError();
+}
+
+// Chunk-serial recurrence and the chunk outputs, over every (sequence, head, value slice):
+// 32-channel slices while 4 CTAs per (sequence, head) fit on the SMs at once, else 64.
 inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_seqs, int64_t total,
                                int H, void* workspace, cudaStream_t stream) {
     const Workspace w = split_workspace(workspace, total, num_seqs);
-    cudaError_t e = cudaFuncSetAttribute(rec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)RecSmem::BYTES);
-    if (e != cudaSuccess) return e;
-    rec_kernel<<<(unsigned)num_seqs * H * NSL, kRecThreads, RecSmem::BYTES, stream>>>(
-        num_seqs, H, w.off, w.tab, w.records, s0, sf, static_cast<__nv_bfloat16*>(out));
-    return cudaGetLastError();
+    const int sms = device_sm_count();
+    if ((int64_t)num_seqs * H * RecCfg<32>::NSL <= (int64_t)sms)
+        return launch_scan_nv<32>(s0, sf, out, num_seqs, w, H, stream);
+    return launch_scan_nv<64>(s0, sf, out, num_seqs, w, H, stream);
 }
 
 inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* g,

@@ -38,6 +38,15 @@ def test_bf16_ragged_varlen_small():
     check_prefill(inp, out, fin)
 
 
+def test_bf16_many_sequence_heads():
+    """More (sequence, head) pairs than SMs / 4: the recurrence takes 64-channel value slices
+    (the other tests here run 32-channel slices).  Ragged and empty sequences included."""
+    lens = [100, 64, 1, 300, 0, 129]
+    inp = _inputs(lens, 32, 128, torch.bfloat16, seed=13)
+    out, fin = run_prefill(inp, C=64)
+    check_prefill(inp, out, fin, heads=[0, 7, 31])
+
+
 def test_bf16_d64():
     inp = _inputs([130, 64, 7], 2, 64, torch.bfloat16, seed=12)
     out, fin = run_prefill(inp, C=64)

@@ -31,6 +31,16 @@ def _sw128(img: np.ndarray, rows: int) -> np.ndarray:
     return _bf16(out.reshape(rows, 128))
 
 
+def _sw64(img: np.ndarray, rows: int) -> np.ndarray:
+    """bf16 image of `rows` rows x 32 elements, 64-byte swizzle -> float array."""
+    b = img[: rows * 64].reshape(rows, 4, 16)
+    out = np.empty_like(b)
+    for r in range(rows):
+        for ch in range(4):
+            out[r, ch] = b[r, ch ^ ((r // 2) % 4)]
+    return _bf16(out.reshape(rows, 64))
+
+
 def _records(nrow, seed):
     inp = synthetic.make_prefill_inputs([nrow], 1, 128, 128, torch.bfloat16, 3.0, 0.0, seed)
     d = to_device(inp)
@@ -55,7 +65,7 @@ def test_prep_record_matches_chunked_oracle(nrow):
     P = np.concatenate([_sw128(rec[kb * 8192:(kb + 1) * 8192], 64) for kb in range(2)], axis=1)
     M = np.concatenate([_sw128(rec[16384 + kb * 16384:16384 + (kb + 1) * 16384], 128) for kb in range(2)], axis=1)
     K_res = np.concatenate([_sw128(rec[49152 + b * 8192:49152 + (b + 1) * 8192], 64) for b in range(2)], axis=1)
-    U = np.concatenate([_sw128(rec[65536 + s * 8192:65536 + (s + 1) * 8192], 64) for s in range(2)], axis=1)
+    U = np.concatenate([_sw64(rec[65536 + s * 4096:65536 + (s + 1) * 4096], 64) for s in range(4)], axis=1)
     Aqk = _sw128(rec[81920:90112], 64)
     gam = rec[90112:90624].copy().view(np.float32).astype(np.float64)
 
