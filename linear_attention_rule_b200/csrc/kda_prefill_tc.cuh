@@ -630,7 +630,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (lane == 0) bulk_s2g(rec + kRecP0 + wh * 8192 + wq * 4096, smem_u32(slot), 4096);
     }
 done:
-    if (lane == 0) bulk_wait_all();   // no copy may still read shared memory at exit
+    // no copy may still read shared memory at exit; their global writes may still be in
+    // flight (they complete before the grid does)
+    if (lane == 0) bulk_wait_read<0>();
     tc_fence_before();
     __syncthreads();
     KDA_TRACE_POINT(ptr_, 8192 + 7);
