@@ -65,13 +65,17 @@ __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + 
 __host__ inline int64_t max_chunks(int64_t total_tokens, int num_seqs) {
     return total_tokens / C + num_seqs;
 }
-// Workspace: [chunk offsets int32 (N+1)] [chunk table int2 (max_chunks)] [records
-// (max_chunks x H)]
+// Workspace: [chunk offsets int32 (N+1)] [chunk table int2 (max_chunks)] [emission slot per
+// chunk int32 (max_chunks)] [records (max_chunks x H)]
 __host__ inline size_t ws_table_offset(int num_seqs) {
     return align_up(sizeof(int32_t) * (size_t)(num_seqs + 1), 16);
 }
+__host__ inline size_t ws_emit_offset(int64_t total_tokens, int num_seqs) {
+    return align_up(ws_table_offset(num_seqs) + sizeof(int2) * (size_t)max_chunks(total_tokens, num_seqs), 16);
+}
 __host__ inline size_t ws_records_offset(int64_t total_tokens, int num_seqs) {
-    return align_up(ws_table_offset(num_seqs) + sizeof(int2) * (size_t)max_chunks(total_tokens, num_seqs),
+    return align_up(ws_emit_offset(total_tokens, num_seqs) +
+                        sizeof(int32_t) * (size_t)max_chunks(total_tokens, num_seqs),
                     1024);
 }
 __host__ inline size_t workspace_bytes(int64_t total_tokens, int num_seqs, int H) {
@@ -96,7 +100,7 @@ __device__ __forceinline__ int find_seq(const int32_t* off, int num_seqs, int c)
 // Inconsistent cu_seqlens -> KDA_ERR_BAD_SEQLENS and every count 0 (nothing downstream runs).
 __global__ void __launch_bounds__(1024)
 chunk_index_kernel(const int32_t* __restrict__ cu, int num_seqs, int64_t total,
-                   int32_t* __restrict__ off, int2* __restrict__ tab) {
+                   int32_t* __restrict__ off, int2* __restrict__ tab, int32_t* __restrict__ etab) {
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t carry;
     __shared__ int bad;
@@ -150,7 +154,32 @@ chunk_index_kernel(const int32_t* __restrict__ cu, int num_seqs, int64_t total,
         const int n = find_seq(off, num_seqs, c);
         const int t0 = cu[n] + (c - off[n]) * C;
         tab[c] = make_int2(t0, min(C, cu[n + 1] - t0));
+        if (etab) etab[c] = -1;
     }
+}
+
+// Emission slots: etab[c] = e for the chunk c that ends at emission boundary e (the state
+// after tokens cu[n] .. emit_pos[e] - 1 of its sequence n).  A boundary must end a chunk:
+// cu[n] < t <= cu[n+1] with (t - cu[n]) a multiple of C, or t = cu[n+1].  Anything else is
+// reported as KDA_ERR_BAD_EMIT_POS and emits nothing.
+__global__ void emit_index_kernel(const int32_t* __restrict__ cu, int num_seqs,
+                                  const int32_t* __restrict__ off, const int64_t* __restrict__ emit_pos,
+                                  int num_emit, int32_t* __restrict__ etab) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= num_emit || off[num_seqs] == 0) return;   // nothing to emit when cu_seqlens were bad
+    const int64_t t = emit_pos[e];
+    // sequence n: the last with cu[n] < t
+    int lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)cu[mid] < t) lo = mid; else hi = mid - 1;
+    }
+    const int64_t a = cu[lo], b = cu[lo + 1];
+    if (!(a < t && t <= b) || ((t - a) % C != 0 && t != b)) {
+        kda_set_status(KDA_ERR_BAD_EMIT_POS);
+        return;
+    }
+    etab[off[lo] + (int)((t - a - 1) / C)] = e;
 }
 
 // 2-D tiled TMA load (no multicast) of box (x, y) of `tmap` into shared memory.
@@ -695,7 +724,7 @@ template <int NV>
 __global__ void __launch_bounds__(kRecThreads, 1)
 rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __restrict__ tab,
            const uint8_t* __restrict__ records, const float* initial_state, float* final_state,
-           __nv_bfloat16* __restrict__ out) {
+           __nv_bfloat16* __restrict__ out, const int32_t* __restrict__ etab, float* emit_states) {
     using S = RecCfg<NV>;
     constexpr int NSL = S::NSL;
     const int sl = blockIdx.x % NSL;
@@ -873,6 +902,16 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
                 for (int j = 0; j < NC; ++j) Sr[j] = fmaf(gam, Sr[j], dsv[j]);
             }
             KDA_TRACE_POINT(tr, kk * 8 + 4);
+            if (etab) {   // emission boundary at the end of this chunk: the fp32 state as it is
+                const int e = etab[c_begin + kk];
+                if (e >= 0) {
+                    float* dst = emit_states + ((((size_t)e * H + h) * D + i) * D + (size_t)sl * NV + NC * cw);
+#pragma unroll
+                    for (int j4 = 0; j4 < NC / 4; ++j4)
+                        reinterpret_cast<float4*>(dst)[j4] =
+                            make_float4(Sr[4 * j4], Sr[4 * j4 + 1], Sr[4 * j4 + 2], Sr[4 * j4 + 3]);
+                }
+            }
             // the image of S_{kk+1} replaces that of S_{kk-1}, whose products (D_S(kk-1), and
             // D_O(kk-1), drained below in the previous pass) are complete
             if (more) put_state(S::SB + ((kk + 1) & 1) * S::kSImg);
@@ -978,23 +1017,30 @@ inline bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, 
 struct Workspace {
     int32_t* off;
     int2* tab;
+    int32_t* etab;
     uint8_t* records;
 };
 inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs) {
     uint8_t* base = static_cast<uint8_t*>(workspace);
     return {reinterpret_cast<int32_t*>(base), reinterpret_cast<int2*>(base + ws_table_offset(num_seqs)),
+            reinterpret_cast<int32_t*>(base + ws_emit_offset(total, num_seqs)),
             base + ws_records_offset(total, num_seqs)};
 }
 
-// Chunk table + chunk-parallel preparation.
+// Chunk table (+ emission slots when emit_pos is given) + chunk-parallel preparation.
 inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, const int32_t* cu, int num_seqs,
-                                  int64_t total, int H, void* workspace, cudaStream_t stream) {
+                                  int64_t total, int H, void* workspace, cudaStream_t stream,
+                                  const int64_t* emit_pos = nullptr, int num_emit = 0) {
     const Workspace w = split_workspace(workspace, total, num_seqs);
     cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepSmem::BYTES);
     if (e != cudaSuccess) return e;
-    chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off, w.tab);
+    chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off, w.tab,
+                                               num_emit > 0 ? w.etab : nullptr);
+    if (num_emit > 0)
+        emit_index_kernel<<<(num_emit + 255) / 256, 256, 0, stream>>>(cu, num_seqs, w.off, emit_pos,
+                                                                       num_emit, w.etab);
     if (total > 0) {
         CUtensorMap tq, tk, tv, tg;
         if (!make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1022,33 +1068,41 @@ inline int device_sm_count() {
 
 template <int NV>
 inline cudaError_t launch_scan_nv(const float* s0, float* sf, void* out, int num_seqs, const Workspace& w,
-                                  int H, cudaStream_t stream) {
+                                  int H, float* emit_states, cudaStream_t stream) {
     using R = RecCfg<NV>;
     cudaError_t e = cudaFuncSetAttribute(rec_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)R::BYTES);
     if (e != cudaSuccess) return e;
     rec_kernel<NV><<<(unsigned)num_seqs * H * R::NSL, kRecThreads, R::BYTES, stream>>>(
-        num_seqs, H, w.off, w.tab, w.records, s0, sf, static_cast<__nv_bfloat16*>(out));
+        num_seqs, H, w.off, w.tab, w.records, s0, sf, static_cast<__nv_bfloat16*>(out),
+        emit_states ? w.etab : nullptr, emit_states);
     return cudaGetLastError();
 }
 
 // Chunk-serial recurrence and the chunk outputs, over every (sequence, head, value slice):
 // 32-channel slices while 4 CTAs per (sequence, head) fit on the SMs at once, else 64.
+// emit_states (nullable) receives the states at the emission slots launch_prepare recorded.
 inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_seqs, int64_t total,
-                               int H, void* workspace, cudaStream_t stream) {
+                               int H, void* workspace, cudaStream_t stream,
+                               float* emit_states = nullptr) {
     const Workspace w = split_workspace(workspace, total, num_seqs);
     const int sms = device_sm_count();
     if ((int64_t)num_seqs * H * RecCfg<32>::NSL <= (int64_t)sms)
-        return launch_scan_nv<32>(s0, sf, out, num_seqs, w, H, stream);
-    return launch_scan_nv<64>(s0, sf, out, num_seqs, w, H, stream);
+        return launch_scan_nv<32>(s0, sf, out, num_seqs, w, H, emit_states, stream);
+    return launch_scan_nv<64>(s0, sf, out, num_seqs, w, H, emit_states, stream);
 }
 
 inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, const float* s0, const int32_t* cu,
                                   int num_seqs, int64_t total, int H, void* out, float* sf,
-                                  void* workspace, cudaStream_t stream) {
-    cudaError_t e = launch_prepare(q, k, v, g, beta, cu, num_seqs, total, H, workspace, stream);
-    if (e == cudaSuccess) e = launch_scan(s0, sf, out, num_seqs, total, H, workspace, stream);
+                                  void* workspace, cudaStream_t stream,
+                                  const int64_t* emit_pos = nullptr, int num_emit = 0,
+                                  float* emit_states = nullptr) {
+    cudaError_t e = launch_prepare(q, k, v, g, beta, cu, num_seqs, total, H, workspace, stream,
+                                   emit_pos, num_emit);
+    if (e == cudaSuccess)
+        e = launch_scan(s0, sf, out, num_seqs, total, H, workspace, stream,
+                        num_emit > 0 ? emit_states : nullptr);
     return e;
 }
 

@@ -45,7 +45,7 @@ cudaError_t dispatch_simt(int32_t dk, int32_t C, const void* q, const void* k, c
 
 extern "C" {
 
-int32_t kda_abi_version(void) { return 2; }
+int32_t kda_abi_version(void) { return 3; }
 
 const char* kda_status_string(kda_status s) {
     switch (s) {
@@ -55,6 +55,7 @@ const char* kda_status_string(kda_status s) {
         case KDA_ERR_CUDA: return "CUDA runtime error";
         case KDA_ERR_TIMEOUT: return "a bounded device wait expired";
         case KDA_ERR_BAD_SEQLENS: return "cu_seqlens inconsistent with total_tokens";
+        case KDA_ERR_BAD_EMIT_POS: return "an emission position is not a chunk boundary of a sequence";
     }
     return "unknown status";
 }
@@ -68,16 +69,24 @@ size_t kda_prefill_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_
     return kda::tc::workspace_bytes(total_tokens, num_seqs, H);
 }
 
-kda_status kda_prefill(const void* q, const void* k, const void* v, const float* g,
-                       const float* beta, const float* initial_state, const int32_t* cu_seqlens,
-                       int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t dk, int32_t dv,
-                       kda_dtype dt, void* out, float* final_state, int32_t C, void* workspace,
-                       size_t ws_bytes, kda_stream_t stream) {
-    if (num_seqs < 0 || total_tokens < 0 || H <= 0 || dk <= 0 || dv <= 0)
+static kda_status prefill_common(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, const float* initial_state,
+                                 const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                 int32_t H, int32_t dk, int32_t dv, kda_dtype dt, void* out,
+                                 float* final_state, int32_t C, const int64_t* emit_pos,
+                                 int32_t num_emit, float* emit_states, void* workspace,
+                                 size_t ws_bytes, kda_stream_t stream) {
+    if (num_seqs < 0 || total_tokens < 0 || H <= 0 || dk <= 0 || dv <= 0 || num_emit < 0)
         return KDA_ERR_INVALID_ARG;
     if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (total_tokens > INT32_MAX) return KDA_ERR_UNSUPPORTED;  // cu_seqlens is int32
     if (!supported_dim(dk, dv) || !valid_chunk(dt, C)) return KDA_ERR_UNSUPPORTED;
+    if (num_emit > 0) {
+        if (!emit_pos || !emit_states || (reinterpret_cast<uintptr_t>(emit_pos) & 7u) != 0 ||
+            !aligned16(emit_states) || num_seqs == 0)
+            return KDA_ERR_INVALID_ARG;
+        if (!tensor_core_path(dt, dk)) return KDA_ERR_UNSUPPORTED;
+    }
     if (num_seqs == 0) return KDA_OK;
     if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
@@ -94,7 +103,8 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
     cudaError_t err;
     if (tensor_core_path(dt, dk))
         err = kda::tc::launch_prefill(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
-                                      total_tokens, H, out, final_state, workspace, st);
+                                      total_tokens, H, out, final_state, workspace, st, emit_pos,
+                                      num_emit, emit_states);
     else if (dt == KDA_F32)
         err = dispatch_simt<float>(dk, C, q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
                                    total_tokens, H, out, final_state, st);
@@ -102,6 +112,27 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
         err = dispatch_simt<__nv_bfloat16>(dk, C, q, k, v, g, beta, initial_state, cu_seqlens,
                                            num_seqs, total_tokens, H, out, final_state, st);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_prefill(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                       int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                       kda_dtype dt, void* out, float* final_state, int32_t C, void* workspace,
+                       size_t ws_bytes, kda_stream_t stream) {
+    return prefill_common(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_tokens, H, dk,
+                          dv, dt, out, final_state, C, nullptr, 0, nullptr, workspace, ws_bytes, stream);
+}
+
+kda_status kda_prefill_emit(const void* q, const void* k, const void* v, const float* g,
+                            const float* beta, const float* initial_state,
+                            const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                            int32_t H, int32_t dk, int32_t dv, kda_dtype dt, void* out,
+                            float* final_state, int32_t C, const int64_t* emit_pos,
+                            int32_t num_emit, float* emit_states, void* workspace,
+                            size_t ws_bytes, kda_stream_t stream) {
+    return prefill_common(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_tokens, H, dk,
+                          dv, dt, out, final_state, C, emit_pos, num_emit, emit_states, workspace,
+                          ws_bytes, stream);
 }
 
 // Checks shared by the staged tensor-core entry points.

@@ -22,13 +22,15 @@ KDA_ERR_UNSUPPORTED = 2
 KDA_ERR_CUDA = 3
 KDA_ERR_TIMEOUT = 4
 KDA_ERR_BAD_SEQLENS = 5
+KDA_ERR_BAD_EMIT_POS = 6
 KDA_F32 = 0
 KDA_BF16 = 1
 
 # Every symbol include/libkda.h declares (checked by the CPU tests).
 EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_status_string",
             "kda_get_device_status", "kda_abi_version", "kda_prefill_noalloc",
-            "kda_prefill_prepare", "kda_prefill_scan", "kda_selftest_bounded_wait")
+            "kda_prefill_prepare", "kda_prefill_scan", "kda_selftest_bounded_wait",
+            "kda_prefill_emit")
 
 # Size of the library-owned scratch behind kda_prefill_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -72,6 +74,9 @@ def load() -> ctypes.CDLL:
     lib.kda_prefill_prepare.restype = ctypes.c_int
     lib.kda_prefill_scan.argtypes = [P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, I32, P, SZ, P]
     lib.kda_prefill_scan.restype = ctypes.c_int
+    lib.kda_prefill_emit.argtypes = [P, P, P, P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, P, P,
+                                     I32, P, I32, P, P, SZ, P]
+    lib.kda_prefill_emit.restype = ctypes.c_int
     lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P]
     lib.kda_selftest_bounded_wait.restype = ctypes.c_int
     _lib = lib
@@ -139,6 +144,32 @@ def kda_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state=None, final_sta
     if st != KDA_OK:
         raise KdaError("kda_prefill", st)
     return out, final_state
+
+
+def kda_prefill_emit(q, k, v, g, beta, cu_seqlens, out, emit_pos, emit_states,
+                     initial_state=None, final_state=None, C: int = 64,
+                     workspace: Optional[torch.Tensor] = None, stream=None):
+    """kda_prefill that also writes the state at the token boundaries emit_pos (int64 [E],
+    device) into emit_states (fp32 [E, H, dk, dv]); see kda_prefill_emit in
+    include/libkda.h."""
+    lib = load()
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    dt = _dtype_code(q)
+    if cu_seqlens.dtype != torch.int32 or emit_pos.dtype != torch.int64:
+        raise TypeError("cu_seqlens must be int32 and emit_pos int64")
+    need = int(lib.kda_prefill_workspace_size(T, N, H, dk, dv, C, dt))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.kda_prefill_emit(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                              _ptr(cu_seqlens), N, T, H, dk, dv, dt, _ptr(out), _ptr(final_state), C,
+                              _ptr(emit_pos), int(emit_pos.shape[0]), _ptr(emit_states),
+                              _ptr(workspace), ws_bytes, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError("kda_prefill_emit", st)
+    return out, final_state, emit_states
 
 
 def kda_prefill_noalloc(q, k, v, g, beta, cu_seqlens, out, initial_state=None,

@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert kda.kda_abi_version() == 2
+    assert kda.kda_abi_version() == 3
     for code in range(6):
         s = kda.kda_status_string(code)
         assert s and s != "unknown status"
@@ -123,6 +123,25 @@ def test_staged_entry_points_reject_bad_arguments(lib):
                                 P((1 << 20) + 16), need, None) == kda.KDA_ERR_INVALID_ARG
     assert lib.kda_prefill_scan(None, None, None, P(4096), 0, 0, 2, 128, 128, kda.KDA_BF16, 64, ws,
                                 need, None) == kda.KDA_OK
+
+
+def test_emit_entry_point_rejects_bad_arguments(lib):
+    P = ctypes.c_void_p
+    need = lib.kda_prefill_workspace_size(256, 1, 2, 128, 128, 64, kda.KDA_BF16)
+    ws = P(1 << 20)
+
+    def emit(dt=kda.KDA_BF16, dk=128, N=1, pos=P(4096), num=2, st=P(8192)):
+        return lib.kda_prefill_emit(P(4096), P(4096), P(4096), P(4096), P(4096), None, P(4096), N,
+                                    256, 2, dk, dk, dt, P(4096), None, 64, pos, num, st, ws, need, None)
+    assert emit(num=-1) == kda.KDA_ERR_INVALID_ARG
+    assert emit(pos=None) == kda.KDA_ERR_INVALID_ARG
+    assert emit(st=None) == kda.KDA_ERR_INVALID_ARG
+    assert emit(pos=P(4100)) == kda.KDA_ERR_INVALID_ARG       # emit_pos must be 8-byte aligned
+    assert emit(st=P(8200)) == kda.KDA_ERR_INVALID_ARG        # emit_states 16-byte aligned
+    assert emit(N=0) == kda.KDA_ERR_INVALID_ARG               # positions but no sequence
+    assert emit(dt=kda.KDA_F32) == kda.KDA_ERR_UNSUPPORTED    # emission: tensor-core path only
+    assert emit(dk=64) == kda.KDA_ERR_UNSUPPORTED
+    assert kda.kda_status_string(kda.KDA_ERR_BAD_EMIT_POS) != "unknown status"
 
 
 def test_selftest_rejects_out_of_range_limits(lib):
