@@ -22,7 +22,7 @@ template <int D, typename T>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
               const float* __restrict__ g, const float* __restrict__ beta,
-              float* __restrict__ state, T* __restrict__ out) {
+              float* __restrict__ state, T* __restrict__ out, int g_scalar) {
     constexpr int CG = D / 4;
     constexpr int RS = kDecodeThreads / CG;
     constexpr int RPT = D / RS;
@@ -48,7 +48,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         const float qq = to_f32(q[nh * D + tid]);
         sk[tid] = kk;
         sq[tid] = qq;
-        sa[tid] = expf(g[nh * D + tid]);
+        sa[tid] = expf(g_scalar ? g[nh] : g[nh * D + tid]);   // scalar gate: one decay per head
         sv[tid] = to_f32(v[nh * D + tid]);
         float kq = kk * qq;
 #pragma unroll
@@ -95,11 +95,11 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 template <int D, typename T>
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* state, void* out, int N, int H,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, bool g_scalar = false) {
     const unsigned blocks = (unsigned)N * (unsigned)H;
     decode_kernel<D, T><<<blocks, kDecodeThreads, 0, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, beta,
-        state, static_cast<T*>(out));
+        state, static_cast<T*>(out), g_scalar ? 1 : 0);
     return cudaGetLastError();
 }
 

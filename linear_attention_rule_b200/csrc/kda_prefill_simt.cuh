@@ -51,7 +51,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
                     const float* __restrict__ g, const float* __restrict__ beta,
                     const float* initial_state, const int32_t* __restrict__ cu_seqlens,
                     int num_seqs, int64_t total_tokens, int H, T* __restrict__ out,
-                    float* final_state) {
+                    float* final_state, int g_scalar) {
     constexpr int DV = DK;
     constexpr int NSL = DV / NV;
     using L = SimtSmem<DK, C, NV>;
@@ -92,7 +92,10 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
         // (1) log-decay rows of the chunk (zero past the end)
         for (int e = tid; e < C * DK; e += kSimtThreads) {
             const int r = e / DK, c = e % DK;
-            sWA[r * PK + c] = r < nrow ? g[((size_t)(t0 + r) * H + h) * DK + c] : 0.f;
+            // per-channel gate g [T, H, DK]; a scalar gate g [T, H] (Gated DeltaNet) is the same
+            // decay on every channel
+            const size_t gi = g_scalar ? (size_t)(t0 + r) * H + h : ((size_t)(t0 + r) * H + h) * DK + c;
+            sWA[r * PK + c] = r < nrow ? g[gi] : 0.f;
         }
         for (int e = tid; e < C; e += kSimtThreads)
             sB[e] = e < nrow ? beta[(size_t)(t0 + e) * H + h] : 0.f;
@@ -274,7 +277,7 @@ template <typename T, int DK, int C>
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, const float* s0, const int32_t* cu,
                                 int num_seqs, int64_t total, int H, void* out, float* sf,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, bool g_scalar = false) {
     constexpr int NV = 32;
     using L = SimtSmem<DK, C, NV>;
     auto kern = prefill_simt_kernel<T, DK, C, NV>;
@@ -284,7 +287,7 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, con
     const unsigned blocks = (unsigned)num_seqs * (unsigned)H * (unsigned)(DK / NV);
     kern<<<blocks, kSimtThreads, L::BYTES, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, beta,
-        s0, cu, num_seqs, total, H, static_cast<T*>(out), sf);
+        s0, cu, num_seqs, total, H, static_cast<T*>(out), sf, g_scalar ? 1 : 0);
     return cudaGetLastError();
 }
 

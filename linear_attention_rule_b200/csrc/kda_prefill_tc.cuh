@@ -228,12 +228,15 @@ __device__ __forceinline__ uint32_t stage_slot(int w) {
     return base + (w & 1) * 4096;
 }
 
-// One CTA per (chunk, head) unit, 2 CTAs per SM.
+// One CTA per (chunk, head) unit, 2 CTAs per SM.  kScalarG: the gate is one log-decay per
+// (token, head), g [T, H] (Gated DeltaNet, the scalar forget gate that KDA makes diagonal):
+// the same decay on every channel, loaded like beta instead of through the g tensor map.
+template <bool kScalarG>
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-            const float* __restrict__ beta, int num_seqs, int H, const int32_t* __restrict__ off,
-            const int2* __restrict__ tab, uint8_t* __restrict__ records) {
+            const float* __restrict__ g_scalar, const float* __restrict__ beta, int num_seqs, int H,
+            const int32_t* __restrict__ off, const int2* __restrict__ tab, uint8_t* __restrict__ records) {
     using S = PrepSmem;
     const int c = blockIdx.x, h = blockIdx.y;
     const int total_chunks = off[num_seqs];
@@ -259,7 +262,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (tid == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar, kPrepTx);
+        mbar_arrive_expect_tx(bar, kScalarG ? kPrepTx - 32768 : kPrepTx);
         const int x0 = h * D;
         tma_load_2d(sb + S::QD0, &tm_q, x0, t0, bar);
         tma_load_2d(sb + S::QD1, &tm_q, x0 + 64, t0, bar);
@@ -267,10 +270,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tma_load_2d(sb + S::KD1, &tm_k, x0 + 64, t0, bar);
         tma_load_2d(sb + S::V0, &tm_v, x0, t0, bar);
         tma_load_2d(sb + S::V1, &tm_v, x0 + 64, t0, bar);
-        tma_load_2d(sb + S::GR, &tm_g, x0, t0, bar);
+        if (!kScalarG) tma_load_2d(sb + S::GR, &tm_g, x0, t0, bar);
     }
     if (warp == 1) tmem_alloc(sb + S::TMEM, kPrepTmemCols);
     if (tid < C) sBeta[tid] = tid < nrow ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+    if (kScalarG && tid >= 64 && tid < 64 + C) {   // scalar gate of each row, in the g tile's place
+        const int r = tid - 64;
+        reinterpret_cast<float*>(sm + S::GR)[r] = r < nrow ? g_scalar[(size_t)(t0 + r) * H + h] : 0.f;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -295,9 +302,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
             const int r = 4 * rb + rr;
-            const float4 g0 = *reinterpret_cast<const float4*>(gt + r * D + 8 * cg);
-            const float4 g1 = *reinterpret_cast<const float4*>(gt + r * D + 8 * cg + 4);
-            const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            float gv[8];
+            if constexpr (kScalarG) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) gv[u] = gt[r];
+            } else {
+                const float4 g0 = *reinterpret_cast<const float4*>(gt + r * D + 8 * cg);
+                const float4 g1 = *reinterpret_cast<const float4*>(gt + r * D + 8 * cg + 4);
+                gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w;
+                gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
+            }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 acc[u] += r < nrow ? gv[u] : 0.f;
@@ -347,10 +361,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + o), qv);
             unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::KD0 + o), kv);
             const bool live = r < nrow;
+            // a scalar gate gives every channel the same decay: two exponentials per row
+            const float ep0 = __expf(base[0] + loc[rr][0]), em0 = __expf(-(base[0] + loc[rr][0]));
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const float a = base[u] + loc[rr][u];
-                const float ep = __expf(a), em = __expf(-a);
+                const float ep = kScalarG ? ep0 : __expf(a), em = kScalarG ? em0 : __expf(-a);
                 qd[u] = live ? qv[u] * ep : 0.f;
                 kd[u] = live ? kv[u] * ep : 0.f;
                 ki[u] = live ? kv[u] * em : 0.f;
@@ -1031,9 +1047,11 @@ inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs) {
 inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, const int32_t* cu, int num_seqs,
                                   int64_t total, int H, void* workspace, cudaStream_t stream,
-                                  const int64_t* emit_pos = nullptr, int num_emit = 0) {
+                                  const int64_t* emit_pos = nullptr, int num_emit = 0,
+                                  bool g_scalar = false) {
     const Workspace w = split_workspace(workspace, total, num_seqs);
-    cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto prep = g_scalar ? prep_kernel<true> : prep_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepSmem::BYTES);
     if (e != cudaSuccess) return e;
     chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off, w.tab,
@@ -1046,11 +1064,13 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
         if (!make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_tmap(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_tmap(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tmap(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+            (!g_scalar &&
+             !make_tmap(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE)))
             return cudaErrorInvalidValue;
+        if (g_scalar) tg = tq;   // a scalar gate is read with plain loads: this map goes unused
         dim3 grid((unsigned)max_chunks(total, num_seqs), (unsigned)H);
-        prep_kernel<<<grid, kPrepThreads, PrepSmem::BYTES, stream>>>(tq, tk, tv, tg, beta, num_seqs,
-                                                                     H, w.off, w.tab, w.records);
+        prep<<<grid, kPrepThreads, PrepSmem::BYTES, stream>>>(tq, tk, tv, tg, g_scalar ? g : nullptr,
+                                                              beta, num_seqs, H, w.off, w.tab, w.records);
     }
     return cudaGetLastError();
 }
@@ -1097,9 +1117,9 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
                                   int num_seqs, int64_t total, int H, void* out, float* sf,
                                   void* workspace, cudaStream_t stream,
                                   const int64_t* emit_pos = nullptr, int num_emit = 0,
-                                  float* emit_states = nullptr) {
+                                  float* emit_states = nullptr, bool g_scalar = false) {
     cudaError_t e = launch_prepare(q, k, v, g, beta, cu, num_seqs, total, H, workspace, stream,
-                                   emit_pos, num_emit);
+                                   emit_pos, num_emit, g_scalar);
     if (e == cudaSuccess)
         e = launch_scan(s0, sf, out, num_seqs, total, H, workspace, stream,
                         num_emit > 0 ? emit_states : nullptr);

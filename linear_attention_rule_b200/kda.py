@@ -30,7 +30,7 @@ KDA_BF16 = 1
 EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_status_string",
             "kda_get_device_status", "kda_abi_version", "kda_prefill_noalloc",
             "kda_prefill_prepare", "kda_prefill_scan", "kda_selftest_bounded_wait",
-            "kda_prefill_emit")
+            "kda_prefill_emit", "kda_prefill_gdn", "kda_decode_gdn")
 
 # Size of the library-owned scratch behind kda_prefill_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -74,6 +74,10 @@ def load() -> ctypes.CDLL:
     lib.kda_prefill_prepare.restype = ctypes.c_int
     lib.kda_prefill_scan.argtypes = [P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, I32, P, SZ, P]
     lib.kda_prefill_scan.restype = ctypes.c_int
+    lib.kda_prefill_gdn.argtypes = list(lib.kda_prefill.argtypes)
+    lib.kda_prefill_gdn.restype = ctypes.c_int
+    lib.kda_decode_gdn.argtypes = list(lib.kda_decode.argtypes)
+    lib.kda_decode_gdn.restype = ctypes.c_int
     lib.kda_prefill_emit.argtypes = [P, P, P, P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, P, P,
                                      I32, P, I32, P, P, SZ, P]
     lib.kda_prefill_emit.restype = ctypes.c_int
@@ -127,6 +131,19 @@ def kda_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state=None, final_sta
     cu_seqlens int32 [N+1] on the device; initial_state / final_state fp32 [N, H, dk, dv]
     or None.  The workspace is allocated with torch when not given.
     """
+    return _prefill("kda_prefill", q, k, v, g, beta, cu_seqlens, out, initial_state, final_state,
+                    C, workspace, stream)
+
+
+def kda_prefill_gdn(q, k, v, g, beta, cu_seqlens, out, initial_state=None, final_state=None,
+                    C: int = 64, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gated DeltaNet prefill: kda_prefill with a scalar gate g [T, H] fp32 (kda_prefill_gdn
+    in include/libkda.h)."""
+    return _prefill("kda_prefill_gdn", q, k, v, g, beta, cu_seqlens, out, initial_state,
+                    final_state, C, workspace, stream)
+
+
+def _prefill(fn, q, k, v, g, beta, cu_seqlens, out, initial_state, final_state, C, workspace, stream):
     lib = load()
     T, H, dk = q.shape
     dv = v.shape[2]
@@ -138,11 +155,11 @@ def kda_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state=None, final_sta
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
-                         _ptr(cu_seqlens), N, T, H, dk, dv, dt, _ptr(out), _ptr(final_state), C,
-                         _ptr(workspace), ws_bytes, _stream(stream))
+    st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                          _ptr(cu_seqlens), N, T, H, dk, dv, dt, _ptr(out), _ptr(final_state), C,
+                          _ptr(workspace), ws_bytes, _stream(stream))
     if st != KDA_OK:
-        raise KdaError("kda_prefill", st)
+        raise KdaError(fn, st)
     return out, final_state
 
 
@@ -233,13 +250,22 @@ def kda_selftest_bounded_wait(limit_ns: int, stream=None):
 
 def kda_decode(q, k, v, g, beta, state, out, stream=None):
     """One KDA decode step in place on `state` [N, H, dk, dv] fp32 (kda_decode in libkda.h)."""
+    return _decode("kda_decode", q, k, v, g, beta, state, out, stream)
+
+
+def kda_decode_gdn(q, k, v, g, beta, state, out, stream=None):
+    """One Gated DeltaNet decode step: kda_decode with a scalar gate g [N, H] fp32."""
+    return _decode("kda_decode_gdn", q, k, v, g, beta, state, out, stream)
+
+
+def _decode(fn, q, k, v, g, beta, state, out, stream):
     lib = load()
     N, H, dk = q.shape
     dv = v.shape[2]
-    st = lib.kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
-                        N, H, dk, dv, _dtype_code(q), _stream(stream))
+    st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
+                          N, H, dk, dv, _dtype_code(q), _stream(stream))
     if st != KDA_OK:
-        raise KdaError("kda_decode", st)
+        raise KdaError(fn, st)
     return out
 
 

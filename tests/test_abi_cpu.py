@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert kda.kda_abi_version() == 3
+    assert kda.kda_abi_version() == 4
     for code in range(6):
         s = kda.kda_status_string(code)
         assert s and s != "unknown status"
@@ -142,6 +142,18 @@ def test_emit_entry_point_rejects_bad_arguments(lib):
     assert emit(dt=kda.KDA_F32) == kda.KDA_ERR_UNSUPPORTED    # emission: tensor-core path only
     assert emit(dk=64) == kda.KDA_ERR_UNSUPPORTED
     assert kda.kda_status_string(kda.KDA_ERR_BAD_EMIT_POS) != "unknown status"
+
+
+def test_gdn_entry_points_check_arguments_like_kda(lib):
+    P = ctypes.c_void_p
+    assert lib.kda_prefill_gdn(P(4096), P(4096), P(4096), P(4096), P(4096), None, P(4096), 1, 256, 2,
+                               32, 32, kda.KDA_BF16, P(4096), None, 64, None, 0, None) == kda.KDA_ERR_UNSUPPORTED
+    assert lib.kda_prefill_gdn(P(4096), P(4096), P(4096), P(4100), P(4096), None, P(4096), 1, 256, 2,
+                               64, 64, kda.KDA_F32, P(4096), None, 64, None, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_decode_gdn(P(4096), P(4096), P(4096), None, P(4096), P(4096), P(4096), 4, 2, 128, 128,
+                              kda.KDA_BF16, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_decode_gdn(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), 0, 2, 128,
+                              128, kda.KDA_BF16, None) == kda.KDA_OK
 
 
 def test_selftest_rejects_out_of_range_limits(lib):
