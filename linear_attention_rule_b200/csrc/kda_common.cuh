@@ -12,6 +12,15 @@ __device__ int g_kda_status;
 
 __device__ __forceinline__ void kda_set_status(int s) { atomicCAS(&g_kda_status, 0, s); }
 
+// Input prologue (the layer's elementwise steps in front of KDA, fused into the kernels):
+// bit flags as in include/libkda.h (KDA_IN_*).
+constexpr uint32_t kInNormQK = 1u, kInGLogits = 2u, kInBetaLogits = 4u, kInGScalar = 8u;
+// log(sigmoid(x)) = min(x, 0) - log(1 + e^{-|x|}), without overflow for either sign
+__device__ __forceinline__ float kda_logsigmoid(float x) { return fminf(x, 0.f) - log1pf(__expf(-fabsf(x))); }
+__device__ __forceinline__ float kda_sigmoid(float x) { return 1.f / (1.f + __expf(-x)); }
+// 1 / max(||x||, 1e-12) from the squared norm (the clamp of torch's F.normalize)
+__device__ __forceinline__ float kda_inv_norm(float sumsq) { return rsqrtf(fmaxf(sumsq, 1e-24f)); }
+
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {

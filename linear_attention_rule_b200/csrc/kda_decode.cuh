@@ -18,11 +18,13 @@ constexpr int kDecodeThreads = 256;
 // One CTA per (sequence, head).  Thread t owns column group cg = t % (D/4) (one float4)
 // of rows rs, rs + RS, rs + 2 RS, ... (RS = 256 / (D/4)): a warp reads whole 512-byte
 // rows (D = 128) or two 256-byte rows (D = 64) per load.
-template <int D, typename T>
+// kPrologue: in_flags may be non-zero (the plain path compiles without the prologue).
+template <int D, typename T, bool kPrologue>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
               const float* __restrict__ g, const float* __restrict__ beta,
-              float* __restrict__ state, T* __restrict__ out, int g_scalar) {
+              float* __restrict__ state, T* __restrict__ out, uint32_t in_flags_arg) {
+    const uint32_t in_flags = kPrologue ? in_flags_arg : 0u;
     constexpr int CG = D / 4;
     constexpr int RS = kDecodeThreads / CG;
     constexpr int RPT = D / RS;
@@ -31,7 +33,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     __shared__ float sk[D], sq[D], sa[D], sv[D], su[D];
     __shared__ __align__(16) float red_p[RS][D];
     __shared__ __align__(16) float red_r[RS][D];
-    __shared__ float skq[D / 32];
+    __shared__ float skq[D / 32], skk[D / 32], sqq[D / 32];
 
     const int tid = threadIdx.x;
     const int cg = tid % CG, rs = tid / CG;
@@ -48,14 +50,35 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         const float qq = to_f32(q[nh * D + tid]);
         sk[tid] = kk;
         sq[tid] = qq;
-        sa[tid] = expf(g_scalar ? g[nh] : g[nh * D + tid]);   // scalar gate: one decay per head
+        const float gx = (in_flags & kInGScalar) ? g[nh] : g[nh * D + tid];   // scalar: one per head
+        // with gate logits x the decay is e^{logsigmoid(x)} = sigmoid(x)
+        sa[tid] = (in_flags & kInGLogits) ? kda_sigmoid(gx) : expf(gx);
         sv[tid] = to_f32(v[nh * D + tid]);
         float kq = kk * qq;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, o);
         if ((tid & 31) == 0) skq[tid >> 5] = kq;
+        if (in_flags & kInNormQK) {
+            float k2 = kk * kk, q2 = qq * qq;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                k2 += __shfl_xor_sync(0xffffffffu, k2, o);
+                q2 += __shfl_xor_sync(0xffffffffu, q2, o);
+            }
+            if ((tid & 31) == 0) { skk[tid >> 5] = k2; sqq[tid >> 5] = q2; }
+        }
     }
     __syncthreads();
+    float kq_scale = 1.f;   // k.q of the normalised vectors = k.q / (|k| |q|)
+    if (in_flags & kInNormQK) {
+        float k2 = 0.f, q2 = 0.f;
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) { k2 += skk[w]; q2 += sqq[w]; }
+        const float ik = kda_inv_norm(k2), iq = kda_inv_norm(q2);
+        kq_scale = ik * iq;
+        if (tid < D) { sk[tid] *= ik; sq[tid] *= iq; }
+        __syncthreads();
+    }
 
     float4 p = make_float4(0.f, 0.f, 0.f, 0.f), r = p;
 #pragma unroll
@@ -76,7 +99,9 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         for (int j = 0; j < RS; ++j) { pp += red_p[j][tid]; rr += red_r[j][tid]; }
 #pragma unroll
         for (int w = 0; w < D / 32; ++w) kq += skq[w];
-        const float u = beta[nh] * (sv[tid] - pp);
+        kq *= kq_scale;
+        const float b = (in_flags & kInBetaLogits) ? kda_sigmoid(beta[nh]) : beta[nh];
+        const float u = b * (sv[tid] - pp);
         su[tid] = u;
         out[nh * D + tid] = from_f32<T>(rr + u * kq);
     }
@@ -95,11 +120,12 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 template <int D, typename T>
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* state, void* out, int N, int H,
-                          cudaStream_t stream, bool g_scalar = false) {
+                          cudaStream_t stream, uint32_t in_flags = 0) {
     const unsigned blocks = (unsigned)N * (unsigned)H;
-    decode_kernel<D, T><<<blocks, kDecodeThreads, 0, stream>>>(
+    auto kern = in_flags ? decode_kernel<D, T, true> : decode_kernel<D, T, false>;
+    kern<<<blocks, kDecodeThreads, 0, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, beta,
-        state, static_cast<T*>(out), g_scalar ? 1 : 0);
+        state, static_cast<T*>(out), in_flags);
     return cudaGetLastError();
 }
 

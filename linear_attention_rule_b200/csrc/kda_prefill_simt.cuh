@@ -41,7 +41,9 @@ struct SimtSmem {
     static constexpr int SS = VV + C * NV;     // state slice [DK][NV]
     static constexpr int GM = SS + DK * NV;    // gamma [DK]
     static constexpr int BT = GM + DK;         // beta [C]
-    static constexpr int TOTAL = BT + C;
+    static constexpr int NQ = BT + C;          // 1 / ||q_r||, 1 / ||k_r|| [C] (input prologue)
+    static constexpr int NK = NQ + C;
+    static constexpr int TOTAL = NK + C;
     static constexpr size_t BYTES = sizeof(float) * TOTAL;
 };
 
@@ -51,7 +53,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
                     const float* __restrict__ g, const float* __restrict__ beta,
                     const float* initial_state, const int32_t* __restrict__ cu_seqlens,
                     int num_seqs, int64_t total_tokens, int H, T* __restrict__ out,
-                    float* final_state, int g_scalar) {
+                    float* final_state, uint32_t in_flags) {
     constexpr int DV = DK;
     constexpr int NSL = DV / NV;
     using L = SimtSmem<DK, C, NV>;
@@ -71,6 +73,9 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
     float* sS = sm + L::SS;
     float* sG = sm + L::GM;
     float* sB = sm + L::BT;
+    float* sNq = sm + L::NQ;
+    float* sNk = sm + L::NK;
+    const bool g_scalar = (in_flags & kInGScalar) != 0;
 
     const int tid = threadIdx.x;
     const int sl = blockIdx.x % NSL;
@@ -95,10 +100,33 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
             // per-channel gate g [T, H, DK]; a scalar gate g [T, H] (Gated DeltaNet) is the same
             // decay on every channel
             const size_t gi = g_scalar ? (size_t)(t0 + r) * H + h : ((size_t)(t0 + r) * H + h) * DK + c;
-            sWA[r * PK + c] = r < nrow ? g[gi] : 0.f;
+            const float x = r < nrow ? g[gi] : 0.f;
+            sWA[r * PK + c] = r < nrow && (in_flags & kInGLogits) ? kda_logsigmoid(x) : x;
         }
-        for (int e = tid; e < C; e += kSimtThreads)
-            sB[e] = e < nrow ? beta[(size_t)(t0 + e) * H + h] : 0.f;
+        for (int e = tid; e < C; e += kSimtThreads) {
+            const float b = e < nrow ? beta[(size_t)(t0 + e) * H + h] : 0.f;
+            sB[e] = e < nrow && (in_flags & kInBetaLogits) ? kda_sigmoid(b) : b;
+        }
+        if (in_flags & kInNormQK) {   // row norms of q and k, one warp per row
+            const int warp = tid >> 5, lane = tid & 31;
+            for (int r = warp; r < C; r += kSimtThreads / 32) {
+                float sq = 0.f, sk = 0.f;
+                if (r < nrow) {
+                    for (int c = lane; c < DK; c += 32) {
+                        const size_t off = ((size_t)(t0 + r) * H + h) * DK + c;
+                        const float qq = to_f32(q[off]), kk = to_f32(k[off]);
+                        sq += qq * qq;
+                        sk += kk * kk;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                }
+                if (lane == 0) { sNq[r] = kda_inv_norm(sq); sNk[r] = kda_inv_norm(sk); }
+            }
+        }
         for (int e = tid; e < C * NV; e += kSimtThreads) {
             const int r = e / NV, j = e % NV;
             sV[e] = r < nrow ? to_f32(v[((size_t)(t0 + r) * H + h) * DV + sl * NV + j]) : 0.f;
@@ -124,6 +152,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
                 const size_t off = ((size_t)(t0 + r) * H + h) * DK + c;
                 qq = to_f32(q[off]);
                 kk = to_f32(k[off]);
+                if (in_flags & kInNormQK) { qq *= sNq[r]; kk *= sNk[r]; }
             }
             const float a = sWA[r * PK + c];
             const float ep = expf(a), em = expf(-a);
@@ -277,7 +306,7 @@ template <typename T, int DK, int C>
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, const float* s0, const int32_t* cu,
                                 int num_seqs, int64_t total, int H, void* out, float* sf,
-                                cudaStream_t stream, bool g_scalar = false) {
+                                cudaStream_t stream, uint32_t in_flags = 0) {
     constexpr int NV = 32;
     using L = SimtSmem<DK, C, NV>;
     auto kern = prefill_simt_kernel<T, DK, C, NV>;
@@ -287,7 +316,7 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, con
     const unsigned blocks = (unsigned)num_seqs * (unsigned)H * (unsigned)(DK / NV);
     kern<<<blocks, kSimtThreads, L::BYTES, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, beta,
-        s0, cu, num_seqs, total, H, static_cast<T*>(out), sf, g_scalar ? 1 : 0);
+        s0, cu, num_seqs, total, H, static_cast<T*>(out), sf, in_flags);
     return cudaGetLastError();
 }
 

@@ -204,8 +204,9 @@ struct PrepSmem {
     static constexpr uint32_t ABAR = GR, AQK = GR + 8192, LI = GR + 16384;   // LI: [64][68]
     static constexpr uint32_t XCH = GR + 33792;      // decay partials [8][128]; later T [32][36]
     static constexpr uint32_t BETA = XCH + 4608;     // [64]
-    static constexpr uint32_t BAR = BETA + 256;
-    static constexpr uint32_t TMEM = BAR + 8;
+    static constexpr uint32_t BAR = BETA + 256;       // TMA and products in order
+    static constexpr uint32_t BAR2 = BAR + 8;         // the last product (Aqk W)
+    static constexpr uint32_t TMEM = BAR2 + 8;
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;  // + alignment slack
 };
 constexpr int kLP = 68;                                   // row pitch of L / INV (16-byte rows)
@@ -231,12 +232,15 @@ __device__ __forceinline__ uint32_t stage_slot(int w) {
 // One CTA per (chunk, head) unit, 2 CTAs per SM.  kScalarG: the gate is one log-decay per
 // (token, head), g [T, H] (Gated DeltaNet, the scalar forget gate that KDA makes diagonal):
 // the same decay on every channel, loaded like beta instead of through the g tensor map.
-template <bool kScalarG>
+// kPrologue: in_flags may hold KDA_IN_* prologue bits (the plain path compiles without them).
+template <bool kScalarG, bool kPrologue>
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
             const float* __restrict__ g_scalar, const float* __restrict__ beta, int num_seqs, int H,
-            const int32_t* __restrict__ off, const int2* __restrict__ tab, uint8_t* __restrict__ records) {
+            const int32_t* __restrict__ off, const int2* __restrict__ tab, uint8_t* __restrict__ records,
+            uint32_t in_flags_arg) {
+    const uint32_t in_flags = kPrologue ? in_flags_arg : 0u;
     using S = PrepSmem;
     const int c = blockIdx.x, h = blockIdx.y;
     const int total_chunks = off[num_seqs];
@@ -261,6 +265,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // barrier is initialised and the copies issued by the same thread, before anything else
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(bar + 8, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(bar, kScalarG ? kPrepTx - 32768 : kPrepTx);
         const int x0 = h * D;
@@ -273,10 +278,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (!kScalarG) tma_load_2d(sb + S::GR, &tm_g, x0, t0, bar);
     }
     if (warp == 1) tmem_alloc(sb + S::TMEM, kPrepTmemCols);
-    if (tid < C) sBeta[tid] = tid < nrow ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+    if (tid < C) {
+        const float b = tid < nrow ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+        sBeta[tid] = tid < nrow && (in_flags & kInBetaLogits) ? kda_sigmoid(b) : b;
+    }
     if (kScalarG && tid >= 64 && tid < 64 + C) {   // scalar gate of each row, in the g tile's place
         const int r = tid - 64;
-        reinterpret_cast<float*>(sm + S::GR)[r] = r < nrow ? g_scalar[(size_t)(t0 + r) * H + h] : 0.f;
+        const float x = r < nrow ? g_scalar[(size_t)(t0 + r) * H + h] : 0.f;
+        reinterpret_cast<float*>(sm + S::GR)[r] = r < nrow && (in_flags & kInGLogits) ? kda_logsigmoid(x) : x;
     }
     tc_fence_before();
     __syncthreads();
@@ -311,6 +320,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const float4 g1 = *reinterpret_cast<const float4*>(gt + r * D + 8 * cg + 4);
                 gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w;
                 gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
+                if (in_flags & kInGLogits) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) gv[u] = kda_logsigmoid(gv[u]);
+                }
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -360,6 +373,19 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             float qv[8], kv[8], qd[8], kd[8], ki[8];
             unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + o), qv);
             unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::KD0 + o), kv);
+            if (in_flags & kInNormQK) {   // the 16 lanes of this half-warp hold the row's 128 channels
+                float sq = 0.f, sk = 0.f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) { sq += qv[u] * qv[u]; sk += kv[u] * kv[u]; }
+#pragma unroll
+                for (int o2 = 1; o2 < 16; o2 <<= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, o2);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, o2);
+                }
+                const float iq = kda_inv_norm(sq), ik = kda_inv_norm(sk);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) { qv[u] *= iq; kv[u] *= ik; }
+            }
             const bool live = r < nrow;
             // a scalar gate gives every channel the same decay: two exponentials per row
             const float ep0 = __expf(base[0] + loc[rr][0]), em0 = __expf(-(base[0] + loc[rr][0]));
@@ -596,18 +622,25 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     KDA_TRACE_POINT(ptr_, 8192 + 5);
 
-    // ---- (5) -M = K_res^T W -> TMEM [0, 128) ----
+    // ---- (5) -M = K_res^T W -> TMEM [0, 128) and Aqk W -> TMEM [128, 256) (lanes 0-63), issued
+    // back to back: the second product runs while the first is drained ----
     if (tid == 0) {
         tc_fence_after();
         // U is final: its image (four value slices) goes to the record as it is
         bulk_s2g(rec + kRecU, sb + S::V0, 8192);
         bulk_s2g(rec + kRecU + 8192, sb + S::V1, 8192);
-        constexpr uint32_t id = idesc_bf16(128, 128, true, true);
+        constexpr uint32_t idM = idesc_bf16(128, 128, true, true);
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
             umma_bf16(tmem, smem_desc(sb + S::KI0 + ks * 2048, S::BLK, 1024, kSwizzle128),
-                      smem_desc(sb + S::KD0 + ks * 2048, S::BLK, 1024, kSwizzle128), id, ks > 0);
+                      smem_desc(sb + S::KD0 + ks * 2048, S::BLK, 1024, kSwizzle128), idM, ks > 0);
         umma_commit(bar);
+        constexpr uint32_t idP = idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+            umma_bf16(tmem + 128, smem_desc(sb + S::AQK + ks * 32, 16, 1024, kSwizzle128),
+                      smem_desc(sb + S::KD0 + ks * 2048, S::BLK, 1024, kSwizzle128), idP, ks > 0);
+        umma_commit(bar + 8);
         bulk_wait_read<2>();   // the K_res / Aqk copies have read their sources
     }
     ok = mbar_wait(bar, phase);
@@ -615,7 +648,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tc_fence_after();
     if (!prep_sync_ok(ok, tid)) goto done;
     {
-        // Drain: warp (wq, wh) turns its 32 TMEM lanes x 64 columns (K block wh of M, rows
+        // Drain of M: warp (wq, wh) turns its 32 TMEM lanes x 64 columns (K block wh of M, rows
         // i = 32 wq ..) into a 4 KB piece of the record (32 complete swizzled rows) staged in a
         // private, now unused 4 KB slot, and copies it out with one bulk copy.
         uint8_t* slot = sm + stage_slot(warp);
@@ -632,47 +665,35 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         __syncwarp();
         if (lane == 0) bulk_s2g(rec + kRecM0 + wh * 16384 + wq * 4096, smem_u32(slot), 4096);
     }
-    tc_fence_before();
-    __syncthreads();
     KDA_TRACE_POINT(ptr_, 8192 + 6);
-
-    // ---- (6) Aqk W -> TMEM [0, 128) (lanes 0-63); P = Q_dec - Aqk W ----
-    if (tid == 0) {
-        tc_fence_after();
-        constexpr uint32_t id = idesc_bf16(128, 128, false, true);
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-            umma_bf16(tmem, smem_desc(sb + S::AQK + ks * 32, 16, 1024, kSwizzle128),
-                      smem_desc(sb + S::KD0 + ks * 2048, S::BLK, 1024, kSwizzle128), id, ks > 0);
-        umma_commit(bar);
-    }
-    ok = mbar_wait(bar, phase);
-    phase ^= 1;
-    tc_fence_after();
-    if (!prep_sync_ok(ok, tid)) goto done;
     if (wq < 2) {
-        // rows r = 32 wq .., K block wh of P
-        const int r = 32 * wq + lane;
-        uint8_t* slot = sm + stage_slot(warp);
-        float d[64];
-        tmem_ld32(tl + 64 * wh, *reinterpret_cast<float(*)[32]>(&d[0]));
-        tmem_ld32(tl + 64 * wh + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
-        tmem_wait_ld();
+        // Drain of P = Q_dec - Aqk W: rows r = 32 wq .., K block wh.  Both products have read W
+        // by now, so its space holds the staging slots.
+        ok = __all_sync(0xffffffffu, mbar_wait(bar + 8, 0));
+        if (!ok) {
+            if (lane == 0) kda_set_status(KDA_ERR_TIMEOUT);
+        } else {
+            tc_fence_after();
+            const int r = 32 * wq + lane;
+            uint8_t* slot = sm + (wh ? S::KD1 : S::KD0) + wq * 4096;
+            float d[64];
+            tmem_ld32(tl + 128 + 64 * wh, *reinterpret_cast<float(*)[32]>(&d[0]));
+            tmem_ld32(tl + 128 + 64 * wh + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
+            tmem_wait_ld();
 #pragma unroll
-        for (int cb = 0; cb < 8; ++cb) {
-            float qv[8];
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + wh * S::BLK + sw128_off(r, cb)), qv);
+            for (int cb = 0; cb < 8; ++cb) {
+                float qv[8];
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + wh * S::BLK + sw128_off(r, cb)), qv);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) d[8 * cb + u] = qv[u] - d[8 * cb + u];
+                for (int u = 0; u < 8; ++u) d[8 * cb + u] = qv[u] - d[8 * cb + u];
+            }
+#pragma unroll
+            for (int cb = 0; cb < 8; ++cb)
+                *reinterpret_cast<uint4*>(slot + sw128_off(lane, cb)) = pack_bf16x8(&d[8 * cb]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) bulk_s2g(rec + kRecP0 + wh * 8192 + wq * 4096, smem_u32(slot), 4096);
         }
-        if (lane == 0) bulk_wait_read<0>();   // this warp's M piece has left the slot
-        __syncwarp();
-#pragma unroll
-        for (int cb = 0; cb < 8; ++cb)
-            *reinterpret_cast<uint4*>(slot + sw128_off(lane, cb)) = pack_bf16x8(&d[8 * cb]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) bulk_s2g(rec + kRecP0 + wh * 8192 + wq * 4096, smem_u32(slot), 4096);
     }
 done:
     // no copy may still read shared memory at exit; their global writes may still be in
@@ -1048,9 +1069,12 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
                                   const float* beta, const int32_t* cu, int num_seqs,
                                   int64_t total, int H, void* workspace, cudaStream_t stream,
                                   const int64_t* emit_pos = nullptr, int num_emit = 0,
-                                  bool g_scalar = false) {
+                                  uint32_t in_flags = 0) {
+    const bool g_scalar = (in_flags & kInGScalar) != 0;
     const Workspace w = split_workspace(workspace, total, num_seqs);
-    auto prep = g_scalar ? prep_kernel<true> : prep_kernel<false>;
+    const bool pro = (in_flags & ~kInGScalar) != 0;
+    auto prep = g_scalar ? (pro ? prep_kernel<true, true> : prep_kernel<true, false>)
+                         : (pro ? prep_kernel<false, true> : prep_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepSmem::BYTES);
     if (e != cudaSuccess) return e;
@@ -1070,7 +1094,8 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
         if (g_scalar) tg = tq;   // a scalar gate is read with plain loads: this map goes unused
         dim3 grid((unsigned)max_chunks(total, num_seqs), (unsigned)H);
         prep<<<grid, kPrepThreads, PrepSmem::BYTES, stream>>>(tq, tk, tv, tg, g_scalar ? g : nullptr,
-                                                              beta, num_seqs, H, w.off, w.tab, w.records);
+                                                              beta, num_seqs, H, w.off, w.tab, w.records,
+                                                              in_flags);
     }
     return cudaGetLastError();
 }
@@ -1117,9 +1142,9 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
                                   int num_seqs, int64_t total, int H, void* out, float* sf,
                                   void* workspace, cudaStream_t stream,
                                   const int64_t* emit_pos = nullptr, int num_emit = 0,
-                                  float* emit_states = nullptr, bool g_scalar = false) {
+                                  float* emit_states = nullptr, uint32_t in_flags = 0) {
     cudaError_t e = launch_prepare(q, k, v, g, beta, cu, num_seqs, total, H, workspace, stream,
-                                   emit_pos, num_emit, g_scalar);
+                                   emit_pos, num_emit, in_flags);
     if (e == cudaSuccess)
         e = launch_scan(s0, sf, out, num_seqs, total, H, workspace, stream,
                         num_emit > 0 ? emit_states : nullptr);

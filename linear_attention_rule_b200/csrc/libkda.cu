@@ -30,11 +30,11 @@ template <typename T>
 cudaError_t dispatch_simt(int32_t dk, int32_t C, const void* q, const void* k, const void* v,
                           const float* g, const float* beta, const float* s0, const int32_t* cu,
                           int num_seqs, int64_t total, int H, void* out, float* sf,
-                          cudaStream_t st, bool g_scalar) {
+                          cudaStream_t st, uint32_t in_flags) {
 #define KDA_SIMT_CASE(D, CC)                                                                  \
     if (dk == D && C == CC)                                                                   \
         return kda::launch_prefill_simt<T, D, CC>(q, k, v, g, beta, s0, cu, num_seqs, total, H, \
-                                                  out, sf, st, g_scalar);
+                                                  out, sf, st, in_flags);
     KDA_SIMT_CASE(64, 16) KDA_SIMT_CASE(64, 32) KDA_SIMT_CASE(64, 64)
     KDA_SIMT_CASE(128, 16) KDA_SIMT_CASE(128, 32) KDA_SIMT_CASE(128, 64)
 #undef KDA_SIMT_CASE
@@ -45,7 +45,7 @@ cudaError_t dispatch_simt(int32_t dk, int32_t C, const void* q, const void* k, c
 
 extern "C" {
 
-int32_t kda_abi_version(void) { return 4; }
+int32_t kda_abi_version(void) { return 5; }
 
 const char* kda_status_string(kda_status s) {
     switch (s) {
@@ -75,8 +75,10 @@ static kda_status prefill_common(const void* q, const void* k, const void* v, co
                                  int32_t H, int32_t dk, int32_t dv, kda_dtype dt, void* out,
                                  float* final_state, int32_t C, const int64_t* emit_pos,
                                  int32_t num_emit, float* emit_states, void* workspace,
-                                 size_t ws_bytes, kda_stream_t stream, bool g_scalar) {
+                                 size_t ws_bytes, kda_stream_t stream, uint32_t in_flags) {
     if (num_seqs < 0 || total_tokens < 0 || H <= 0 || dk <= 0 || dv <= 0 || num_emit < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (in_flags & ~(uint32_t)(KDA_IN_NORMALIZE_QK | KDA_IN_G_LOGITS | KDA_IN_BETA_LOGITS | KDA_IN_G_SCALAR))
         return KDA_ERR_INVALID_ARG;
     if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (total_tokens > INT32_MAX) return KDA_ERR_UNSUPPORTED;  // cu_seqlens is int32
@@ -104,13 +106,13 @@ static kda_status prefill_common(const void* q, const void* k, const void* v, co
     if (tensor_core_path(dt, dk))
         err = kda::tc::launch_prefill(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
                                       total_tokens, H, out, final_state, workspace, st, emit_pos,
-                                      num_emit, emit_states, g_scalar);
+                                      num_emit, emit_states, in_flags);
     else if (dt == KDA_F32)
         err = dispatch_simt<float>(dk, C, q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
-                                   total_tokens, H, out, final_state, st, g_scalar);
+                                   total_tokens, H, out, final_state, st, in_flags);
     else
         err = dispatch_simt<__nv_bfloat16>(dk, C, q, k, v, g, beta, initial_state, cu_seqlens,
-                                           num_seqs, total_tokens, H, out, final_state, st, g_scalar);
+                                           num_seqs, total_tokens, H, out, final_state, st, in_flags);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -121,7 +123,7 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
                        size_t ws_bytes, kda_stream_t stream) {
     return prefill_common(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_tokens, H, dk,
                           dv, dt, out, final_state, C, nullptr, 0, nullptr, workspace, ws_bytes, stream,
-                          false);
+                          0u);
 }
 
 kda_status kda_prefill_gdn(const void* q, const void* k, const void* v, const float* g,
@@ -131,7 +133,18 @@ kda_status kda_prefill_gdn(const void* q, const void* k, const void* v, const fl
                            size_t ws_bytes, kda_stream_t stream) {
     return prefill_common(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_tokens, H, dk,
                           dv, dt, out, final_state, C, nullptr, 0, nullptr, workspace, ws_bytes, stream,
-                          true);
+                          (uint32_t)KDA_IN_G_SCALAR);
+}
+
+kda_status kda_prefill_ex(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                          int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                          kda_dtype dt, void* out, float* final_state, int32_t C, uint32_t in_flags,
+                          const int64_t* emit_pos, int32_t num_emit, float* emit_states,
+                          void* workspace, size_t ws_bytes, kda_stream_t stream) {
+    return prefill_common(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_tokens, H, dk,
+                          dv, dt, out, final_state, C, emit_pos, num_emit, emit_states, workspace,
+                          ws_bytes, stream, in_flags);
 }
 
 kda_status kda_prefill_emit(const void* q, const void* k, const void* v, const float* g,
@@ -143,7 +156,7 @@ kda_status kda_prefill_emit(const void* q, const void* k, const void* v, const f
                             size_t ws_bytes, kda_stream_t stream) {
     return prefill_common(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_tokens, H, dk,
                           dv, dt, out, final_state, C, emit_pos, num_emit, emit_states, workspace,
-                          ws_bytes, stream, false);
+                          ws_bytes, stream, 0u);
 }
 
 // Checks shared by the staged tensor-core entry points.
@@ -201,8 +214,10 @@ kda_status kda_selftest_bounded_wait(uint64_t limit_ns, kda_stream_t stream) {
 
 static kda_status decode_common(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, float* state_inout, void* out, int32_t N, int32_t H,
-                                int32_t dk, int32_t dv, kda_dtype dt, kda_stream_t stream, bool g_scalar) {
+                                int32_t dk, int32_t dv, kda_dtype dt, kda_stream_t stream, uint32_t in_flags) {
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (in_flags & ~(uint32_t)(KDA_IN_NORMALIZE_QK | KDA_IN_G_LOGITS | KDA_IN_BETA_LOGITS | KDA_IN_G_SCALAR))
+        return KDA_ERR_INVALID_ARG;
     if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (!supported_dim(dk, dv)) return KDA_ERR_UNSUPPORTED;
     if (N == 0) return KDA_OK;
@@ -214,26 +229,33 @@ static kda_status decode_common(const void* q, const void* k, const void* v, con
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t err;
     if (dt == KDA_F32)
-        err = dk == 64 ? kda::launch_decode<64, float>(q, k, v, g, beta, state_inout, out, N, H, st, g_scalar)
-                       : kda::launch_decode<128, float>(q, k, v, g, beta, state_inout, out, N, H, st, g_scalar);
+        err = dk == 64 ? kda::launch_decode<64, float>(q, k, v, g, beta, state_inout, out, N, H, st, in_flags)
+                       : kda::launch_decode<128, float>(q, k, v, g, beta, state_inout, out, N, H, st, in_flags);
     else
         err = dk == 64 ? kda::launch_decode<64, __nv_bfloat16>(q, k, v, g, beta, state_inout, out, N, H, st,
-                                                               g_scalar)
+                                                               in_flags)
                        : kda::launch_decode<128, __nv_bfloat16>(q, k, v, g, beta, state_inout, out, N, H,
-                                                                st, g_scalar);
+                                                                st, in_flags);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status kda_decode(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* state_inout, void* out, int32_t N, int32_t H,
                       int32_t dk, int32_t dv, kda_dtype dt, kda_stream_t stream) {
-    return decode_common(q, k, v, g, beta, state_inout, out, N, H, dk, dv, dt, stream, false);
+    return decode_common(q, k, v, g, beta, state_inout, out, N, H, dk, dv, dt, stream, 0u);
 }
 
 kda_status kda_decode_gdn(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* state_inout, void* out, int32_t N, int32_t H,
                           int32_t dk, int32_t dv, kda_dtype dt, kda_stream_t stream) {
-    return decode_common(q, k, v, g, beta, state_inout, out, N, H, dk, dv, dt, stream, true);
+    return decode_common(q, k, v, g, beta, state_inout, out, N, H, dk, dv, dt, stream,
+                         (uint32_t)KDA_IN_G_SCALAR);
+}
+
+kda_status kda_decode_ex(const void* q, const void* k, const void* v, const float* g,
+                         const float* beta, float* state_inout, void* out, int32_t N, int32_t H,
+                         int32_t dk, int32_t dv, kda_dtype dt, uint32_t in_flags, kda_stream_t stream) {
+    return decode_common(q, k, v, g, beta, state_inout, out, N, H, dk, dv, dt, stream, in_flags);
 }
 
 #ifdef KDA_TRACE

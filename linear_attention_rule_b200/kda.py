@@ -23,6 +23,11 @@ KDA_ERR_CUDA = 3
 KDA_ERR_TIMEOUT = 4
 KDA_ERR_BAD_SEQLENS = 5
 KDA_ERR_BAD_EMIT_POS = 6
+# input prologue flags (kda_prefill_ex / kda_decode_ex)
+KDA_IN_NORMALIZE_QK = 1
+KDA_IN_G_LOGITS = 2
+KDA_IN_BETA_LOGITS = 4
+KDA_IN_G_SCALAR = 8
 KDA_F32 = 0
 KDA_BF16 = 1
 
@@ -30,7 +35,8 @@ KDA_BF16 = 1
 EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_status_string",
             "kda_get_device_status", "kda_abi_version", "kda_prefill_noalloc",
             "kda_prefill_prepare", "kda_prefill_scan", "kda_selftest_bounded_wait",
-            "kda_prefill_emit", "kda_prefill_gdn", "kda_decode_gdn")
+            "kda_prefill_emit", "kda_prefill_gdn", "kda_decode_gdn", "kda_prefill_ex",
+            "kda_decode_ex")
 
 # Size of the library-owned scratch behind kda_prefill_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -74,6 +80,12 @@ def load() -> ctypes.CDLL:
     lib.kda_prefill_prepare.restype = ctypes.c_int
     lib.kda_prefill_scan.argtypes = [P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, I32, P, SZ, P]
     lib.kda_prefill_scan.restype = ctypes.c_int
+    U32 = ctypes.c_uint32
+    lib.kda_prefill_ex.argtypes = [P, P, P, P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, P, P,
+                                   I32, U32, P, I32, P, P, SZ, P]
+    lib.kda_prefill_ex.restype = ctypes.c_int
+    lib.kda_decode_ex.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, ctypes.c_int, U32, P]
+    lib.kda_decode_ex.restype = ctypes.c_int
     lib.kda_prefill_gdn.argtypes = list(lib.kda_prefill.argtypes)
     lib.kda_prefill_gdn.restype = ctypes.c_int
     lib.kda_decode_gdn.argtypes = list(lib.kda_decode.argtypes)
@@ -189,6 +201,30 @@ def kda_prefill_emit(q, k, v, g, beta, cu_seqlens, out, emit_pos, emit_states,
     return out, final_state, emit_states
 
 
+def kda_prefill_ex(q, k, v, g, beta, cu_seqlens, out, in_flags: int = 0, initial_state=None,
+                   final_state=None, emit_pos=None, emit_states=None, C: int = 64,
+                   workspace: Optional[torch.Tensor] = None, stream=None):
+    """kda_prefill with an input prologue (KDA_IN_* flags) and optional state emission
+    (kda_prefill_ex in include/libkda.h).  With KDA_IN_G_SCALAR, g is [T, H]."""
+    lib = load()
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    dt = _dtype_code(q)
+    need = int(lib.kda_prefill_workspace_size(T, N, H, dk, dv, C, dt))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    num_emit = 0 if emit_pos is None else int(emit_pos.shape[0])
+    st = lib.kda_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                            _ptr(cu_seqlens), N, T, H, dk, dv, dt, _ptr(out), _ptr(final_state), C,
+                            int(in_flags), _ptr(emit_pos), num_emit, _ptr(emit_states),
+                            _ptr(workspace), ws_bytes, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError("kda_prefill_ex", st)
+    return out, final_state
+
+
 def kda_prefill_noalloc(q, k, v, g, beta, cu_seqlens, out, initial_state=None,
                         final_state=None, C: int = 64, stream=None):
     """kda_prefill without a workspace, for callers that cannot allocate device memory
@@ -256,6 +292,18 @@ def kda_decode(q, k, v, g, beta, state, out, stream=None):
 def kda_decode_gdn(q, k, v, g, beta, state, out, stream=None):
     """One Gated DeltaNet decode step: kda_decode with a scalar gate g [N, H] fp32."""
     return _decode("kda_decode_gdn", q, k, v, g, beta, state, out, stream)
+
+
+def kda_decode_ex(q, k, v, g, beta, state, out, in_flags: int = 0, stream=None):
+    """kda_decode with an input prologue (KDA_IN_* flags; with KDA_IN_G_SCALAR g is [N, H])."""
+    lib = load()
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    st = lib.kda_decode_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
+                           N, H, dk, dv, _dtype_code(q), int(in_flags), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError("kda_decode_ex", st)
+    return out
 
 
 def _decode(fn, q, k, v, g, beta, state, out, stream):

@@ -190,3 +190,30 @@ def make_prefill_inputs_device(lengths: Sequence[int], H: int, dk: int, dv: int,
             s0[:, h] = cpu["s0"][:, j].to(device)
     return dict(q=q, k=k, v=v, g=g, beta=beta, cu_seqlens=cu_seqlens_of(lengths).to(device),
                 s0=s0, cpu=cpu)
+
+
+def make_raw_prefill_inputs(lengths: Sequence[int], H: int, dk: int, dv: int, dtype: torch.dtype,
+                            g_mean: float, s0_std: float, seed: int, scalar_gate: bool = False) -> dict:
+    """Inputs as the layer hands them over before its elementwise prologue: q, k ~ N(0, 1)
+    not normalised (cast to `dtype`), v ~ N(0, 1); gate logits ~ N(g_mean, 1) fp32 [T, H, dk]
+    (or [T, H] with scalar_gate); beta logits ~ N(0, 1) fp32 [T, H]; initial state as in
+    make_prefill_inputs.  One seeded CPU generator per head, in the order q, k, v,
+    beta-logits, gate-logits, initial state."""
+    T = int(sum(lengths))
+    N = len(lengths)
+    q = torch.empty(T, H, dk, dtype=dtype)
+    k = torch.empty(T, H, dk, dtype=dtype)
+    v = torch.empty(T, H, dv, dtype=dtype)
+    g = torch.empty((T, H) if scalar_gate else (T, H, dk), dtype=torch.float32)
+    beta = torch.empty(T, H, dtype=torch.float32)
+    s0 = torch.empty(N, H, dk, dv, dtype=torch.float32) if s0_std > 0 else None
+    for h in range(H):
+        gen = _head_generator(seed, h)
+        q[:, h] = torch.randn(T, dk, generator=gen).to(dtype)
+        k[:, h] = torch.randn(T, dk, generator=gen).to(dtype)
+        v[:, h] = torch.randn(T, dv, generator=gen).to(dtype)
+        beta[:, h] = torch.randn(T, generator=gen)
+        g[:, h] = g_mean + torch.randn(*((T,) if scalar_gate else (T, dk)), generator=gen)
+        if s0 is not None:
+            s0[:, h] = s0_std * torch.randn(N, dk, dv, generator=gen)
+    return dict(q=q, k=k, v=v, g=g, beta=beta, cu_seqlens=cu_seqlens_of(lengths), s0=s0)

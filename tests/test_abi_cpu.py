@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert kda.kda_abi_version() == 4
+    assert kda.kda_abi_version() == 5
     for code in range(6):
         s = kda.kda_status_string(code)
         assert s and s != "unknown status"
@@ -154,6 +154,21 @@ def test_gdn_entry_points_check_arguments_like_kda(lib):
                               kda.KDA_BF16, None) == kda.KDA_ERR_INVALID_ARG
     assert lib.kda_decode_gdn(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), 0, 2, 128,
                               128, kda.KDA_BF16, None) == kda.KDA_OK
+
+
+def test_prologue_entry_points_reject_unknown_flags(lib):
+    P = ctypes.c_void_p
+    need = lib.kda_prefill_workspace_size(256, 1, 2, 128, 128, 64, kda.KDA_BF16)
+    ex = lambda flags: lib.kda_prefill_ex(P(4096), P(4096), P(4096), P(4096), P(4096), None, P(4096), 1, 256,
+                                          2, 128, 128, kda.KDA_BF16, P(4096), None, 64, flags, None, 0, None,
+                                          P(1 << 20), need, None)
+    assert ex(16) == kda.KDA_ERR_INVALID_ARG
+    assert ex(1 << 31) == kda.KDA_ERR_INVALID_ARG
+    dec = lambda flags: lib.kda_decode_ex(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), 2,
+                                          2, 128, 128, kda.KDA_BF16, flags, None)
+    assert dec(32) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_decode_ex(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), 0, 2, 128, 128,
+                             kda.KDA_BF16, 15, None) == kda.KDA_OK
 
 
 def test_selftest_rejects_out_of_range_limits(lib):
