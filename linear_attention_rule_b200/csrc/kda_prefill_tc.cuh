@@ -239,14 +239,22 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
             const float* __restrict__ g_scalar, const float* __restrict__ beta, int num_seqs, int H,
             const int32_t* __restrict__ off, const int2* __restrict__ tab, uint8_t* __restrict__ records,
-            uint32_t in_flags_arg) {
+            uint32_t in_flags_arg, int64_t total) {
     const uint32_t in_flags = kPrologue ? in_flags_arg : 0u;
     using S = PrepSmem;
     const int c = blockIdx.x, h = blockIdx.y;
-    const int total_chunks = off[num_seqs];
-    const int2 e = tab[c];   // in bounds for every c < max_chunks; meaningful for c < total
+    int total_chunks, t0, nrow;
+    if (num_seqs == 1) {   // one sequence: chunk c is tokens 64 c .., no table load before the TMA
+        total_chunks = (int)((total + C - 1) / C);
+        t0 = c * C;
+        nrow = (int)(total - t0 < C ? total - t0 : C);
+    } else {
+        total_chunks = off[num_seqs];
+        const int2 e = tab[c];   // in bounds for every c < max_chunks; meaningful for c < total
+        t0 = e.x;
+        nrow = e.y;
+    }
     if (c >= total_chunks) return;
-    const int t0 = e.x, nrow = e.y;
     uint8_t* rec = records + ((size_t)c * H + h) * kRecBytes;
 
     extern __shared__ uint8_t smem_raw[];
@@ -472,6 +480,41 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             __syncwarp();
 #pragma unroll
             for (int r = 0; r < 16; ++r) sLI[(16 * b + r) * kLP + 16 * b + j] = x[r];
+            __syncwarp();
+            // 16 -> 32 for the same warp's block pair (warp 0: blocks 0, 1; warp 5: 2, 3):
+            // X = -D_hi (L_lo D_lo) into rows R .. R+15, columns Cc .. Cc+15; lane = (row r,
+            // 8 columns); T through the scratch rows 16 p .. 16 p + 15
+            {
+                float* sT = sX;
+                const int p = warp == 5 ? 1 : 0, r = lane >> 1, c8 = 8 * (lane & 1);
+                const int R = 16 * (2 * p + 1), Cc = 32 * p;
+                float t[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) t[u] = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < 16; ++s2) {
+                    const float l = sLI[(R + r) * kLP + Cc + s2];
+                    const float4 d0 = *reinterpret_cast<const float4*>(sLI + (Cc + s2) * kLP + Cc + c8);
+                    const float4 d1 = *reinterpret_cast<const float4*>(sLI + (Cc + s2) * kLP + Cc + c8 + 4);
+                    t[0] += l * d0.x; t[1] += l * d0.y; t[2] += l * d0.z; t[3] += l * d0.w;
+                    t[4] += l * d1.x; t[5] += l * d1.y; t[6] += l * d1.z; t[7] += l * d1.w;
+                }
+                *reinterpret_cast<float4*>(sT + (16 * p + r) * kTP + c8) = make_float4(t[0], t[1], t[2], t[3]);
+                *reinterpret_cast<float4*>(sT + (16 * p + r) * kTP + c8 + 4) = make_float4(t[4], t[5], t[6], t[7]);
+                __syncwarp();
+#pragma unroll
+                for (int u = 0; u < 8; ++u) t[u] = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < 16; ++s2) {   // D_hi is lower triangular: its zeros add nothing
+                    const float dh = sLI[(R + r) * kLP + R + s2];
+                    const float4 t0 = *reinterpret_cast<const float4*>(sT + (16 * p + s2) * kTP + c8);
+                    const float4 t1 = *reinterpret_cast<const float4*>(sT + (16 * p + s2) * kTP + c8 + 4);
+                    t[0] -= dh * t0.x; t[1] -= dh * t0.y; t[2] -= dh * t0.z; t[3] -= dh * t0.w;
+                    t[4] -= dh * t1.x; t[5] -= dh * t1.y; t[6] -= dh * t1.z; t[7] -= dh * t1.w;
+                }
+                *reinterpret_cast<float4*>(sLI + (R + r) * kLP + Cc + c8) = make_float4(t[0], t[1], t[2], t[3]);
+                *reinterpret_cast<float4*>(sLI + (R + r) * kLP + Cc + c8 + 4) = make_float4(t[4], t[5], t[6], t[7]);
+            }
         }
         // K_res = K_inv gamma, in place (the first MMA has finished reading K_inv); warps 1
         // and 4 also take the rows of warps 0 and 5
@@ -507,35 +550,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // the inverse is lower triangular), so the block products below need no masks.
     {
         float* sT = sX;
-        // 16 -> 32, block pairs (0,1) and (2,3): X = -D_hi (L_lo D_lo); 1x4 tiles per thread
-        if (tid < 128) {
-            const int p = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
-            const int R = 16 * (2 * p + 1), Cc = 32 * p;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int s2 = 0; s2 < 16; ++s2) {
-                const float l = sLI[(R + r) * kLP + Cc + s2];
-                const float4 dv = *reinterpret_cast<const float4*>(sLI + (Cc + s2) * kLP + Cc + c4);
-                acc.x += l * dv.x; acc.y += l * dv.y; acc.z += l * dv.z; acc.w += l * dv.w;
-            }
-            *reinterpret_cast<float4*>(sT + (16 * p + r) * kTP + c4) = acc;
-        }
-        __syncthreads();
-        if (tid < 128) {
-            const int p = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
-            const int R = 16 * (2 * p + 1), Cc = 32 * p;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            const int smax = ((tid >> 2) & 15) | 7;   // last row of this warp's rows (upper zeros)
-#pragma unroll
-            for (int s2 = 0; s2 < 16; ++s2) {
-                if (s2 > smax) break;
-                const float dh = sLI[(R + r) * kLP + R + s2];
-                const float4 tv = *reinterpret_cast<const float4*>(sT + (16 * p + s2) * kTP + c4);
-                acc.x -= dh * tv.x; acc.y -= dh * tv.y; acc.z -= dh * tv.z; acc.w -= dh * tv.w;
-            }
-            *reinterpret_cast<float4*>(sLI + (R + r) * kLP + Cc + c4) = acc;
-        }
-        __syncthreads();
         KDA_TRACE_POINT(ptr_, 8192 + 18);
         // 32 -> 64: X = -B^{-1} (L[32:64, 0:32] A^{-1}); thread (row r, 4 columns)
         {
@@ -1095,7 +1109,7 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
         dim3 grid((unsigned)max_chunks(total, num_seqs), (unsigned)H);
         prep<<<grid, kPrepThreads, PrepSmem::BYTES, stream>>>(tq, tk, tv, tg, g_scalar ? g : nullptr,
                                                               beta, num_seqs, H, w.off, w.tab, w.records,
-                                                              in_flags);
+                                                              in_flags, total);
     }
     return cudaGetLastError();
 }
