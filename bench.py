@@ -369,7 +369,7 @@ def bench_decode(args, dev, stream, rank, world, peaks):
         "seq_tokens_per_s": round(world * Nd * dcfg.steps / (ms * 1e-3), 1),
         "roofline": {"bound": "hbm", "achieved": round(gbs_local, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(gbs_local / peaks["hbm_gbs"], 4),
-                     "traffic": None, "kernel": "kda::decode_kernel",
+                     "traffic": recorded_traffic("decode_kernel"), "kernel": "kda::decode_kernel",
                      "bytes_per_launch": 8 * Dd * Dd * Nd * Hd,
                      "counts": "pages' 8 D^2 bytes per head-token", "peak_source": peaks["source"]},
         "clocks": clocks, "gpu_launches": dcfg.steps * args.steps,

@@ -26,11 +26,12 @@
 //                         -M = K_res^T W                                             (MMA 128x128x64)
 //                         Aqk W -> P = Q_dec - Aqk W                                 (MMA 128x128x64)
 //                       and writes one record per (chunk, head): the shared-memory
-//                       operand images of P, M, K_res, U (2 value slices), Aqk, and gamma.
-//   rec_kernel          one CTA per (sequence, head, 64 value channels): the chunk chain
-//                       with the fp32 state slice in registers and, beside it, the chunk
-//                       outputs O = P S_in + R; two loader warps stream the records in (bulk
-//                       copies into rings of 3 and 2 stages) and an issuer warp launches the
+//                       operand images of P, M, K_res, U (4 value slices), Aqk, and gamma.
+//   emit_index_kernel   (kda_prefill_emit only) chunk boundaries at which to emit states.
+//   rec_kernel<NV>      one CTA per (sequence, head, NV = 32 or 64 value channels): the
+//                       chunk chain with the fp32 state slice in registers and, beside it,
+//                       the chunk outputs O = P S_in + Aqk U; a loader warp streams the
+//                       records in (bulk copies, 2 stages) and two issuer warps launch the
 //                       tensor-core products, hand-offs through mbarriers only.
 #pragma once
 
