@@ -377,30 +377,59 @@ def bench_decode(args, dev, stream, rank, world, peaks):
 
 
 def bench_e2e(args, P, pre, dev, stream, world):
-    """Same metric through the public API with host buffers: pinned host -> device copies
-    of the step's inputs, the prefill, and device -> host copies of O and the final state,
-    all inside the timed region."""
+    """Same metric through the public API with host buffers: every step copies its inputs
+    from pinned host memory to the device, runs the prefill and copies O and the final
+    state back, all inside the timed region.  Steps are pipelined the way a serving loop
+    would run them: the read-back of step i (on a second stream, from one of two output
+    buffers) overlaps the upload of step i+1 (two input buffers), so the two PCIe
+    directions run at the same time."""
     import torch
-    d, out, fin, inp = P["d"], P["out"], P["fin"], P["inp"]
+    from linear_attention_rule_b200 import kda
+    inp, C = P["inp"], P["C"]
     h = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
-    hout = torch.empty_like(out, device="cpu").pin_memory()
-    hfin = torch.empty_like(fin, device="cpu").pin_memory()
     keys = ("q", "k", "v", "g", "beta", "cu_seqlens") + (("s0",) if inp["s0"] is not None else ())
+    dbuf = [P["d"], {k: (P["d"][k].clone() if P["d"][k] is not None else None) for k in P["d"]}]
+    obuf = [(P["out"], P["fin"]), (torch.empty_like(P["out"]), torch.empty_like(P["fin"]))]
+    hout = [torch.empty_like(P["out"], device="cpu").pin_memory() for _ in range(2)]
+    hfin = [torch.empty_like(P["fin"], device="cpu").pin_memory() for _ in range(2)]
+    back = torch.cuda.Stream(dev)
+    done = [torch.cuda.Event() for _ in range(2)]    # prefill i done (on `stream`)
+    freed = [None, None]                              # read-back of the buffer's last step done
+    counter = [0]
 
     def step():
+        i = counter[0]
+        counter[0] += 1
+        b = i & 1
+        d, (out, fin) = dbuf[b], obuf[b]
         for k in keys:
             d[k].copy_(h[k], non_blocking=True)
-        pre["step"]()
-        hout.copy_(out, non_blocking=True)
-        hfin.copy_(fin, non_blocking=True)
+        if freed[b] is not None:
+            stream.wait_event(freed[b])              # out / fin of step i-2 have been read back
+        kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out,
+                        initial_state=d["s0"], final_state=fin, C=C, workspace=P["ws"], stream=stream)
+        done[b].record(stream)
+        back.wait_event(done[b])
+        with torch.cuda.stream(back):
+            hout[b].copy_(out, non_blocking=True)
+            hfin[b].copy_(fin, non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record(back)
+        freed[b] = ev
 
-    for _ in range(args.warmup):
-        step()
-    _, ms, _ = timed(stream, dev, world, args.steps, step)
+    def run(n):
+        for _ in range(n):
+            step()
+        stream.wait_stream(back)                      # the last read-back inside the region
+
+    run(args.warmup)
+    _, ms, _ = timed(stream, dev, world, 1, lambda: run(args.steps))
+    ms /= args.steps
     h2d = sum(h[k].numel() * h[k].element_size() for k in keys)
-    d2h = hout.numel() * hout.element_size() + hfin.numel() * hfin.element_size()
+    d2h = hout[0].numel() * hout[0].element_size() + hfin[0].numel() * hfin[0].element_size()
     return {"value": round(world * P["T"] / (ms * 1e-3), 1), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4)}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4),
+            "pipelined": "read-back of step i overlaps upload of step i+1"}
 
 
 def bench_gpu(args):
