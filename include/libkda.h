@@ -83,9 +83,12 @@ typedef enum {
  *                 entry do not matter; it is clobbered.  Two calls in flight at once need
  *                 two workspaces.
  * Supported: dk == dv, both 64 or 128.  num_seqs == 0 or total_tokens == 0 are valid.
- * Exponents of the decay are taken relative to each chunk's start, so their range is
- * bounded by one chunk's total decay: |sum of g over a chunk| must stay below ~80 per
- * channel (exp(-a) must be finite in fp32).
+ * Decay range: the decayed operands carry factors exp(a) and exp(-a), a the cumulative
+ * log-decay within a chunk.  With exponents relative to the chunk's start, as on the
+ * tensor-core path (bf16, d 128) by default, |sum of g over a chunk| must stay below ~80
+ * per channel (exp(-a) finite in fp32 and bf16).  The CUDA-core paths, and the tensor-core
+ * path under KDA_IN_STRONG_DECAY (kda_prefill_ex), take exponents relative to half of the
+ * chunk's total decay, which raises the bound to ~170.
  */
 kda_status kda_prefill(const void *q, const void *k, const void *v, const float *g,
                        const float *beta, const float *initial_state,
@@ -104,12 +107,18 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
  *   KDA_IN_G_LOGITS      g holds logits x; the log-decay is logsigmoid(x) = log(sigmoid(x))
  *   KDA_IN_BETA_LOGITS   beta holds logits x; beta = sigmoid(x)
  *   KDA_IN_G_SCALAR      g holds one gate per (token, head) (Gated DeltaNet, below)
+ *   KDA_IN_STRONG_DECAY  not a prologue step: on the tensor-core prefill path, channels whose
+ *                        total log-decay over a chunk is below -64 take exponents relative to
+ *                        half of it (decay range above).  Milder channels give bit-identical
+ *                        results; the preparation kernel runs ~5% slower.  No effect on the
+ *                        CUDA-core paths (always so) or on decode (accepted and ignored).
  */
 enum {
     KDA_IN_NORMALIZE_QK = 1,
     KDA_IN_G_LOGITS = 2,
     KDA_IN_BETA_LOGITS = 4,
-    KDA_IN_G_SCALAR = 8
+    KDA_IN_G_SCALAR = 8,
+    KDA_IN_STRONG_DECAY = 16
 };
 
 /*

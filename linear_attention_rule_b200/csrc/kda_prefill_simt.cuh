@@ -43,7 +43,8 @@ struct SimtSmem {
     static constexpr int BT = GM + DK;         // beta [C]
     static constexpr int NQ = BT + C;          // 1 / ||q_r||, 1 / ||k_r|| [C] (input prologue)
     static constexpr int NK = NQ + C;
-    static constexpr int TOTAL = NK + C;
+    static constexpr int HM = NK + C;          // e^{m}, m = a_last / 2, per key channel [DK]
+    static constexpr int TOTAL = HM + DK;
     static constexpr size_t BYTES = sizeof(float) * TOTAL;
 };
 
@@ -75,6 +76,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
     float* sB = sm + L::BT;
     float* sNq = sm + L::NQ;
     float* sNk = sm + L::NK;
+    float* sH = sm + L::HM;
     const bool g_scalar = (in_flags & kInGScalar) != 0;
 
     const int tid = threadIdx.x;
@@ -133,7 +135,10 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
         }
         __syncthreads();
 
-        // (2) inclusive cumulative sum over the chunk, per key channel; gamma = e^{a_last}
+        // (2) inclusive cumulative sum over the chunk, per key channel; gamma = e^{a_last}.
+        // The decayed operands use exponents relative to m = a_last / 2 (stored as a - m):
+        // the products need only ratios e^{a_r - a_s}, and e^{a - m}, e^{m - a} stay within
+        // e^{|a_last| / 2} where e^{-a} alone would overflow once |a_last| nears 88.
         for (int c = tid; c < DK; c += kSimtThreads) {
             float acc = 0.f;
             for (int r = 0; r < C; ++r) {
@@ -141,6 +146,8 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
                 sWA[r * PK + c] = acc;
             }
             sG[c] = expf(acc);
+            sH[c] = expf(0.5f * acc);
+            for (int r = 0; r < C; ++r) sWA[r * PK + c] -= 0.5f * acc;
         }
         __syncthreads();
 
@@ -206,6 +213,8 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
                     const float4 x = reinterpret_cast<const float4*>(sKd + s * PK)[c4];
                     w.x += co * x.x; w.y += co * x.y; w.z += co * x.z; w.w += co * x.w;
                 }
+                const float4 hm = reinterpret_cast<const float4*>(sH)[c4];   // K_dec = K_dec' e^{m}
+                w.x *= hm.x; w.y *= hm.y; w.z *= hm.z; w.w *= hm.w;
                 reinterpret_cast<float4*>(sWA + r * PK)[c4] = w;
             }
         }
@@ -247,7 +256,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
             for (int r = tid / JG; r < C; r += RG) {
                 float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int c = 0; c < DK; ++c) {
-                    const float a = sQd[r * PK + c];
+                    const float a = sQd[r * PK + c] * sH[c];   // Q_dec = Q_dec' e^{m}
                     const float4 x = reinterpret_cast<const float4*>(sS + c * NV)[j4];
                     o.x += a * x.x; o.y += a * x.y; o.z += a * x.z; o.w += a * x.w;
                 }
@@ -272,14 +281,17 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
 #pragma unroll
             for (int i = 0; i < CPT; ++i) {
                 const int c = tid / JG + i * CGR;
-                float4 acc = reinterpret_cast<const float4*>(sS + c * NV)[j4];
+                // S_out = gamma S_in + (K_inv' e^{a_last - m})^T U' with e^{a_last - m} = e^{m}
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int r = 0; r < C; ++r) {
                     const float kinv = sKi[r * PK + c];
                     const float4 x = reinterpret_cast<const float4*>(sU + r * NV)[j4];
                     acc.x += kinv * x.x; acc.y += kinv * x.y; acc.z += kinv * x.z; acc.w += kinv * x.w;
                 }
-                const float gm = sG[c];
-                acc.x *= gm; acc.y *= gm; acc.z *= gm; acc.w *= gm;
+                const float gm = sG[c], hm = sH[c];
+                const float4 s0v = reinterpret_cast<const float4*>(sS + c * NV)[j4];
+                acc.x = gm * s0v.x + hm * acc.x; acc.y = gm * s0v.y + hm * acc.y;
+                acc.z = gm * s0v.z + hm * acc.z; acc.w = gm * s0v.w + hm * acc.w;
                 snew[i] = acc;
             }
         }

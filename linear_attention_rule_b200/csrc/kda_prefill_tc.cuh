@@ -36,6 +36,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <type_traits>
 
 #include "kda_common.cuh"
 #include "kda_sm100.cuh"
@@ -234,7 +235,8 @@ __device__ __forceinline__ uint32_t stage_slot(int w) {
 // (token, head), g [T, H] (Gated DeltaNet, the scalar forget gate that KDA makes diagonal):
 // the same decay on every channel, loaded like beta instead of through the g tensor map.
 // kPrologue: in_flags may hold KDA_IN_* prologue bits (the plain path compiles without them).
-template <bool kScalarG, bool kPrologue>
+// kStrong: channels whose chunk total decay passes -64 take exponents relative to half of it.
+template <bool kScalarG, bool kPrologue, bool kStrong>
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -268,6 +270,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wh = warp >> 2;   // TMEM lane quarter, column half
     bool ok = true;
+    uint32_t shifted = 0;   // kStrong: this thread's channels whose exponents are relative to a_last / 2
     uint32_t phase = 0;
 
     // ---- (0) TMA: rows t0..t0+63 of q, k, v (two 64-channel boxes each) and g; the
@@ -374,6 +377,25 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             float4* gdst = reinterpret_cast<float4*>(rec + kRecGamma + 32 * cg);
             gdst[0] = make_float4(gam[0], gam[1], gam[2], gam[3]);
             gdst[1] = make_float4(gam[4], gam[5], gam[6], gam[7]);
+        }
+        // Strong decay (kStrong): in a channel whose total |a_last| passes 64 (e^{-a} overflows
+        // fp32 and bf16 near 88), the exponents are taken relative to half the chunk's total
+        // decay, m = a_last / 2.  L and Aqk only need the ratios e^{a_r - a_s}, and e^{a - m},
+        // e^{m - a} stay within e^{|a_last| / 2}.  Then gam = e^{m} for that channel, and after
+        // the first product K_dec and Q_dec are scaled back by it in place, and
+        // K_res = K_inv' e^{a_last - m} = K_inv' e^{m}.  Every thread holding a channel sees
+        // the same total, so the choice is the same for all its rows without a barrier.
+        // Milder channels keep a = 0 at the chunk start, K_res = K_inv gamma, bit for bit as
+        // without kStrong.
+        if constexpr (kStrong) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (tot[u] < -64.f) {
+                    shifted |= 1u << u;
+                    base[u] -= 0.5f * tot[u];
+                    gam[u] = __expf(0.5f * tot[u]);
+                }
+            }
         }
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
@@ -517,17 +539,32 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 *reinterpret_cast<float4*>(sLI + (R + r) * kLP + Cc + c8 + 4) = make_float4(t[4], t[5], t[6], t[7]);
             }
         }
-        // K_res = K_inv gamma, in place (the first MMA has finished reading K_inv); warps 1
-        // and 4 also take the rows of warps 0 and 5
+        // K_res = K_inv gamma (kStrong: K_inv' e^{m} in the shifted channels, whose K_dec and
+        // Q_dec are also scaled by e^{m}), in place: the first MMA has finished reading them;
+        // warps 1 and 4 also take the rows of warps 0 and 5
         auto kres_rows = [&](int wsrc) {
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr) {
-                const uint32_t o = S::KI0 + kb * S::BLK + sw128_off(4 * (2 * wsrc + half) + rr, c8);
-                float ki[8];
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + o), ki);
+                const uint32_t o = kb * S::BLK + sw128_off(4 * (2 * wsrc + half) + rr, c8);
+                if constexpr (kStrong) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) ki[u] *= gam[u];
-                *reinterpret_cast<uint4*>(sm + o) = pack_bf16x8(ki);
+                    for (int img = 0; img < 3; ++img) {
+                        if (img > 0 && !shifted) break;
+                        uint8_t* pimg = sm + (img == 0 ? S::KI0 : img == 1 ? S::KD0 : S::QD0) + o;
+                        float x[8];
+                        unpack_bf16x8(*reinterpret_cast<const uint4*>(pimg), x);
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            x[u] *= (img == 0 || ((shifted >> u) & 1u)) ? gam[u] : 1.f;
+                        *reinterpret_cast<uint4*>(pimg) = pack_bf16x8(x);
+                    }
+                } else {
+                    float ki[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::KI0 + o), ki);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) ki[u] *= gam[u];
+                    *reinterpret_cast<uint4*>(sm + S::KI0 + o) = pack_bf16x8(ki);
+                }
             }
         };
         if (warp != 0 && warp != 5) kres_rows(warp);
@@ -1087,9 +1124,14 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
                                   uint32_t in_flags = 0) {
     const bool g_scalar = (in_flags & kInGScalar) != 0;
     const Workspace w = split_workspace(workspace, total, num_seqs);
-    const bool pro = (in_flags & ~kInGScalar) != 0;
-    auto prep = g_scalar ? (pro ? prep_kernel<true, true> : prep_kernel<true, false>)
-                         : (pro ? prep_kernel<false, true> : prep_kernel<false, false>);
+    const bool pro = (in_flags & ~(kInGScalar | kInStrongDecay)) != 0;
+    const bool strong = (in_flags & kInStrongDecay) != 0;
+    auto pick = [&](auto sc) {
+        constexpr bool kSc = decltype(sc)::value;
+        return strong ? (pro ? prep_kernel<kSc, true, true> : prep_kernel<kSc, false, true>)
+                      : (pro ? prep_kernel<kSc, true, false> : prep_kernel<kSc, false, false>);
+    };
+    auto prep = g_scalar ? pick(std::true_type{}) : pick(std::false_type{});
     cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepSmem::BYTES);
     if (e != cudaSuccess) return e;

@@ -78,7 +78,8 @@ static kda_status prefill_common(const void* q, const void* k, const void* v, co
                                  size_t ws_bytes, kda_stream_t stream, uint32_t in_flags) {
     if (num_seqs < 0 || total_tokens < 0 || H <= 0 || dk <= 0 || dv <= 0 || num_emit < 0)
         return KDA_ERR_INVALID_ARG;
-    if (in_flags & ~(uint32_t)(KDA_IN_NORMALIZE_QK | KDA_IN_G_LOGITS | KDA_IN_BETA_LOGITS | KDA_IN_G_SCALAR))
+    if (in_flags & ~(uint32_t)(KDA_IN_NORMALIZE_QK | KDA_IN_G_LOGITS | KDA_IN_BETA_LOGITS |
+                               KDA_IN_G_SCALAR | KDA_IN_STRONG_DECAY))
         return KDA_ERR_INVALID_ARG;
     if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (total_tokens > INT32_MAX) return KDA_ERR_UNSUPPORTED;  // cu_seqlens is int32
@@ -216,8 +217,10 @@ static kda_status decode_common(const void* q, const void* k, const void* v, con
                                 const float* beta, float* state_inout, void* out, int32_t N, int32_t H,
                                 int32_t dk, int32_t dv, kda_dtype dt, kda_stream_t stream, uint32_t in_flags) {
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
-    if (in_flags & ~(uint32_t)(KDA_IN_NORMALIZE_QK | KDA_IN_G_LOGITS | KDA_IN_BETA_LOGITS | KDA_IN_G_SCALAR))
+    if (in_flags & ~(uint32_t)(KDA_IN_NORMALIZE_QK | KDA_IN_G_LOGITS | KDA_IN_BETA_LOGITS |
+                               KDA_IN_G_SCALAR | KDA_IN_STRONG_DECAY))
         return KDA_ERR_INVALID_ARG;
+    in_flags &= ~(uint32_t)KDA_IN_STRONG_DECAY;   // one token's decay is applied directly
     if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (!supported_dim(dk, dv)) return KDA_ERR_UNSUPPORTED;
     if (N == 0) return KDA_OK;

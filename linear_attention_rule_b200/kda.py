@@ -28,6 +28,7 @@ KDA_IN_NORMALIZE_QK = 1
 KDA_IN_G_LOGITS = 2
 KDA_IN_BETA_LOGITS = 4
 KDA_IN_G_SCALAR = 8
+KDA_IN_STRONG_DECAY = 16
 KDA_F32 = 0
 KDA_BF16 = 1
 

@@ -16,8 +16,9 @@ def to_device(d: dict) -> dict:
     return {k: (None if v is None else v.cuda()) for k, v in d.items()}
 
 
-def run_prefill(inp: dict, C: int = 64, initial=True, want_final=True, workspace=None):
-    """Run kda_prefill on CPU-drawn inputs; returns (out fp64 numpy, final fp64 numpy|None)."""
+def run_prefill(inp: dict, C: int = 64, initial=True, want_final=True, workspace=None, in_flags=0):
+    """Run kda_prefill (kda_prefill_ex when in_flags is given) on CPU-drawn inputs; returns
+    (out fp64 numpy, final fp64 numpy|None)."""
     d = to_device(inp)
     T, H, _ = d["q"].shape
     dv = d["v"].shape[2]
@@ -25,9 +26,13 @@ def run_prefill(inp: dict, C: int = 64, initial=True, want_final=True, workspace
     dk = d["q"].shape[2]
     out = torch.full((T, H, dv), float("nan"), dtype=d["q"].dtype, device="cuda")
     sf = torch.full((N, H, dk, dv), float("nan"), device="cuda") if want_final else None
-    kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out,
-                    initial_state=d["s0"] if initial else None, final_state=sf, C=C,
-                    workspace=workspace)
+    s0 = d["s0"] if initial else None
+    if in_flags:
+        kda.kda_prefill_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out, in_flags,
+                           initial_state=s0, final_state=sf, C=C, workspace=workspace)
+    else:
+        kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out,
+                        initial_state=s0, final_state=sf, C=C, workspace=workspace)
     status = kda.kda_get_device_status()
     assert status == kda.KDA_OK, kda.kda_status_string(status)
     o = out.double().cpu().numpy()

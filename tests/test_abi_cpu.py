@@ -162,13 +162,13 @@ def test_prologue_entry_points_reject_unknown_flags(lib):
     ex = lambda flags: lib.kda_prefill_ex(P(4096), P(4096), P(4096), P(4096), P(4096), None, P(4096), 1, 256,
                                           2, 128, 128, kda.KDA_BF16, P(4096), None, 64, flags, None, 0, None,
                                           P(1 << 20), need, None)
-    assert ex(16) == kda.KDA_ERR_INVALID_ARG
+    assert ex(32) == kda.KDA_ERR_INVALID_ARG
     assert ex(1 << 31) == kda.KDA_ERR_INVALID_ARG
     dec = lambda flags: lib.kda_decode_ex(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), 2,
                                           2, 128, 128, kda.KDA_BF16, flags, None)
     assert dec(32) == kda.KDA_ERR_INVALID_ARG
     assert lib.kda_decode_ex(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), 0, 2, 128, 128,
-                             kda.KDA_BF16, 15, None) == kda.KDA_OK
+                             kda.KDA_BF16, 31, None) == kda.KDA_OK   # every known bit, N = 0
 
 
 def test_selftest_rejects_out_of_range_limits(lib):

@@ -47,6 +47,31 @@ def test_bf16_many_sequence_heads():
     check_prefill(inp, out, fin, heads=[0, 7, 31])
 
 
+@pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.bfloat16, 64), (torch.float32, 64),
+                                     (torch.float32, 128)])
+def test_strong_decay_beyond_fp32_exponent_range(dtype, D):
+    """Gates logsigmoid(N(-1.5, 1)): a full chunk's total log-decay is about -115 per channel,
+    so e^{-a} alone would overflow fp32 (and bf16); exponents relative to half the chunk's
+    decay (KDA_IN_STRONG_DECAY on the tensor-core path, always on the CUDA-core paths) keep
+    every factor within e^{|a_last| / 2}."""
+    inp = _inputs([200, 64, 70], 2, D, dtype, seed=17, g_mean=-1.5)
+    assert float(inp["g"][:64].sum(0).min()) < -100      # the premise: far beyond e^{88}
+    out, fin = run_prefill(inp, C=64, in_flags=kda.KDA_IN_STRONG_DECAY)
+    check_prefill(inp, out, fin)
+
+
+@pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_strong_decay_flag_is_bit_identical_on_mild_decay(dtype, D):
+    """Channels whose chunk total stays above -64 keep the chunk-start reference: the flag
+    changes nothing there, bit for bit (and the CUDA-core paths ignore it)."""
+    inp = _inputs([300, 64, 1, 129], 3, D, dtype, seed=19, g_mean=3.0)
+    assert float(inp["g"][:64].sum(0).min()) > -64
+    o0, f0 = run_prefill(inp, C=64)
+    o1, f1 = run_prefill(inp, C=64, in_flags=kda.KDA_IN_STRONG_DECAY)
+    np.testing.assert_array_equal(o0, o1)
+    np.testing.assert_array_equal(f0, f1)
+
+
 def test_bf16_d64():
     inp = _inputs([130, 64, 7], 2, 64, torch.bfloat16, seed=12)
     out, fin = run_prefill(inp, C=64)
