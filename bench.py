@@ -95,12 +95,21 @@ def prefill_stage_page_bytes(lengths, H, D, C):
     return prep, rest
 
 
-def source_digest():
-    """Short hash of the CUDA sources, to tell whether recorded ncu counters still apply."""
+# CUDA sources each kernel's recorded counters depend on (its own file and the helpers it uses)
+KERNEL_SOURCES = {
+    "prep_kernel": ("kda_common.cuh", "kda_sm100.cuh", "kda_prefill_tc.cuh"),
+    "rec_kernel": ("kda_common.cuh", "kda_sm100.cuh", "kda_prefill_tc.cuh"),
+    "decode_kernel": ("kda_common.cuh", "kda_decode.cuh"),
+}
+
+
+def source_digest(files=None):
+    """Short hash of the CUDA sources (all of csrc, or the named files), to tell whether
+    recorded ncu counters still apply."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_rule_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -109,14 +118,14 @@ def source_digest():
 def recorded_traffic(kernel: str):
     """DRAM bytes per launch of `kernel` recorded from an ncu capture in profiles/
     ('<kernel> traffic_bytes_per_launch <N> sources <digest>'), or None when absent or
-    taken on different sources."""
+    taken on different sources of that kernel (KERNEL_SOURCES)."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         with open(path) as fh:
             for line in fh:
                 f = line.split()
                 if len(f) >= 5 and f[0] == kernel and f[1] == "traffic_bytes_per_launch":
-                    return int(f[2]) if f[4] == source_digest() else None
+                    return int(f[2]) if f[4] == source_digest(KERNEL_SOURCES.get(kernel)) else None
     except OSError:
         pass
     return None
@@ -502,8 +511,10 @@ def bench_reference(args):
                                         cfg.s0_std, cfg.seed)
     H = cfg.H
     threads = min(oracle.default_threads(), H)
-    # size one step for about args.cpu_seconds / 2 of fp64 work
-    _, ts, _, _ = oracle_sample_tokens_per_s(inp, max(1.0, args.cpu_seconds / 2))
+    # size one step for about args.cpu_seconds / 2 of fp64 work, less when many steps are
+    # asked for, so that warm-up and timed steps together take about 90 s at most
+    per_step = max(0.05, min(args.cpu_seconds / 2, 90.0 / (args.steps + args.warmup)))
+    _, ts, _, _ = oracle_sample_tokens_per_s(inp, per_step)
 
     def step():
         oracle.prefill(inp["q"][:ts], inp["k"][:ts], inp["v"][:ts], inp["g"][:ts],
@@ -535,7 +546,7 @@ def bench_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--no-e2e", action="store_true")

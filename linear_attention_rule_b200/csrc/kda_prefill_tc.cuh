@@ -196,6 +196,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tma
 
 // ------------------------------------------------------------------ chunk preparation
 constexpr int kPrepThreads = 256;
+constexpr int kPrepCtasPerSm = 2;
 struct PrepSmem {
     // operand region: 128-byte-swizzled tiles of 64 rows (tokens) x 64 channels
     static constexpr uint32_t KD0 = 0, QD0 = 8192, KD1 = 16384, QD1 = 24576;
@@ -206,15 +207,17 @@ struct PrepSmem {
     static constexpr uint32_t ABAR = GR, AQK = GR + 8192, LI = GR + 16384;   // LI: [64][68]
     static constexpr uint32_t XCH = GR + 33792;      // decay partials [8][128]; later T [32][36]
     static constexpr uint32_t BETA = XCH + 4608;     // [64]
-    static constexpr uint32_t BAR = BETA + 256;       // TMA and products in order
+    static constexpr uint32_t BAR = BETA + 256;       // g's TMA, then the products in order
     static constexpr uint32_t BAR2 = BAR + 8;         // the last product (Aqk W)
-    static constexpr uint32_t TMEM = BAR2 + 8;
+    static constexpr uint32_t BARQK = BAR2 + 8;       // TMA of q and k
+    static constexpr uint32_t BARV = BARQK + 8;       // TMA of v
+    static constexpr uint32_t TMEM = BARV + 8;
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;  // + alignment slack
 };
 constexpr int kLP = 68;                                   // row pitch of L / INV (16-byte rows)
 constexpr int kTP = 36;                                   // row pitch of the product scratch
 constexpr uint32_t kPrepTmemCols = 256;
-constexpr uint32_t kPrepTx = 3 * 16384 + 32768;           // q, k, v (2 boxes of 8 KB each) + g
+constexpr uint32_t kPrepTxG = 32768, kPrepTxQK = 2 * 16384, kPrepTxV = 16384;   // bytes per barrier
 
 __device__ __forceinline__ bool prep_sync_ok(bool ok, int tid) {
     if (__syncthreads_or(!ok)) {
@@ -237,7 +240,7 @@ __device__ __forceinline__ uint32_t stage_slot(int w) {
 // kPrologue: in_flags may hold KDA_IN_* prologue bits (the plain path compiles without them).
 // kStrong: channels whose chunk total decay passes -64 take exponents relative to half of it.
 template <bool kScalarG, bool kPrologue, bool kStrong>
-__global__ void __launch_bounds__(kPrepThreads, 2)
+__global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
             const float* __restrict__ g_scalar, const float* __restrict__ beta, int num_seqs, int H,
@@ -269,25 +272,34 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     float* sLI = reinterpret_cast<float*>(sm + S::LI);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wh = warp >> 2;   // TMEM lane quarter, column half
-    bool ok = true;
+    bool ok = true, v_ok = true;
     uint32_t shifted = 0;   // kStrong: this thread's channels whose exponents are relative to a_last / 2
     uint32_t phase = 0;
 
-    // ---- (0) TMA: rows t0..t0+63 of q, k, v (two 64-channel boxes each) and g; the
-    // barrier is initialised and the copies issued by the same thread, before anything else
+    // ---- (0) TMA: rows t0..t0+63 of g, then q and k, then v (two 64-channel boxes each),
+    // on three barriers in the order of use: the decay's prefix sums start once g is in, the
+    // decayed operands once q and k are, and v is first read by the product of step (4).  The
+    // barriers are initialised and the copies issued by the same thread, before anything else.
+    const uint32_t barqk = sb + S::BARQK, barv = sb + S::BARV;
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(bar + 8, 1);
+        mbar_init(barqk, 1);
+        mbar_init(barv, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar, kScalarG ? kPrepTx - 32768 : kPrepTx);
         const int x0 = h * D;
-        tma_load_2d(sb + S::QD0, &tm_q, x0, t0, bar);
-        tma_load_2d(sb + S::QD1, &tm_q, x0 + 64, t0, bar);
-        tma_load_2d(sb + S::KD0, &tm_k, x0, t0, bar);
-        tma_load_2d(sb + S::KD1, &tm_k, x0 + 64, t0, bar);
-        tma_load_2d(sb + S::V0, &tm_v, x0, t0, bar);
-        tma_load_2d(sb + S::V1, &tm_v, x0 + 64, t0, bar);
-        if (!kScalarG) tma_load_2d(sb + S::GR, &tm_g, x0, t0, bar);
+        if (!kScalarG) {
+            mbar_arrive_expect_tx(bar, kPrepTxG);
+            tma_load_2d(sb + S::GR, &tm_g, x0, t0, bar);
+        }
+        mbar_arrive_expect_tx(barqk, kPrepTxQK);
+        tma_load_2d(sb + S::QD0, &tm_q, x0, t0, barqk);
+        tma_load_2d(sb + S::QD1, &tm_q, x0 + 64, t0, barqk);
+        tma_load_2d(sb + S::KD0, &tm_k, x0, t0, barqk);
+        tma_load_2d(sb + S::KD1, &tm_k, x0 + 64, t0, barqk);
+        mbar_arrive_expect_tx(barv, kPrepTxV);
+        tma_load_2d(sb + S::V0, &tm_v, x0, t0, barv);
+        tma_load_2d(sb + S::V1, &tm_v, x0 + 64, t0, barv);
     }
     if (warp == 1) tmem_alloc(sb + S::TMEM, kPrepTmemCols);
     if (tid < C) {
@@ -307,10 +319,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const bool ptr_ = blockIdx.x == 37 && blockIdx.y == 3 && tid == 0;
     (void)ptr_;
     KDA_TRACE_POINT(ptr_, 8192 + 0);
-    ok = mbar_wait(bar, phase);
-    phase ^= 1;
+    if constexpr (!kScalarG) {   // a scalar gate came with plain loads, before the barrier above
+        ok = mbar_wait(bar, phase);
+        phase ^= 1;
+        if (!prep_sync_ok(ok, tid)) goto done;
+    }
     KDA_TRACE_POINT(ptr_, 8192 + 1);
-    if (!prep_sync_ok(ok, tid)) goto done;
 
     {
         // ---- (1) decay: thread = (block of 4 tokens rb, group of 8 channels cg) ----
@@ -397,6 +411,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
         }
+        ok = mbar_wait(barqk, 0);   // q, k in (a failure is acted on at the barrier below)
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
             const int r = 4 * rb + rr;
@@ -433,7 +448,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             *reinterpret_cast<uint4*>(sm + S::KI0 + o) = pack_bf16x8(ki);
         }
         fence_proxy_async_smem();
-        __syncthreads();
+        if (!prep_sync_ok(ok, tid)) goto done;
         KDA_TRACE_POINT(ptr_, 8192 + 2);
 
         // ---- (2) [K_dec ; Q_dec] K_inv^T -> TMEM [0, 64) ----
@@ -631,7 +646,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     KDA_TRACE_POINT(ptr_, 8192 + 4);
 
     // ---- (4) [W | U] = Abar [K_dec | V] -> TMEM [0, 256) (lanes 0-63 meaningful) ----
+    // Only the issuing thread waits for v; a failure is carried into the check after the
+    // product (which then read whatever v's buffer held: nothing is kept).
     if (tid == 0) {
+        v_ok = mbar_wait(barv, 0);
         tc_fence_after();
         constexpr uint32_t id = idesc_bf16(128, 256, false, true);
 #pragma unroll
@@ -640,7 +658,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                       smem_desc(sb + S::KD0 + ks * 2048, S::BLK, 1024, kSwizzle128), id, ks > 0);
         umma_commit(bar);
     }
-    ok = mbar_wait(bar, phase);
+    ok = mbar_wait(bar, phase) && v_ok;
     phase ^= 1;
     tc_fence_after();
     if (!prep_sync_ok(ok, tid)) goto done;
@@ -749,8 +767,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
 done:
     // no copy may still read shared memory at exit; their global writes may still be in
-    // flight (they complete before the grid does)
+    // flight (they complete before the grid does).  After a failed wait the input copies may
+    // still be landing: give them their bounded waits (immediate once complete).
     if (lane == 0) bulk_wait_read<0>();
+    if (tid == 0) {
+        (void)mbar_wait(barqk, 0);
+        (void)mbar_wait(barv, 0);
+    }
     tc_fence_before();
     __syncthreads();
     KDA_TRACE_POINT(ptr_, 8192 + 7);
@@ -1116,6 +1139,17 @@ inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs) {
             base + ws_records_offset(total, num_seqs)};
 }
 
+// SMs of the current device (cached per device; 0 when the query fails).
+inline int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cached[dev] == 0 &&
+        cudaDeviceGetAttribute(&cached[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cached[dev] = 0;
+    return cached[dev];
+}
+
 // Chunk table (+ emission slots when emit_pos is given) + chunk-parallel preparation.
 inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, const int32_t* cu, int num_seqs,
@@ -1155,17 +1189,6 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
                                                               in_flags, total);
     }
     return cudaGetLastError();
-}
-
-// SMs of the current device (cached per device; 0 when the query fails).
-inline int device_sm_count() {
-    static int cached[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (cached[dev] == 0 &&
-        cudaDeviceGetAttribute(&cached[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        cached[dev] = 0;
-    return cached[dev];
 }
 
 template <int NV>
