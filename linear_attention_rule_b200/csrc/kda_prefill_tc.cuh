@@ -16,7 +16,8 @@
 //   chunk_index_kernel  cu_seqlens -> first chunk of every sequence and the chunk table
 //                       (first token, rows) (device side, no host sync); validates cu_seqlens.
 //   prep_kernel         one CTA of 8 warps per (chunk, head), fully parallel, 2 CTAs per SM:
-//                         TMA: q, k, v tiles (128-byte swizzled) and g into shared memory
+//                         TMA: g, then q and k, then v tiles (128-byte swizzled) into
+//                              shared memory, each group on its own barrier
 //                         a, gamma, Q_dec = q e^a, K_dec = k e^a, K_inv = k e^-a      (FFMA/MUFU)
 //                         [K_dec; Q_dec] K_inv^T                                      (MMA 128x64x128)
 //                         L = strict_tril(beta K_dec K_inv^T), Aqk = tril(Q_dec K_inv^T)
