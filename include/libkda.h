@@ -56,7 +56,8 @@ typedef enum {
 
 typedef enum {
     KDA_F32 = 0,   /* q, k, v, out in fp32: the CUDA-core (FFMA) chunked path */
-    KDA_BF16 = 1   /* q, k, v, out in bf16: the tensor-core (tcgen05) chunked path */
+    KDA_BF16 = 1   /* q, k, v, out in bf16: the tensor-core (tcgen05) chunked path at
+                      dk = dv = 128, the CUDA-core path at 64 */
 } kda_dtype;
 
 /*
