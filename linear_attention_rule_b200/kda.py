@@ -116,6 +116,68 @@ def _ptr(t: Optional[torch.Tensor]):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _check(device, **args):
+    """Validate the tensors of one call before any pointer reaches the library: each value
+    is (tensor or None, expected shape, expected dtype).  Shapes and dtypes are checked
+    first, then that every tensor is contiguous and on `device` (the device of q or out),
+    so a mistake raises here instead of becoming an out-of-bounds access on the GPU."""
+    for name, (t, shape, dtype) in args.items():
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise TypeError("%s must be a torch.Tensor" % name)
+        if t.dtype != dtype:
+            raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    for name, (t, _, _) in args.items():
+        if t is None:
+            continue
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous" % name)
+        if t.device.type != "cuda" or t.device != device:
+            raise ValueError("%s must be on %s (libkda takes device pointers), got %s"
+                             % (name, device, t.device))
+
+
+def _check_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state, final_state, scalar_g=False,
+                   workspace=None, emit_pos=None, emit_states=None):
+    """Shapes of a prefill call: q, k [T, H, dk], v, out [T, H, dv] in q's dtype; g [T, H, dk]
+    (or [T, H] for a scalar gate) and beta [T, H] fp32; cu_seqlens int32 [N+1]; states fp32
+    [N, H, dk, dv]; workspace uint8 (its size is checked by the library); emission positions
+    int64 [E] with their states fp32 [E, H, dk, dv]."""
+    if q.dim() != 3 or v.dim() != 3 or cu_seqlens.dim() != 1:
+        raise ValueError("q and v must be [T, H, d] and cu_seqlens [N+1]")
+    if (emit_pos is None) != (emit_states is None):
+        raise ValueError("emit_pos and emit_states go together")
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    E = emit_pos.shape[0] if emit_pos is not None and emit_pos.dim() == 1 else -1
+    dt = q.dtype
+    _check(q.device, q=(q, (T, H, dk), dt), k=(k, (T, H, dk), dt), v=(v, (T, H, dv), dt),
+           out=(out, (T, H, dv), dt), g=(g, (T, H) if scalar_g else (T, H, dk), torch.float32),
+           beta=(beta, (T, H), torch.float32), cu_seqlens=(cu_seqlens, (N + 1,), torch.int32),
+           initial_state=(initial_state, (N, H, dk, dv), torch.float32),
+           final_state=(final_state, (N, H, dk, dv), torch.float32),
+           workspace=(workspace, (workspace.numel(),) if workspace is not None else (), torch.uint8),
+           emit_pos=(emit_pos, (E,), torch.int64),
+           emit_states=(emit_states, (E, H, dk, dv), torch.float32))
+
+
+def _check_decode(q, k, v, g, beta, state, out, scalar_g=False):
+    """Shapes of a decode call: q, k [N, H, dk], v, out [N, H, dv] in q's dtype; g [N, H, dk]
+    (or [N, H]) and beta [N, H] fp32; state fp32 [N, H, dk, dv]."""
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q and v must be [N, H, d]")
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    dt = q.dtype
+    _check(q.device, q=(q, (N, H, dk), dt), k=(k, (N, H, dk), dt), v=(v, (N, H, dv), dt),
+           out=(out, (N, H, dv), dt), g=(g, (N, H) if scalar_g else (N, H, dk), torch.float32),
+           beta=(beta, (N, H), torch.float32), state=(state, (N, H, dk, dv), torch.float32))
+
+
 def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -158,12 +220,12 @@ def kda_prefill_gdn(q, k, v, g, beta, cu_seqlens, out, initial_state=None, final
 
 def _prefill(fn, q, k, v, g, beta, cu_seqlens, out, initial_state, final_state, C, workspace, stream):
     lib = load()
+    dt = _dtype_code(q)
+    _check_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state, final_state,
+                   scalar_g=fn == "kda_prefill_gdn", workspace=workspace)
     T, H, dk = q.shape
     dv = v.shape[2]
     N = cu_seqlens.shape[0] - 1
-    dt = _dtype_code(q)
-    if cu_seqlens.dtype != torch.int32:
-        raise TypeError("cu_seqlens must be int32")
     need = int(lib.kda_prefill_workspace_size(T, N, H, dk, dv, C, dt))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -183,12 +245,12 @@ def kda_prefill_emit(q, k, v, g, beta, cu_seqlens, out, emit_pos, emit_states,
     device) into emit_states (fp32 [E, H, dk, dv]); see kda_prefill_emit in
     include/libkda.h."""
     lib = load()
+    dt = _dtype_code(q)
+    _check_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state, final_state, workspace=workspace,
+                   emit_pos=emit_pos, emit_states=emit_states)
     T, H, dk = q.shape
     dv = v.shape[2]
     N = cu_seqlens.shape[0] - 1
-    dt = _dtype_code(q)
-    if cu_seqlens.dtype != torch.int32 or emit_pos.dtype != torch.int64:
-        raise TypeError("cu_seqlens must be int32 and emit_pos int64")
     need = int(lib.kda_prefill_workspace_size(T, N, H, dk, dv, C, dt))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -208,10 +270,13 @@ def kda_prefill_ex(q, k, v, g, beta, cu_seqlens, out, in_flags: int = 0, initial
     """kda_prefill with an input prologue (KDA_IN_* flags) and optional state emission
     (kda_prefill_ex in include/libkda.h).  With KDA_IN_G_SCALAR, g is [T, H]."""
     lib = load()
+    dt = _dtype_code(q)
+    _check_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state, final_state,
+                   scalar_g=bool(int(in_flags) & KDA_IN_G_SCALAR), workspace=workspace,
+                   emit_pos=emit_pos, emit_states=emit_states)
     T, H, dk = q.shape
     dv = v.shape[2]
     N = cu_seqlens.shape[0] - 1
-    dt = _dtype_code(q)
     need = int(lib.kda_prefill_workspace_size(T, N, H, dk, dv, C, dt))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -234,11 +299,11 @@ def kda_prefill_noalloc(q, k, v, g, beta, cu_seqlens, out, initial_state=None,
     d = 128 and C = 64 only; problems needing more than NOALLOC_SCRATCH_BYTES of scratch
     are rejected.  Calls sharing a device must not overlap on the GPU."""
     lib = load()
+    _dtype_code(q)
+    _check_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state, final_state)
     T, H, dk = q.shape
     dv = v.shape[2]
     N = cu_seqlens.shape[0] - 1
-    if cu_seqlens.dtype != torch.int32:
-        raise TypeError("cu_seqlens must be int32")
     st = lib.kda_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                  _ptr(initial_state), _ptr(cu_seqlens), N, T, H, dk, dv,
                                  _dtype_code(q), _ptr(out), _ptr(final_state), C, _stream(stream))
@@ -254,6 +319,10 @@ def _ws(workspace):
 def kda_prefill_prepare(q, k, v, g, beta, cu_seqlens, workspace, C: int = 64, stream=None):
     """Stage 1 of the tensor-core prefill (chunk table + preparation) into `workspace`."""
     lib = load()
+    _dtype_code(q)
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q and v must be [T, H, d]")
+    _check_prefill(q, k, v, g, beta, cu_seqlens, None, None, None, workspace=workspace)
     T, H, dk = q.shape
     dv = v.shape[2]
     N = cu_seqlens.shape[0] - 1
@@ -269,8 +338,15 @@ def kda_prefill_scan(out, cu_seqlens, workspace, initial_state=None, final_state
     """Stage 2: the chunk recurrence with the chunk outputs beside it; reads initial_state,
     writes `out` [T, H, D] bf16 and final_state."""
     lib = load()
+    _dtype_code(out)
+    if out.dim() != 3 or cu_seqlens.dim() != 1:
+        raise ValueError("out must be [T, H, D] and cu_seqlens [N+1]")
     T, H, D = out.shape
     N = cu_seqlens.shape[0] - 1
+    _check(out.device, out=(out, (T, H, D), out.dtype), cu_seqlens=(cu_seqlens, (N + 1,), torch.int32),
+           initial_state=(initial_state, (N, H, D, D), torch.float32),
+           final_state=(final_state, (N, H, D, D), torch.float32),
+           workspace=(workspace, (workspace.numel(),) if workspace is not None else (), torch.uint8))
     st = lib.kda_prefill_scan(_ptr(initial_state), _ptr(final_state), _ptr(out), _ptr(cu_seqlens), N,
                               T, H, D, D, _dtype_code(out), C, _ptr(workspace), _ws(workspace),
                               _stream(stream))
@@ -298,6 +374,8 @@ def kda_decode_gdn(q, k, v, g, beta, state, out, stream=None):
 def kda_decode_ex(q, k, v, g, beta, state, out, in_flags: int = 0, stream=None):
     """kda_decode with an input prologue (KDA_IN_* flags; with KDA_IN_G_SCALAR g is [N, H])."""
     lib = load()
+    _dtype_code(q)
+    _check_decode(q, k, v, g, beta, state, out, scalar_g=bool(int(in_flags) & KDA_IN_G_SCALAR))
     N, H, dk = q.shape
     dv = v.shape[2]
     st = lib.kda_decode_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
@@ -309,6 +387,8 @@ def kda_decode_ex(q, k, v, g, beta, state, out, in_flags: int = 0, stream=None):
 
 def _decode(fn, q, k, v, g, beta, state, out, stream):
     lib = load()
+    _dtype_code(q)
+    _check_decode(q, k, v, g, beta, state, out, scalar_g=fn == "kda_decode_gdn")
     N, H, dk = q.shape
     dv = v.shape[2]
     st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
