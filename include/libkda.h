@@ -292,7 +292,7 @@ const char *kda_status_string(kda_status s);
  */
 kda_status kda_get_device_status(kda_stream_t stream);
 
-/* ABI version of this header: 5. */
+/* ABI version of this header: 6. */
 int32_t kda_abi_version(void);
 
 #ifdef __cplusplus

@@ -45,7 +45,7 @@ cudaError_t dispatch_simt(int32_t dk, int32_t C, const void* q, const void* k, c
 
 extern "C" {
 
-int32_t kda_abi_version(void) { return 5; }
+int32_t kda_abi_version(void) { return 6; }
 
 const char* kda_status_string(kda_status s) {
     switch (s) {

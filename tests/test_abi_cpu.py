@@ -30,14 +30,24 @@ def test_header_declares_expected_entry_points():
     assert set(declared_functions()) == set(kda.EXPORTED)
 
 
+def test_header_constants_match_the_binding():
+    """Every KDA_* enum value the header declares has the same value in the binding."""
+    with open(os.path.join(ROOT, "include", "libkda.h")) as fh:
+        text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+    consts = dict((n, int(v)) for n, v in re.findall(r"\b(KDA_[A-Z0-9_]+)\s*=\s*(\d+)", text))
+    assert len(consts) >= 13
+    for name, value in consts.items():
+        assert getattr(kda, name) == value, name
+
+
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
 
 
 def test_status_strings_and_version(lib):
-    assert kda.kda_abi_version() == 5
-    for code in range(6):
+    assert kda.kda_abi_version() == 6
+    for code in range(7):
         s = kda.kda_status_string(code)
         assert s and s != "unknown status"
     assert kda.kda_status_string(99) == "unknown status"
