@@ -72,6 +72,55 @@ def test_strong_decay_flag_is_bit_identical_on_mild_decay(dtype, D):
     np.testing.assert_array_equal(f0, f1)
 
 
+@pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_degenerate_beta_zero_is_pure_channel_decay(dtype, D):
+    """beta = 0 writes nothing: the state only decays channel-wise, S_T = diag(e^{sum g}) S_0
+    (closed form, checked directly in fp64), and every output is read from it."""
+    lens = [200, 64, 7]
+    inp = _inputs(lens, 2, D, dtype, seed=23)
+    inp["beta"].zero_()
+    out, fin = run_prefill(inp)
+    check_prefill(inp, out, fin)
+    cu = inp["cu_seqlens"].tolist()
+    g = inp["g"].double().numpy()
+    s0 = inp["s0"].double().numpy()
+    import oracle
+    for n in range(len(lens)):
+        decay = np.exp(g[cu[n]:cu[n + 1]].sum(0))          # [H, dk]
+        ref = decay[:, :, None] * s0[n]
+        assert oracle.max_rel_frobenius_states(fin[n:n + 1], ref[None]) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_degenerate_no_decay_is_the_delta_rule(dtype, D):
+    """g = 0 (alpha = 1): the plain delta rule, no forgetting over 300 tokens."""
+    inp = _inputs([300, 65], 2, D, dtype, seed=29)
+    inp["g"].zero_()
+    out, fin = run_prefill(inp)
+    check_prefill(inp, out, fin)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_degenerate_orthonormal_keys_retrieve_values_exactly(D):
+    """beta = 1, alpha = 1, orthonormal keys (T <= dk), zero initial state, fp32: after
+    every token t the state returns each value written so far exactly, S_t^T k_i = v_i, so
+    with q_t = k_t the output is v_t; checked on the GPU's outputs and final state."""
+    T, H = 48, 2
+    gen = torch.Generator().manual_seed(37)
+    k = torch.empty(T, H, D)
+    for h in range(H):
+        Q, _ = torch.linalg.qr(torch.randn(D, D, generator=gen, dtype=torch.float64))
+        k[:, h] = Q[:, :T].T.float()
+    inp = dict(q=k.clone(), k=k, v=torch.randn(T, H, D, generator=gen), g=torch.zeros(T, H, D),
+               beta=torch.ones(T, H), cu_seqlens=torch.tensor([0, T], dtype=torch.int32), s0=None)
+    out, fin = run_prefill(inp)
+    v = inp["v"].double().numpy()
+    kk = k.double().numpy()
+    retrieved = np.einsum("hcv,thc->thv", fin[0], kk)        # S_T^T k_i for every key
+    assert np.abs(retrieved - v).max() <= 1e-4 * np.abs(v).max()
+    assert np.abs(out - v).max() <= 1e-4 * np.abs(v).max()
+
+
 def test_bf16_d64():
     inp = _inputs([130, 64, 7], 2, 64, torch.bfloat16, seed=12)
     out, fin = run_prefill(inp, C=64)
