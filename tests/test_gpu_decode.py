@@ -77,3 +77,33 @@ def test_decode_chain_equals_prefill_fp32():
         kda.kda_decode(d["q"], d["k"], d["v"], d["g"], d["beta"], S, o)
         assert oracle.rel_frobenius(o[0].double().cpu().numpy(), out[t]) <= 1e-4
     assert oracle.rel_frobenius(S.double().cpu().numpy(), fin) <= 1e-4
+
+
+@pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_decode_degenerate_cases_closed_form(dtype, D):
+    """beta = 0: one step only decays the state, S = diag(e^g) S, and reads o = S^T q.
+    beta = 1 with a unit key k: the step stores v under k exactly, S^T k = v.  Both are
+    checked in fp64 against the closed forms (fp32 state arithmetic throughout)."""
+    N, H = 4, 2
+    S0 = synthetic.make_decode_state(N, H, D, D, 0.02, 11)
+    x = _step(N, H, D, dtype, 11, 0)
+    q, k, v, g = (x[n].double().numpy() for n in ("q", "k", "v", "g"))
+    # beta = 0
+    S = S0.cuda()
+    out = torch.empty(N, H, D, dtype=dtype, device="cuda")
+    kda.kda_decode(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), x["g"].cuda(),
+                   torch.zeros(N, H, device="cuda"), S, out)
+    S_ref = np.exp(g)[..., None] * S0.double().numpy()
+    o_ref = np.einsum("nhcv,nhc->nhv", S_ref, q)
+    assert oracle.max_rel_frobenius_states(S.double().cpu().numpy(), S_ref) <= 1e-6
+    assert oracle.rel_frobenius(out.double().cpu().numpy(), o_ref) <= (1e-5 if dtype == torch.float32 else 5e-3)
+    # beta = 1: the step stores u = v - S'^T k under k, so S^T k = v |k|^2 + S'^T k (1 - |k|^2)
+    # (= v for a unit key; bf16 keys are unit only to ~2^-9, hence the general form)
+    S = S0.cuda()
+    kda.kda_decode(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), x["g"].cuda(),
+                   torch.ones(N, H, device="cuda"), S, out)
+    err = np.einsum("nhcv,nhc->nhv", S.double().cpu().numpy(), k) - v * (k * k).sum(-1, keepdims=True)
+    Sp = np.exp(g)[..., None] * S0.double().numpy()
+    err -= np.einsum("nhcv,nhc->nhv", Sp, k) * (1 - (k * k).sum(-1, keepdims=True))
+    assert np.abs(err).max() <= 1e-5 * max(1.0, np.abs(v).max())
+    assert kda.kda_get_device_status() == kda.KDA_OK
