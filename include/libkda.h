@@ -25,6 +25,9 @@
  *   - Work is enqueued on `stream` (NULL = the legacy default stream) and is
  *     asynchronous: no entry point synchronises the host with the device, except
  *     kda_get_device_status.
+ *   - Entry points may be called from several host threads at once; calls whose work
+ *     may overlap on the GPU must not share a workspace (nor, for kda_prefill_noalloc,
+ *     a device).
  *   - Arguments are checked before anything is launched; a bad argument returns a
  *     status and launches nothing.  Nothing aborts, throws or prints.
  *   - Errors the device detects (inconsistent cu_seqlens, an expired bounded wait)

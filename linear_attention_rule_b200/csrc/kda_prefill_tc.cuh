@@ -37,6 +37,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <atomic>
 #include <type_traits>
 
 #include "kda_common.cuh"
@@ -1100,17 +1101,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Looked up once; a function-local static is initialised exactly once even when several
+// host threads make their first call at the same time.
 inline EncodeTiledFn encode_tiled() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
+    static const EncodeTiledFn fn = [] {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-        tried = true;
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return static_cast<EncodeTiledFn>(nullptr);
+    }();
     return fn;
 }
 
@@ -1140,15 +1141,18 @@ inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs) {
             base + ws_records_offset(total, num_seqs)};
 }
 
-// SMs of the current device (cached per device; 0 when the query fails).
+// SMs of the current device (cached per device; 0 when the query fails).  Host threads
+// may race on the first query of a device: they store the same value, atomically.
 inline int device_sm_count() {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (cached[dev] == 0 &&
-        cudaDeviceGetAttribute(&cached[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        cached[dev] = 0;
-    return cached[dev];
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cached[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
 }
 
 // Chunk table (+ emission slots when emit_pos is given) + chunk-parallel preparation.
