@@ -1,7 +1,7 @@
 """GPU: the fused input prologue (kda_prefill_ex / kda_decode_ex with KDA_IN_* flags) on raw
-layer inputs, against the fp64 oracle given the inputs transformed on the CPU in fp64 from
-the same bytes: q / ||q||, k / ||k||, logsigmoid of the gate logits, sigmoid of the beta
-logits (the plain definitions; clamp of the norm as torch's F.normalize)."""
+layer inputs, against the fp64 oracle given the inputs transformed by the oracle's own
+fp64 prologue (oracle.prologue: q / max(||q||, 1e-12), the same for k, logsigmoid of the
+gate logits, sigmoid of the beta logits) from the same bytes."""
 import numpy as np
 import pytest
 import torch
@@ -16,20 +16,16 @@ ALL = kda.KDA_IN_NORMALIZE_QK | kda.KDA_IN_G_LOGITS | kda.KDA_IN_BETA_LOGITS
 
 
 def _transformed(raw, flags, scalar_gate=False):
-    """fp64 restatement of the prologue, returned as fp32 tensors for the oracle."""
-    f = lambda t: t.double()
-    q, k, g, b = f(raw["q"]), f(raw["k"]), f(raw["g"]), f(raw["beta"])
-    if flags & kda.KDA_IN_NORMALIZE_QK:
-        q = q / q.norm(dim=-1, keepdim=True).clamp_min(1e-12)
-        k = k / k.norm(dim=-1, keepdim=True).clamp_min(1e-12)
-    if flags & kda.KDA_IN_G_LOGITS:
-        g = -torch.nn.functional.softplus(-g)
-    if flags & kda.KDA_IN_BETA_LOGITS:
-        b = torch.sigmoid(b)
+    """oracle.prologue on the raw inputs; fp64 arrays for the oracle's recurrence (which
+    reads its inputs as fp32, so they are handed over rounded to fp32)."""
+    q, k, g, b = oracle.prologue(raw["q"], raw["k"], raw["g"], raw["beta"],
+                                 bool(flags & kda.KDA_IN_NORMALIZE_QK),
+                                 bool(flags & kda.KDA_IN_G_LOGITS),
+                                 bool(flags & kda.KDA_IN_BETA_LOGITS))
     if scalar_gate:
-        g = g[..., None].expand(*g.shape, q.shape[-1])
-    return {"q": q.float(), "k": k.float(), "v": raw["v"].float(), "g": g.float().contiguous(),
-            "beta": b.float()}
+        g = np.broadcast_to(g[..., None], g.shape + (q.shape[-1],))
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return {"q": f32(q), "k": f32(k), "v": raw["v"].float(), "g": f32(g), "beta": f32(b)}
 
 
 @pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.float32, 64), (torch.bfloat16, 64)])
@@ -39,12 +35,11 @@ def test_prefill_prologue_matches_oracle(dtype, D, flags):
     raw = synthetic.make_raw_prefill_inputs(lens, 3, D, D, dtype, 3.0, 0.02, 121 + D + flags)
     if not flags & kda.KDA_IN_NORMALIZE_QK:  # then q and k must arrive normalised (the method
         for key in ("q", "k"):                # assumes unit keys: the delta rule is unstable without)
-            x = raw[key].float()
-            raw[key] = (x / x.norm(dim=-1, keepdim=True).clamp_min(1e-12)).to(dtype)
+            raw[key] = torch.from_numpy(oracle.l2_normalize(raw[key])).to(dtype)
     if not flags & kda.KDA_IN_G_LOGITS:      # then g must already be a log-decay
-        raw["g"] = -torch.nn.functional.softplus(-raw["g"])
+        raw["g"] = torch.from_numpy(oracle.logsigmoid(raw["g"])).float()
     if not flags & kda.KDA_IN_BETA_LOGITS:
-        raw["beta"] = torch.sigmoid(raw["beta"])
+        raw["beta"] = torch.from_numpy(oracle.sigmoid(raw["beta"])).float()
     d = to_device(raw)
     T = d["q"].shape[0]
     out = torch.full((T, 3, D), float("nan"), dtype=dtype, device="cuda")

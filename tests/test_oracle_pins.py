@@ -251,3 +251,117 @@ def test_metric_helpers():
     ref = np.ones((4, 3))
     assert oracle.rel_frobenius(ref * 1.01, ref) == pytest.approx(0.01)
     assert oracle.rel_frobenius(np.zeros(3) + 1e-3, np.zeros(3)) == pytest.approx(math.sqrt(3) * 1e-3)
+
+
+def _slices_with_known_errors():
+    """Outputs [T=5, H=2, dv=2] of three sequences (lengths 2, 0, 3) with reference 1
+    everywhere and one perturbed element per (sequence, head) slice, so each slice's
+    relative Frobenius error is delta / sqrt(2 len) (hand-computed below).  The worst
+    slice is the last sequence's last head."""
+    cu = [0, 2, 2, 5]
+    ref = np.ones((5, 2, 2))
+    out = ref.copy()
+    out[0, 0, 0] += 0.02      # seq 0 head 0: 0.02 / sqrt(4) = 0.01
+    out[1, 1, 1] += 0.04      # seq 0 head 1: 0.04 / 2 = 0.02
+    out[3, 0, 0] += 0.06      # seq 2 head 0: 0.06 / sqrt(6) = 0.0244949
+    out[4, 1, 0] -= 0.12      # seq 2 head 1: 0.12 / sqrt(6) = 0.0489898
+    return cu, out, ref
+
+
+def test_max_rel_frobenius_per_slice_takes_the_worst_slice():
+    cu, out, ref = _slices_with_known_errors()
+    worst = oracle.max_rel_frobenius_per_slice(out, ref, cu)
+    assert worst == pytest.approx(0.12 / math.sqrt(6), rel=1e-12)
+    # not the mean of the four slices, not the first sequence alone, not the global error
+    assert worst > 1.5 * np.mean([0.01, 0.02, 0.06 / math.sqrt(6), 0.12 / math.sqrt(6)])
+    assert worst > 0.02 + 1e-9
+    assert abs(worst - oracle.rel_frobenius(out, ref)) > 1e-3
+    # dropping the last sequence (an off-by-one on cu_seqlens) would miss the worst slice
+    assert oracle.max_rel_frobenius_per_slice(out[:2], ref[:2], cu[:2]) == pytest.approx(0.02)
+    # the empty sequence contributes nothing; its neighbours still count
+    assert oracle.max_rel_frobenius_per_slice(out, ref, [0, 0, 2, 5]) == pytest.approx(worst)
+
+
+def test_max_rel_frobenius_per_slice_absolute_branch():
+    """A slice whose reference is zero is judged by its absolute error."""
+    cu = [0, 1, 3]
+    ref = np.ones((3, 2, 2))
+    ref[1:, 1] = 0.0                 # seq 1, head 1: zero reference
+    out = ref.copy()
+    out[2, 1, 0] = 3e-3              # absolute error 3e-3 there
+    out[0, 0, 0] += 1e-4             # seq 0 head 0: 1e-4 / sqrt(2)
+    assert oracle.max_rel_frobenius_per_slice(out, ref, cu) == pytest.approx(3e-3, rel=1e-12)
+
+
+def test_max_rel_frobenius_states_takes_the_worst_state():
+    ref = np.ones((3, 2, 2, 2))      # [N, H, dk, dv]: every state has norm 2
+    S = ref.copy()
+    S[0, 0, 0, 0] += 0.01            # 0.005
+    S[1, 1, 1, 0] += 0.02            # 0.01
+    S[2, 1, 1, 1] -= 0.08            # 0.04: the last sequence's last head
+    assert oracle.max_rel_frobenius_states(S, ref) == pytest.approx(0.04, rel=1e-12)
+    assert oracle.max_rel_frobenius_states(S[:2], ref[:2]) == pytest.approx(0.01, rel=1e-12)
+    Z = np.zeros((1, 1, 2, 2))
+    assert oracle.max_rel_frobenius_states(Z + 2e-3, Z) == pytest.approx(4e-3, rel=1e-12)
+
+
+def test_max_rel_frobenius_per_chunk_sees_one_bad_row():
+    """One wrong row in a 600-token slice: the per-slice error stays small, the error of
+    its own chunk (C = 64, the row's chunk 2 of 10, the last one 24 rows) does not."""
+    T, C = 600, 64
+    ref = np.ones((T, 1, 4))
+    out = ref.copy()
+    out[150, 0, :] = 0.0             # row 150 lies in chunk [128, 192)
+    per_slice = oracle.max_rel_frobenius_per_slice(out, ref, [0, T])
+    per_chunk = oracle.max_rel_frobenius_per_chunk(out, ref, [0, T], C)
+    assert per_slice == pytest.approx(math.sqrt(4 / (4 * T)), rel=1e-12)     # 0.0408
+    assert per_chunk == pytest.approx(math.sqrt(4 / (4 * C)), rel=1e-12)     # 0.125
+    # chunks restart at each sequence start: the same row as the 23rd of a second
+    # sequence starting at 128 falls in that sequence's first chunk [128, 192)
+    assert oracle.max_rel_frobenius_per_chunk(out, ref, [0, 128, T], C) == pytest.approx(0.125)
+    # the partial last chunk (rows 576..599) is compared on its own rows
+    out2 = ref.copy()
+    out2[590, 0, 0] = 1.48
+    assert oracle.max_rel_frobenius_per_chunk(out2, ref, [0, T], C) == pytest.approx(
+        0.48 / math.sqrt(4 * 24), rel=1e-12)
+
+
+def test_prologue_definitions():
+    """The prologue's three functions at values fixed by their definitions."""
+    assert oracle.logsigmoid(np.array([0.0]))[0] == pytest.approx(-math.log(2), rel=1e-15)
+    assert oracle.sigmoid(np.array([0.0]))[0] == 0.5
+    # sigmoid(ln 3) = 3/4, logsigmoid(ln 3) = ln(3/4), sigmoid(-ln 3) = 1/4
+    x = np.array([math.log(3.0), -math.log(3.0)])
+    np.testing.assert_allclose(oracle.sigmoid(x), [0.75, 0.25], rtol=1e-15)
+    np.testing.assert_allclose(oracle.logsigmoid(x), [math.log(0.75), math.log(0.25)], rtol=1e-15)
+    # tails: logsigmoid(x) -> x as x -> -inf and -> -e^{-x} as x -> +inf; no overflow
+    big = np.array([-1000.0, 1000.0, 40.0])
+    ls = oracle.logsigmoid(big)
+    assert ls[0] == -1000.0 and ls[1] == 0.0
+    assert ls[2] == pytest.approx(-math.exp(-40.0), rel=1e-12)
+    np.testing.assert_array_equal(oracle.sigmoid(big[:2]), [0.0, 1.0])
+    # the log-decay is log(sigmoid) (a sign or a dropped log fails here)
+    xs = np.linspace(-20, 20, 81)
+    np.testing.assert_allclose(np.exp(oracle.logsigmoid(xs)), oracle.sigmoid(xs), rtol=1e-14)
+    assert np.all(oracle.logsigmoid(xs) < 0)
+    # L2 norm over the last axis with a 1e-12 clamp
+    np.testing.assert_allclose(oracle.l2_normalize(np.array([3.0, 4.0])), [0.6, 0.8], rtol=1e-15)
+    np.testing.assert_array_equal(oracle.l2_normalize(np.zeros((2, 3))), np.zeros((2, 3)))
+    np.testing.assert_allclose(oracle.l2_normalize(np.array([1e-13, 0.0])), [0.1, 0.0], rtol=1e-12)
+    m = oracle.l2_normalize(np.array([[[1.0, 0.0], [0.0, 2.0]]]))        # per row, not per tensor
+    np.testing.assert_array_equal(m, [[[1.0, 0.0], [0.0, 1.0]]])
+
+
+def test_prologue_applies_each_flag_alone():
+    rng = np.random.default_rng(5)
+    q, k = rng.standard_normal((3, 2, 4)), rng.standard_normal((3, 2, 4))
+    g, b = rng.standard_normal((3, 2, 4)), rng.standard_normal((3, 2))
+    q1, k1, g1, b1 = oracle.prologue(q, k, g, b, True, False, False)
+    np.testing.assert_allclose(np.linalg.norm(q1, axis=-1), 1.0, rtol=1e-15)
+    np.testing.assert_allclose(q1 * np.linalg.norm(q, axis=-1, keepdims=True), q, rtol=1e-14)
+    np.testing.assert_array_equal(g1, g)
+    np.testing.assert_array_equal(b1, b)
+    _, k2, g2, b2 = oracle.prologue(q, k, g, b, False, True, True)
+    np.testing.assert_array_equal(k2, k)
+    np.testing.assert_allclose(g2, np.log(1.0 / (1.0 + np.exp(-g))), rtol=1e-14)
+    np.testing.assert_allclose(b2, 1.0 / (1.0 + np.exp(-b)), rtol=1e-14)
