@@ -106,3 +106,62 @@ def kda_prefill_chunked(q, k, v, g, beta, cu_seqlens, C, s0=None):
                 out[t0:t1, h] = O
             s_final[n, h] = S
     return out, s_final
+
+
+def chunk_affine(T):
+    """One chunk as an affine map of its starting state: S_out = A S_in + b with
+    A = diag(gamma) - K_res^T W and b = K_res^T U (chunk_step with U' = U - W S_in
+    substituted)."""
+    A = np.diag(T["gamma"]) - T["K_res"].T @ T["W"]
+    b = T["K_res"].T @ T["U"]
+    return A, b
+
+
+def kda_prefill_segmented(q, k, v, g, beta, cu_seqlens, C, seg, s0=None):
+    """The chunked prefill computed as a chunk-parallel scan, in fp64.  Each sequence's
+    chunks are cut into segments of `seg` chunks.  Pass 1: every segment, from a zero
+    state, gives its local final state b_p and its transition A_p (the product of the
+    chunks' affine maps, later chunks on the left).  Pass 2: the segments' starting states
+    S_in(p+1) = A_p S_in(p) + b_p from S_in(0) = the initial state.  Pass 3: every segment
+    runs chunk_step from its S_in(p) and writes its outputs.  Returns (out, s_final) as
+    kda_prefill_chunked does.  (Derived from the FlashKDA section's unrolled form: the
+    recurrence over a span of tokens is affine in the state it starts from.)"""
+    q, k, v, g, beta = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, beta))
+    cu = [int(x) for x in np.asarray(cu_seqlens)]
+    T_, H, dk = q.shape
+    dv = v.shape[2]
+    N = len(cu) - 1
+    out = np.zeros((T_, H, dv))
+    s_final = np.zeros((N, H, dk, dv))
+    for n in range(N):
+        starts = list(range(cu[n], cu[n + 1], C))
+        segments = [starts[i:i + seg] for i in range(0, len(starts), seg)] or [[]]
+        for h in range(H):
+            tens = {}
+            for t0 in starts:
+                t1 = min(t0 + C, cu[n + 1])
+                tens[t0] = chunk_tensors(q[t0:t1, h], k[t0:t1, h], v[t0:t1, h], g[t0:t1, h],
+                                         beta[t0:t1, h])
+            # pass 1
+            trans = []
+            for sg in segments:
+                A = np.eye(dk)
+                b = np.zeros((dk, dv))
+                for t0 in sg:
+                    Ac, bc = chunk_affine(tens[t0])
+                    A = Ac @ A
+                    b = Ac @ b + bc
+                trans.append((A, b))
+            # pass 2
+            S_in = [np.zeros((dk, dv)) if s0 is None else np.asarray(s0[n, h], dtype=np.float64).copy()]
+            for A, b in trans[:-1]:
+                S_in.append(A @ S_in[-1] + b)
+            # pass 3
+            for p, sg in enumerate(segments):
+                S = S_in[p]
+                for t0 in sg:
+                    O, S = chunk_step(S, tens[t0])
+                    out[t0:t0 + O.shape[0], h] = O
+                if p == len(segments) - 1:
+                    s_final[n, h] = S
+    return out, s_final

@@ -75,3 +75,31 @@ def test_forward_substitution_against_closed_form_2x2():
     L = np.array([[0.0, 0.0], [0.3, 0.0]])
     np.testing.assert_array_equal(chunked.forward_substitution_inverse(L),
                                   np.array([[1.0, 0.0], [-0.3, 1.0]]))
+
+
+@pytest.mark.parametrize("seg", [1, 2, 3, 7])
+def test_segmented_scan_equals_recurrence(seg):
+    """The chunk-parallel scan (segment transitions composed, then every segment run from
+    its starting state) equals the token recurrence, for varlen sequences with empty, short
+    and long members and a nonzero initial state."""
+    lens = [0, 1, 63, 64, 65, 700]
+    T, H, dk, dv = sum(lens), 2, 8, 5
+    q, k, v, g, beta = _inputs(T, H, dk, dv, 90 + seg)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    s0 = np.random.default_rng(91).standard_normal((len(lens), H, dk, dv))
+    o_ref, f_ref = oracle.prefill(q, k, v, g, beta, cu, s0=s0)
+    o, f = chunked.kda_prefill_segmented(q, k, v, g, beta, cu, 64, seg, s0=s0)
+    assert oracle.rel_frobenius(o, o_ref) < 1e-12
+    assert oracle.rel_frobenius(f, f_ref) < 1e-12
+
+
+def test_chunk_affine_map_matches_chunk_step():
+    """chunk_step is affine in S_in: S_out(S) = A S + b, with b the result from zero."""
+    q, k, v, g, beta = _inputs(64, 1, 8, 5, 93)
+    Tc = chunked.chunk_tensors(q[:, 0], k[:, 0], v[:, 0], g[:, 0], beta[:, 0])
+    A, b = chunked.chunk_affine(Tc)
+    S = np.random.default_rng(94).standard_normal((8, 5))
+    _, S_out = chunked.chunk_step(S, Tc)
+    _, b0 = chunked.chunk_step(np.zeros((8, 5)), Tc)
+    np.testing.assert_allclose(b, b0, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(S_out, A @ S + b, rtol=1e-12, atol=1e-12)
