@@ -149,7 +149,7 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, device, period_s: float = 0.002):
+    def __init__(self, device, period_s: float = 0.0002):
         self.period = period_s
         self.samples, self.max_mhz, self.ok = [], None, False
         self._stop = threading.Event()
@@ -250,7 +250,7 @@ def setup_prefill(dev, rank, cfg_id=PREFILL_CFG):
     cfg = synthetic.CONFIGS[cfg_id]
     lengths = synthetic.draw_lengths(cfg)
     D, H, C = cfg.D, cfg.H, cfg.C
-    if sum(lengths) * H > (1 << 24):   # large batches are drawn on the device (same recipe)
+    if sum(lengths) * H > (1 << 22):   # large batches are drawn on the device (same recipe)
         d = synthetic.make_prefill_inputs_device(lengths, H, D, D, cfg.dtype, cfg.g_mean,
                                                  cfg.s0_std, rank_seed(cfg.seed, rank), device=dev)
         d.pop("cpu")
@@ -288,7 +288,7 @@ def bench_prefill(args, P, dev, stream, world, peaks):
                                   d["s0"] is not None, True)
     t_s = ms_local * 1e-3
     res = dict(value=world * T / (ms * 1e-3), ms=ms, ms_local=ms_local, clocks=clocks,
-               launches=kda.prefill_launches(cfg.dtype, D) * args.steps, step=step,
+               launches=kda.kda_prefill_launches(T, P["N"], H, D, D, C, cfg.dtype) * args.steps, step=step,
                whole_frac=page_bytes / t_s / 1e9 / peaks["hbm_gbs"],
                tensor_frac=flops / t_s / 1e12 / peaks["bf16_tflops"],
                strict_frac=strict / t_s / 1e9 / peaks["hbm_gbs"])
@@ -296,7 +296,7 @@ def bench_prefill(args, P, dev, stream, world, peaks):
     # Per kernel: the same work through the staged entry points, CUDA events between the
     # stages on the launching stream.
     stage_ms = None
-    if kda.prefill_launches(cfg.dtype, D) > 1:
+    if kda.tensor_core_path(cfg.dtype, D):
         ws = P["ws"]
         stages = [
             ("prep_kernel", lambda: kda.kda_prefill_prepare(d["q"], d["k"], d["v"], d["g"], d["beta"],
@@ -441,6 +441,40 @@ def bench_e2e(args, P, pre, dev, stream, world):
             "pipelined": "read-back of step i overlaps upload of step i+1"}
 
 
+def bench_crossover(args, dev, stream):
+    """Serial chains vs the chunk-parallel scan of the recurrence: kda_prefill_ex with and
+    without KDA_IN_SERIAL_CHAINS (the preparation is the same in both) on one long sequence
+    for a grid of (H, T); inputs drawn on the device."""
+    import torch
+    from linear_attention_rule_b200 import kda, synthetic
+    rows = []
+    for H, T in [(2, 1 << 18), (2, 1 << 20), (4, 1 << 16), (4, 1 << 18), (4, 1 << 20), (8, 1 << 16),
+                 (8, 1 << 18), (8, 1 << 20), (16, 1 << 15), (16, 1 << 18), (32, 8192), (32, 1 << 15),
+                 (32, 1 << 18)]:
+        d = synthetic.make_prefill_inputs_device([T], H, 128, 128, torch.bfloat16, 3.0, 0.0, 77, device=dev)
+        d.pop("cpu")
+        out = torch.empty(T, H, 128, dtype=torch.bfloat16, device=dev)
+        fin = torch.empty(1, H, 128, 128, device=dev)
+        ws = torch.empty(kda.kda_prefill_workspace_size(T, 1, H, 128, 128, 64, torch.bfloat16),
+                         dtype=torch.uint8, device=dev)
+        res = {}
+        for name, flags in (("serial", kda.KDA_IN_SERIAL_CHAINS), ("auto", 0)):
+            def step():
+                kda.kda_prefill_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out, flags,
+                                   final_state=fin, workspace=ws, stream=stream)
+            for _ in range(args.warmup):
+                step()
+            steps = max(2, min(args.steps, int(2e7 // (T * H)) + 2))
+            ms, _, _ = timed(stream, dev, 1, steps, step)
+            assert kda.kda_get_device_status(stream) == kda.KDA_OK
+            res[name] = round(ms, 4)
+        rows.append({"H": H, "T": T, "serial_ms": res["serial"], "auto_ms": res["auto"],
+                     "speedup": round(res["serial"] / res["auto"], 3)})
+        del d, out, fin, ws
+        torch.cuda.empty_cache()
+    return {"crossover": rows}
+
+
 def bench_gpu(args):
     import torch
     from linear_attention_rule_b200 import kda
@@ -455,8 +489,28 @@ def bench_gpu(args):
     peaks = load_peaks()
     stream = torch.cuda.current_stream(dev)
 
+    def prefill_config_entry(cfg_id):
+        """Another prefill configuration of the metric (few steps): tokens/s, the dominant
+        kernel's roofline and the path fractions, stage times and clocks."""
+        import argparse as _ap
+        sub = _ap.Namespace(**vars(args))
+        sub.steps = min(args.steps, 5)
+        P = setup_prefill(dev, rank, cfg_id)
+        pre = bench_prefill(sub, P, dev, stream, world, peaks)
+        entry = {"workload": P["cfg"].name, "T": P["T"], "num_seqs": P["N"],
+                 "value": round(pre["value"], 1), "unit": "tokens/s", "steps": sub.steps,
+                 "warmup": sub.warmup, "ms_per_step": round(pre["ms"], 4),
+                 "roofline": pre["roofline"], "stage_ms": pre.get("stage_ms"),
+                 "clocks": pre["clocks"], "gpu_launches": pre["launches"]}
+        del P, pre
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+        return entry
+
     line = {}
-    if args.workload in ("config2", "config4"):
+    if args.workload == "crossover":
+        line = bench_crossover(args, dev, stream)
+    elif args.workload in ("config2", "config4"):
         P = setup_prefill(dev, rank, int(args.workload[-1]))
         pre = bench_prefill(args, P, dev, stream, world, peaks)
         line = {"workload": P["cfg"].name, "value": round(pre["value"], 1), "unit": "tokens/s",
@@ -489,6 +543,12 @@ def bench_gpu(args):
             "e2e": e2e, "cpu_baseline": cpu, "clocks": pre["clocks"],
             "gpu_launches": pre["launches"],
         }
+        if args.workload == "all" and not args.no_extra_configs:
+            del P, pre
+            torch.cuda.synchronize(dev)
+            torch.cuda.empty_cache()
+            line["prefill_configs"] = {"config2": prefill_config_entry(2),
+                                       "config4": prefill_config_entry(4)}
     else:
         line = {"decode": bench_decode(args, dev, stream, rank, world, peaks)}
     if world > 1:
@@ -551,8 +611,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-configs", action="store_true",
+                    help="skip the varlen (config 2) and long-context (config 4) prefill entries")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--workload", choices=["all", "prefill", "decode", "config2", "config4"],
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "config2", "config4", "crossover"],
                     default="all",
                     help="restrict the run (profiling) or measure another prefill config; "
                          "the driver's JSON line is 'all'")

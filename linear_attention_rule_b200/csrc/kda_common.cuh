@@ -15,7 +15,7 @@ __device__ __forceinline__ void kda_set_status(int s) { atomicCAS(&g_kda_status,
 // Input prologue (the layer's elementwise steps in front of KDA, fused into the kernels):
 // bit flags as in include/libkda.h (KDA_IN_*).
 constexpr uint32_t kInNormQK = 1u, kInGLogits = 2u, kInBetaLogits = 4u, kInGScalar = 8u,
-                   kInStrongDecay = 16u;
+                   kInStrongDecay = 16u, kInSerialChains = 32u;
 // log(sigmoid(x)) = min(x, 0) - log(1 + e^{-|x|}), without overflow for either sign
 __device__ __forceinline__ float kda_logsigmoid(float x) { return fminf(x, 0.f) - log1pf(__expf(-fabsf(x))); }
 __device__ __forceinline__ float kda_sigmoid(float x) { return 1.f / (1.f + __expf(-x)); }

@@ -9,16 +9,23 @@
 // tokens i..j from S_in with the cumulative decay D_{j:i}; Q_decay, K_inv, K_restore,
 // the causal mask M_qk, the UT transform giving the pseudo-values U).  With the state
 // stored S[key][value] and a_r the inclusive, chunk-relative cumulative log-decay:
-//   Q_dec = q e^{a}, K_dec = k e^{a}, K_inv = k e^{-a}, K_res = K_inv e^{a_last},
-//   gamma = e^{a_last}
-//   L   = strict_tril(diag(beta) K_dec K_inv^T),  INV = (I + L)^{-1}
+//   Q_dec = q e^{a}, K_dec = k e^{a}, K_res = k e^{a_last - a}, gamma = e^{a_last}
+//   L   = strict_tril(diag(beta) (K_dec K_inv^T)),  INV = (I + L)^{-1}
 //   W   = INV diag(beta) K_dec,   U = INV diag(beta) V
 //   Aqk = tril(Q_dec K_inv^T)               (diagonal included)
 //   U'  = U - W S_in;  O = Q_dec S_in + Aqk U';  S_out = diag(gamma) S_in + K_res^T U'
+// where (X K_inv^T)[r][s] = sum_c x_rc k_sc e^{a_rc - a_sc}, K_inv = k e^{-a}.  Every factor
+// above is at most 1 except e^{-a}, which overflows fp32 once a chunk decays by ~88 in
+// some channel; so the products with K_inv are formed without it, per 16-token block b of
+// the rows r (chunk_l_aqk): with m_b = a at the row before the block,
+//   s in an earlier block:  (x_r e^{a_r - m_b}) . (k_s e^{m_b - a_s}),  both factors <= 1
+//   s in the same block:    sum_c x_rc k_sc e^{a_rc - a_sc}, one exponential per term,
+// so no exponent is ever positive and no decay, however strong, overflows.
 // Rows past the end of a partial chunk are zero-filled (q = k = v = g = beta = 0), which
 // makes them contribute nothing and leaves gamma = e^{a of the last real row}.
 #pragma once
 
+#include "kda_chunk_simt.cuh"
 #include "kda_common.cuh"
 
 namespace kda {
@@ -43,8 +50,7 @@ struct SimtSmem {
     static constexpr int BT = GM + DK;         // beta [C]
     static constexpr int NQ = BT + C;          // 1 / ||q_r||, 1 / ||k_r|| [C] (input prologue)
     static constexpr int NK = NQ + C;
-    static constexpr int HM = NK + C;          // e^{m}, m = a_last / 2, per key channel [DK]
-    static constexpr int TOTAL = HM + DK;
+    static constexpr int TOTAL = NK + C;
     static constexpr size_t BYTES = sizeof(float) * TOTAL;
 };
 
@@ -76,7 +82,6 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
     float* sB = sm + L::BT;
     float* sNq = sm + L::NQ;
     float* sNk = sm + L::NK;
-    float* sH = sm + L::HM;
     const bool g_scalar = (in_flags & kInGScalar) != 0;
 
     const int tid = threadIdx.x;
@@ -135,10 +140,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
         }
         __syncthreads();
 
-        // (2) inclusive cumulative sum over the chunk, per key channel; gamma = e^{a_last}.
-        // The decayed operands use exponents relative to m = a_last / 2 (stored as a - m):
-        // the products need only ratios e^{a_r - a_s}, and e^{a - m}, e^{m - a} stay within
-        // e^{|a_last| / 2} where e^{-a} alone would overflow once |a_last| nears 88.
+        // (2) inclusive cumulative sum over the chunk, per key channel; gamma = e^{a_last}
         for (int c = tid; c < DK; c += kSimtThreads) {
             float acc = 0.f;
             for (int r = 0; r < C; ++r) {
@@ -146,61 +148,48 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
                 sWA[r * PK + c] = acc;
             }
             sG[c] = expf(acc);
-            sH[c] = expf(0.5f * acc);
-            for (int r = 0; r < C; ++r) sWA[r * PK + c] -= 0.5f * acc;
         }
         __syncthreads();
 
-        // (3) decayed operands
-        for (int e = tid; e < C * DK; e += kSimtThreads) {
-            const int r = e / DK, c = e % DK;
-            float qq = 0.f, kk = 0.f;
+        // (3) raw q and k rows (the input prologue's norm applied)
+        auto load_qk = [&](int r, int c, float& qq, float& kk) {
+            qq = 0.f;
+            kk = 0.f;
             if (r < nrow) {
                 const size_t off = ((size_t)(t0 + r) * H + h) * DK + c;
                 qq = to_f32(q[off]);
                 kk = to_f32(k[off]);
                 if (in_flags & kInNormQK) { qq *= sNq[r]; kk *= sNk[r]; }
             }
+        };
+        for (int e = tid; e < C * DK; e += kSimtThreads) {
+            const int r = e / DK, c = e % DK;
+            load_qk(r, c, sQd[r * PK + c], sKd[r * PK + c]);
+        }
+        __syncthreads();
+
+        // (4) L = strict_tril(beta (K_dec K_inv^T)), Aqk = tril(Q_dec K_inv^T), with no
+        // positive exponent
+        chunk_l_aqk<DK, C, PK, PC, kSimtThreads>(sQd, sKd, sKi, sWA, sB, sL, sA, tid, [&](int r, int c) {
+            float qq, kk;
+            load_qk(r, c, qq, kk);
+            return kk;
+        });
+        // decayed operands relative to the chunk start (every factor <= 1)
+        for (int e = tid; e < C * DK; e += kSimtThreads) {
+            const int r = e / DK, c = e % DK;
+            float qq, kk;
+            load_qk(r, c, qq, kk);
             const float a = sWA[r * PK + c];
-            const float ep = expf(a), em = expf(-a);
+            const float ep = expf(a);
             sQd[r * PK + c] = qq * ep;
             sKd[r * PK + c] = kk * ep;
-            sKi[r * PK + c] = kk * em;
+            sKi[r * PK + c] = kk * expf(sWA[(C - 1) * PK + c] - a);   // K_res
         }
         __syncthreads();
 
-        // (4) L = strict_tril(beta K_dec K_inv^T), Aqk = tril(Q_dec K_inv^T)
-        for (int p = tid; p < C * C; p += kSimtThreads) {
-            const int r = p / C, s = p % C;
-            float l = 0.f, aq = 0.f;
-            if (s <= r) {
-                const float4* kd = reinterpret_cast<const float4*>(sKd + r * PK);
-                const float4* qd = reinterpret_cast<const float4*>(sQd + r * PK);
-                const float4* ki = reinterpret_cast<const float4*>(sKi + s * PK);
-#pragma unroll 8
-                for (int c4 = 0; c4 < DK / 4; ++c4) {
-                    const float4 x = ki[c4], y = kd[c4], z = qd[c4];
-                    l += y.x * x.x + y.y * x.y + y.z * x.z + y.w * x.w;
-                    aq += z.x * x.x + z.y * x.y + z.z * x.z + z.w * x.w;
-                }
-                l = s < r ? sB[r] * l : 0.f;
-            }
-            sL[r * PC + s] = l;
-            sA[r * PC + s] = aq;
-        }
-        __syncthreads();
-
-        // (5) UT transform: INV = (I + L)^{-1} by forward substitution, one column per thread
-        for (int j = tid; j < C; j += kSimtThreads) {
-            for (int r = 0; r < j; ++r) sI[r * PC + j] = 0.f;
-            sI[j * PC + j] = 1.f;
-            for (int r = j + 1; r < C; ++r) {
-                float acc = 0.f;
-                for (int s = j; s < r; ++s) acc += sL[r * PC + s] * sI[s * PC + j];
-                sI[r * PC + j] = -acc;
-            }
-        }
-        __syncthreads();
+        // (5) UT transform: INV = (I + L)^{-1} by forward substitution
+        chunk_ut_inverse<C, PC, kSimtThreads>(sL, sI, tid);
 
         // (6) W = INV diag(beta) K_dec  [C][DK];  U = INV diag(beta) V  [C][NV]
         {
@@ -213,8 +202,6 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
                     const float4 x = reinterpret_cast<const float4*>(sKd + s * PK)[c4];
                     w.x += co * x.x; w.y += co * x.y; w.z += co * x.z; w.w += co * x.w;
                 }
-                const float4 hm = reinterpret_cast<const float4*>(sH)[c4];   // K_dec = K_dec' e^{m}
-                w.x *= hm.x; w.y *= hm.y; w.z *= hm.z; w.w *= hm.w;
                 reinterpret_cast<float4*>(sWA + r * PK)[c4] = w;
             }
         }
@@ -256,7 +243,7 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
             for (int r = tid / JG; r < C; r += RG) {
                 float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int c = 0; c < DK; ++c) {
-                    const float a = sQd[r * PK + c] * sH[c];   // Q_dec = Q_dec' e^{m}
+                    const float a = sQd[r * PK + c];
                     const float4 x = reinterpret_cast<const float4*>(sS + c * NV)[j4];
                     o.x += a * x.x; o.y += a * x.y; o.z += a * x.z; o.w += a * x.w;
                 }
@@ -281,17 +268,16 @@ prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* _
 #pragma unroll
             for (int i = 0; i < CPT; ++i) {
                 const int c = tid / JG + i * CGR;
-                // S_out = gamma S_in + (K_inv' e^{a_last - m})^T U' with e^{a_last - m} = e^{m}
+                // S_out = gamma S_in + K_res^T U'
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int r = 0; r < C; ++r) {
-                    const float kinv = sKi[r * PK + c];
+                    const float kres = sKi[r * PK + c];
                     const float4 x = reinterpret_cast<const float4*>(sU + r * NV)[j4];
-                    acc.x += kinv * x.x; acc.y += kinv * x.y; acc.z += kinv * x.z; acc.w += kinv * x.w;
+                    acc.x += kres * x.x; acc.y += kres * x.y; acc.z += kres * x.z; acc.w += kres * x.w;
                 }
-                const float gm = sG[c], hm = sH[c];
+                const float gm = sG[c];
                 const float4 s0v = reinterpret_cast<const float4*>(sS + c * NV)[j4];
-                acc.x = gm * s0v.x + hm * acc.x; acc.y = gm * s0v.y + hm * acc.y;
-                acc.z = gm * s0v.z + hm * acc.z; acc.w = gm * s0v.w + hm * acc.w;
+                acc.x += gm * s0v.x; acc.y += gm * s0v.y; acc.z += gm * s0v.z; acc.w += gm * s0v.w;
                 snew[i] = acc;
             }
         }

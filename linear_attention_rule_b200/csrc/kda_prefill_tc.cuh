@@ -37,6 +37,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <algorithm>
 #include <atomic>
 #include <type_traits>
 
@@ -52,15 +53,18 @@ constexpr int D = 128;   // d_k = d_v
 constexpr int C = 64;    // chunk
 
 // ---- record of one (chunk, head) ---------------------------------------------------------
-// Shared-memory operand images (rows of 128 B, 128-byte swizzle), each 1024-byte aligned:
-constexpr uint32_t kRecP0 = 0;          // P     K-major rows r (64), key channels 0..63 / 64..127 (2 x 8 KB)
-constexpr uint32_t kRecM0 = 16384;      // M     K-major rows i (128), key channels 0..63 / 64..127 (2 x 16 KB)
-constexpr uint32_t kRecKR = 49152;      // K_res rows t (64), key channels i 0..63 / 64..127 (2 x 8 KB);
-                                        //       the MN-major A operand K_res^T
-constexpr uint32_t kRecU = 65536;       // U     rows t (64), value channels 32 s .. 32 s + 31 for the 4
-                                        //       value slices s (4 x 4 KB, rows of 64 B, 64-byte
-                                        //       swizzle): an MN-major B operand per slice
-constexpr uint32_t kRecAQ = 81920;      // Aqk   K-major rows r (64), tokens s (8 KB)
+// Shared-memory operand images (bf16, rows of 128 B, 128-byte swizzle unless said), each
+// 1024-byte aligned.  The recurrence reads two of them as the B operands of one product
+// stream of N = 192 (its state columns and its output columns together):
+constexpr uint32_t kRecSB = 0;          // [M ; P]  K-major, rows n: M's rows i (0..127), then P's rows r
+                                        //          (128..191); key channels 0..63 / 64..127 in two halves
+constexpr uint32_t kRecSBHalf = 24576;  //          of 24 KB
+constexpr uint32_t kRecP = 16384;       //          P's first row inside each half
+constexpr uint32_t kRecUB = 49152;      // K_res  rows t (64 tokens), key channels i 0..63 / 64..127 (2 x 8 KB):
+                                        //        the MN-major A operand K_res^T
+constexpr uint32_t kRecAQ = 65536;      // Aqk    K-major rows r (64), tokens s (8 KB)
+constexpr uint32_t kRecU = 73728;       // U  rows t (64), value channels 32 s .. 32 s + 31 for 4 slices s
+                                        //    (4 x 4 KB, rows of 64 B, 64-byte swizzle): MN-major U^T
 constexpr uint32_t kRecGamma = 90112;   // gamma fp32 [128]
 constexpr uint32_t kRecBytes = 90624;
 
@@ -70,21 +74,79 @@ __host__ inline int64_t max_chunks(int64_t total_tokens, int num_seqs) {
     return total_tokens / C + num_seqs;
 }
 // Workspace: [chunk offsets int32 (N+1)] [chunk table int2 (max_chunks)] [emission slot per
-// chunk int32 (max_chunks)] [records (max_chunks x H)]
+// chunk int32 (max_chunks)] [strong-decay count int32, pad] [strong-decay units int2
+// (max_chunks x H)] [records (max_chunks x H)]
 __host__ inline size_t ws_table_offset(int num_seqs) {
     return align_up(sizeof(int32_t) * (size_t)(num_seqs + 1), 16);
 }
 __host__ inline size_t ws_emit_offset(int64_t total_tokens, int num_seqs) {
     return align_up(ws_table_offset(num_seqs) + sizeof(int2) * (size_t)max_chunks(total_tokens, num_seqs), 16);
 }
-__host__ inline size_t ws_records_offset(int64_t total_tokens, int num_seqs) {
+__host__ inline size_t ws_strong_offset(int64_t total_tokens, int num_seqs) {
     return align_up(ws_emit_offset(total_tokens, num_seqs) +
                         sizeof(int32_t) * (size_t)max_chunks(total_tokens, num_seqs),
+                    16);
+}
+// Chunk-parallel scan over long chains ("SemiAnalysis Kimi K3", FlashKDA section: the
+// recurrence unrolled from S_in over a span of tokens is affine in S_in).  When few
+// (sequence, head) chains are long, each sequence is cut into segments of `seg` chunks:
+// every segment but the last runs from a zero state and composes its transition
+// T = prod (diag(gamma) + M) over its chunks (seg_kernel), the segments' starting states
+// follow as S_in(p+1) = T_p S_in(p) + S_local(p) (combine_kernel), and the recurrence then
+// runs every segment from its starting state (rec_kernel over segments).
+constexpr int kScanTargetCtas = 148;     // segments x heads aimed at (a B200's SM count)
+constexpr int kScanMinSegChunks = 64;    // shortest segment worth the extra passes (measured)
+// Chunks per segment, or 0 for one chain per (sequence, head).  The recurrence runs every
+// chain (or segment) as four value-slice CTAs, so segments pay while chains x 4 leave at least
+// half of the SMs idle.  Depends on the sizes only.
+__host__ inline int scan_segment_chunks(int64_t total_tokens, int num_seqs, int H) {
+    const int64_t chains = (int64_t)num_seqs * H;
+    if (num_seqs <= 0) return 0;
+    const int64_t segs = kScanTargetCtas / (chains * 4);   // segments per chain
+    if (segs < 2) return 0;
+    const int64_t per_chain = (total_tokens / num_seqs + C - 1) / C;   // mean chunks per sequence
+    const int64_t len = (per_chain + segs - 1) / segs;
+    return len >= kScanMinSegChunks && len < per_chain ? (int)len : 0;
+}
+__host__ inline int64_t max_segments(int64_t total_tokens, int num_seqs, int seg) {
+    return seg > 0 ? max_chunks(total_tokens, num_seqs) / seg + num_seqs : 0;
+}
+constexpr size_t kSegStateBytes = 3 * sizeof(float) * D * D;   // S_local, T, S_in per (segment, head)
+// [segment offsets int32 (N+1)] [segment count int32, pad] [segment table int4 (max_segs)]
+// [segment states (max_segs x H)]
+__host__ inline size_t ws_scan_offset(int64_t total_tokens, int num_seqs, int H) {
+    return align_up(ws_strong_offset(total_tokens, num_seqs) + 16 +
+                        sizeof(int2) * (size_t)max_chunks(total_tokens, num_seqs) * H,
+                    16);
+}
+__host__ inline size_t ws_scan_bytes(int64_t total_tokens, int num_seqs, int H) {
+    const int seg = scan_segment_chunks(total_tokens, num_seqs, H);
+    if (seg == 0) return 0;
+    const size_t ms = (size_t)max_segments(total_tokens, num_seqs, seg);
+    return align_up(sizeof(int32_t) * (num_seqs + 1), 16) + 16 + align_up(sizeof(int4) * ms, 1024) +
+           ms * H * kSegStateBytes;
+}
+__host__ inline size_t ws_records_offset(int64_t total_tokens, int num_seqs, int H) {
+    return align_up(ws_scan_offset(total_tokens, num_seqs, H) + ws_scan_bytes(total_tokens, num_seqs, H),
                     1024);
 }
 __host__ inline size_t workspace_bytes(int64_t total_tokens, int num_seqs, int H) {
-    return ws_records_offset(total_tokens, num_seqs) +
+    return ws_records_offset(total_tokens, num_seqs, H) +
            (size_t)max_chunks(total_tokens, num_seqs) * H * kRecBytes;
+}
+// The same size, or false when the problem exceeds what the launches can address: H above
+// the grid's y limit, a grid.x (chunks, or sequences x heads x value slices) beyond 2^31 - 1,
+// or a byte count that does not fit in size_t.
+__host__ inline bool workspace_bytes_checked(int64_t total_tokens, int num_seqs, int H, size_t* bytes) {
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0 || H > 65535) return false;
+    const int64_t mc = max_chunks(total_tokens, num_seqs);
+    if (mc > INT32_MAX || (int64_t)num_seqs * H * 4 > INT32_MAX) return false;
+    size_t rec = 0, total = 0;
+    if (__builtin_mul_overflow((size_t)mc * (size_t)H, (size_t)kRecBytes + sizeof(int2), &rec)) return false;
+    if (__builtin_add_overflow(rec, ws_records_offset(total_tokens, num_seqs, H), &total)) return false;
+    total = workspace_bytes(total_tokens, num_seqs, H);
+    *bytes = total;
+    return true;
 }
 
 // ------------------------------------------------------------------ chunk index
@@ -100,16 +162,17 @@ __device__ __forceinline__ int find_seq(const int32_t* off, int num_seqs, int c)
 
 // Single CTA of 1024 threads: off[n] = sum_{m<n} ceil(len_m / C), off[N] = total chunks,
 // and the chunk table tab[c] = (first token, rows) of every chunk c < off[N], so that the
-// chunk-parallel kernels find their tokens with one load.
+// chunk-parallel kernels find their tokens with one load; also empties the strong-decay list.
 // Inconsistent cu_seqlens -> KDA_ERR_BAD_SEQLENS and every count 0 (nothing downstream runs).
 __global__ void __launch_bounds__(1024)
 chunk_index_kernel(const int32_t* __restrict__ cu, int num_seqs, int64_t total,
-                   int32_t* __restrict__ off, int2* __restrict__ tab, int32_t* __restrict__ etab) {
+                   int32_t* __restrict__ off, int2* __restrict__ tab, int32_t* __restrict__ etab,
+                   int32_t* __restrict__ strong_count) {
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t carry;
     __shared__ int bad;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    if (tid == 0) { carry = 0; bad = 0; }
+    if (tid == 0) { carry = 0; bad = 0; *strong_count = 0; }
     __syncthreads();
     for (int base = 0; base < num_seqs; base += 1024) {
         const int n = base + tid;
@@ -214,6 +277,7 @@ struct PrepSmem {
     static constexpr uint32_t BARQK = BAR2 + 8;       // TMA of q and k
     static constexpr uint32_t BARV = BARQK + 8;       // TMA of v
     static constexpr uint32_t TMEM = BARV + 8;
+    static constexpr uint32_t STRONG = TMEM + 4;       // some channel's chunk decay is below kStrongDecay
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;  // + alignment slack
 };
 constexpr int kLP = 68;                                   // row pitch of L / INV (16-byte rows)
@@ -236,17 +300,22 @@ __device__ __forceinline__ uint32_t stage_slot(int w) {
     return base + (w & 1) * 4096;
 }
 
+// A chunk whose cumulative log-decay falls below this in some channel is not prepared here:
+// K_inv = k e^{-a} would leave the range of bf16 (~e^{88}).  The CTA lists it for
+// prep_strong_kernel, which forms the products with K_inv without a positive exponent.
+constexpr float kStrongDecay = -64.f;
+
 // One CTA per (chunk, head) unit, 2 CTAs per SM.  kScalarG: the gate is one log-decay per
 // (token, head), g [T, H] (Gated DeltaNet, the scalar forget gate that KDA makes diagonal):
 // the same decay on every channel, loaded like beta instead of through the g tensor map.
 // kPrologue: in_flags may hold KDA_IN_* prologue bits (the plain path compiles without them).
-// kStrong: channels whose chunk total decay passes -64 take exponents relative to half of it.
-template <bool kScalarG, bool kPrologue, bool kStrong>
+template <bool kScalarG, bool kPrologue>
 __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
             const float* __restrict__ g_scalar, const float* __restrict__ beta, int num_seqs, int H,
             const int32_t* __restrict__ off, const int2* __restrict__ tab, uint8_t* __restrict__ records,
+            int32_t* __restrict__ strong_count, int2* __restrict__ strong_units,
             uint32_t in_flags_arg, int64_t total) {
     const uint32_t in_flags = kPrologue ? in_flags_arg : 0u;
     using S = PrepSmem;
@@ -275,8 +344,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wh = warp >> 2;   // TMEM lane quarter, column half
     bool ok = true, v_ok = true;
-    uint32_t shifted = 0;   // kStrong: this thread's channels whose exponents are relative to a_last / 2
     uint32_t phase = 0;
+    volatile int* strong_flag = reinterpret_cast<volatile int*>(sm + S::STRONG);
 
     // ---- (0) TMA: rows t0..t0+63 of g, then q and k, then v (two 64-channel boxes each),
     // on three barriers in the order of use: the decay's prefix sums start once g is in, the
@@ -289,6 +358,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(barqk, 1);
         mbar_init(barv, 1);
         fence_mbar_init();
+        *strong_flag = 0;
         const int x0 = h * D;
         if (!kScalarG) {
             mbar_arrive_expect_tx(bar, kPrepTxG);
@@ -394,24 +464,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             gdst[0] = make_float4(gam[0], gam[1], gam[2], gam[3]);
             gdst[1] = make_float4(gam[4], gam[5], gam[6], gam[7]);
         }
-        // Strong decay (kStrong): in a channel whose total |a_last| passes 64 (e^{-a} overflows
-        // fp32 and bf16 near 88), the exponents are taken relative to half the chunk's total
-        // decay, m = a_last / 2.  L and Aqk only need the ratios e^{a_r - a_s}, and e^{a - m},
-        // e^{m - a} stay within e^{|a_last| / 2}.  Then gam = e^{m} for that channel, and after
-        // the first product K_dec and Q_dec are scaled back by it in place, and
-        // K_res = K_inv' e^{a_last - m} = K_inv' e^{m}.  Every thread holding a channel sees
-        // the same total, so the choice is the same for all its rows without a barrier.
-        // Milder channels keep a = 0 at the chunk start, K_res = K_inv gamma, bit for bit as
-        // without kStrong.
-        if constexpr (kStrong) {
+        {   // strong decay: acted on at the barrier after the decayed images (which may then
+            // hold infinities, never used)
+            bool strong = false;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (tot[u] < -64.f) {
-                    shifted |= 1u << u;
-                    base[u] -= 0.5f * tot[u];
-                    gam[u] = __expf(0.5f * tot[u]);
-                }
-            }
+            for (int u = 0; u < 8; ++u) strong |= tot[u] < kStrongDecay;
+            if (strong) *strong_flag = 1;
         }
         ok = mbar_wait(barqk, 0);   // q, k in (a failure is acted on at the barrier below)
 #pragma unroll
@@ -451,6 +509,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         fence_proxy_async_smem();
         if (!prep_sync_ok(ok, tid)) goto done;
+        if (*strong_flag) {   // every thread sees the flag after the barrier
+            if (tid == 0) {
+                const int slot = atomicAdd(strong_count, 1);
+                strong_units[slot] = make_int2(c, h);
+            }
+            goto done;
+        }
         KDA_TRACE_POINT(ptr_, 8192 + 2);
 
         // ---- (2) [K_dec ; Q_dec] K_inv^T -> TMEM [0, 64) ----
@@ -556,32 +621,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 *reinterpret_cast<float4*>(sLI + (R + r) * kLP + Cc + c8 + 4) = make_float4(t[4], t[5], t[6], t[7]);
             }
         }
-        // K_res = K_inv gamma (kStrong: K_inv' e^{m} in the shifted channels, whose K_dec and
-        // Q_dec are also scaled by e^{m}), in place: the first MMA has finished reading them;
-        // warps 1 and 4 also take the rows of warps 0 and 5
+        // K_res = K_inv gamma, in place: the first MMA has finished reading K_inv; warps 1
+        // and 4 also take the rows of warps 0 and 5
         auto kres_rows = [&](int wsrc) {
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr) {
                 const uint32_t o = kb * S::BLK + sw128_off(4 * (2 * wsrc + half) + rr, c8);
-                if constexpr (kStrong) {
+                float ki[8];
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::KI0 + o), ki);
 #pragma unroll
-                    for (int img = 0; img < 3; ++img) {
-                        if (img > 0 && !shifted) break;
-                        uint8_t* pimg = sm + (img == 0 ? S::KI0 : img == 1 ? S::KD0 : S::QD0) + o;
-                        float x[8];
-                        unpack_bf16x8(*reinterpret_cast<const uint4*>(pimg), x);
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            x[u] *= (img == 0 || ((shifted >> u) & 1u)) ? gam[u] : 1.f;
-                        *reinterpret_cast<uint4*>(pimg) = pack_bf16x8(x);
-                    }
-                } else {
-                    float ki[8];
-                    unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::KI0 + o), ki);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) ki[u] *= gam[u];
-                    *reinterpret_cast<uint4*>(sm + S::KI0 + o) = pack_bf16x8(ki);
-                }
+                for (int u = 0; u < 8; ++u) ki[u] *= gam[u];
+                *reinterpret_cast<uint4*>(sm + S::KI0 + o) = pack_bf16x8(ki);
             }
         };
         if (warp != 0 && warp != 5) kres_rows(warp);
@@ -595,8 +645,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // K_res and Aqk are final: their images go to the record as they are (thread 0 waits for
     // these copies to have read K_res before the K_res space is reused for staging)
     if (tid == 0) {
-        bulk_s2g(rec + kRecKR, sb + S::KI0, 8192);
-        bulk_s2g(rec + kRecKR + 8192, sb + S::KI1, 8192);
+        bulk_s2g(rec + kRecUB, sb + S::KI0, 8192);
+        bulk_s2g(rec + kRecUB + 8192, sb + S::KI1, 8192);
         bulk_s2g(rec + kRecAQ, sb + S::AQK, 8192);
     }
 
@@ -735,7 +785,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             *reinterpret_cast<uint4*>(slot + sw128_off(lane, cb)) = pack_bf16x8(&d[8 * cb]);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) bulk_s2g(rec + kRecM0 + wh * 16384 + wq * 4096, smem_u32(slot), 4096);
+        if (lane == 0) bulk_s2g(rec + kRecSB + wh * kRecSBHalf + wq * 4096, smem_u32(slot), 4096);
     }
     KDA_TRACE_POINT(ptr_, 8192 + 6);
     if (wq < 2) {
@@ -764,7 +814,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 *reinterpret_cast<uint4*>(slot + sw128_off(lane, cb)) = pack_bf16x8(&d[8 * cb]);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) bulk_s2g(rec + kRecP0 + wh * 8192 + wq * 4096, smem_u32(slot), 4096);
+            if (lane == 0) bulk_s2g(rec + kRecSB + wh * kRecSBHalf + kRecP + wq * 4096, smem_u32(slot), 4096);
         }
     }
 done:
@@ -785,47 +835,56 @@ done:
     }
 }
 
+}  // namespace tc
+}  // namespace kda
+
+#include "kda_prep_strong.cuh"
+
+namespace kda {
+namespace tc {
+
 // ------------------------------------------------------------------ chunk recurrence + outputs
-// One CTA per (sequence, head, NV value channels), NV = 32 or 64.  Per chunk, two tensor-core
-// products read the same bf16 image of S_in and this slice of U:
-//   D_S = [M | K_res^T] [S_in ; U]   (128 x NV, K = 128 + 64)  -> S_out = gamma S_in + D_S
-//   D_O = [P | Aqk]     [S_in ; U]   ( 64 x NV, K = 128 + 64)  -> O = D_O
-// so the state warps only scale, add and convert; the chain is D_S -> state update -> the
-// next S_in image -> the next D_S.  Narrow slices shorten each chain step (half the columns
-// per thread, half the product) at the price of loading P, M, K_res and Aqk once per slice:
-// the launch takes NV = 32 while four CTAs per (sequence, head) still fit on the SMs at once.
-// warps 0-7: state (warp w: rows 32 (w % 4) .. +31 = its TMEM lanes, columns NV/2 (w / 4) ..
-// of the slice), then this chunk's output rows 16 (w % 4) .. +15 (the M = 64 accumulator
-// puts row r in lane 32 (r / 16) + r % 16); warp 8: loader (2 stages of P, M, K_res, the U
-// slice and Aqk); warp 9: issuer of D_S; warp 10: issuer of D_O.  The two issuers are
-// separate threads, so that the output product never holds back the chain's.
+// One CTA per (sequence, head, NV = 32 or 64 value channels).  Per chunk, two tensor-core
+// product streams read the same bf16 image of S_in's slice and the slice of U:
+//   D_S = K_res^T U + M S_in     (128 x NV, K = 64 + 128)  -> S_out = gamma S_in + D_S
+//   D_O = Aqk U + P S_in         ( 64 x NV, K = 64 + 128)  -> O = D_O
+// The U terms do not depend on S_in: they are issued into the (double-buffered) accumulators
+// before the state of the chunk is ready, so the serial chain is S image -> M S_in (8 MMAs)
+// -> drain and update -> next image.  Narrow slices (small N) keep each instruction of the
+// chain cheap; the launch takes NV = 32 while four CTAs per (sequence, head) fit on the SMs
+// at once, else 64.
+//   warps 0-7: state (warp w: key rows 32 (w % 4) .. +31 = its TMEM lanes, columns NV/2 (w / 4)
+//   .. of the slice), then this chunk's output rows 16 (w % 4) .. +15 (the M = 64 accumulator
+//   puts row r in lane 32 (r / 16) + r % 16); warp 8: loader (2 stages); warp 9: issuer of D_S;
+//   warp 10: issuer of D_O.  The two issuers are separate threads, so that the output product
+//   never holds back the chain's.
 constexpr int kRecThreads = 352;
-constexpr int kRecComputeWarps = 8;
-constexpr int kLoaderWarp = 8, kIssuerWarp = 9, kIssuerOWarp = 10;
+constexpr int kRecStateWarps = 8;
+constexpr int kRecLoaderWarp = 8, kIssuerWarp = 9, kIssuerOWarp = 10;
 constexpr int kStages = 2, kPrefetchAhead = 4;
 constexpr uint32_t kUSlice = 4096;    // one 32-column U slice: 64 token rows of 64 B
+constexpr uint32_t kRecHead = kRecU;  // [M ; P], K_res and Aqk: the record's first 72 KB
 
 template <int NV_>
 struct RecCfg {
     static constexpr int NV = NV_, NSL = D / NV, NC = NV / 2;   // NC: columns per thread
-    // stage: the record's first 64 KB (P, M, K_res) as they are, then the U slices and Aqk
-    static constexpr uint32_t kStP = 0, kStM = 16384, kStKR = 49152, kStU = 65536;
+    // stage: [M ; P], K_res and Aqk as stored, then this CTA's U slice
+    static constexpr uint32_t kStU = kRecHead;
     static constexpr uint32_t kUBytes = (NV / 32) * kUSlice;
-    static constexpr uint32_t kStAQ = kStU + kUBytes;
-    static constexpr uint32_t kStageBytes = kStAQ + 8192;
+    static constexpr uint32_t kStageBytes = kStU + kUBytes;
     // S image (MN-major B operand): 128 key rows of 2 NV bytes, 128- or 64-byte swizzle
     static constexpr uint32_t kSRow = 2 * NV, kSImg = 128 * kSRow, kSSbo = 8 * kSRow;
     static constexpr uint32_t kSSwz = NV == 64 ? kSwizzle128 : kSwizzle64;
     static constexpr uint32_t SB = kStages * kStageBytes;   // S images, 2 buffers
     static constexpr uint32_t OST = SB + 2 * kSImg;          // output staging [64 rows][2 NV B]
-    // full[2] empty[2] mma_s mma_o[2] ofree[2] sbr[2]
+    // full[2] empty[2] mma_s[2] mma_o[2] ofree[2] sbr[2] sdrain[2] fin[2]
     static constexpr uint32_t BAR = OST + 64 * kSRow;
-    static constexpr uint32_t TMEM = BAR + 11 * 8;
+    static constexpr uint32_t TMEM = BAR + 16 * 8;
     static constexpr uint32_t FLAG = TMEM + 4;
     static constexpr uint32_t BYTES = FLAG + 4 + 1024;
-    // D_S [0, NV), D_O buffers [NV, 2 NV), [2 NV, 3 NV)
-    static constexpr uint32_t kTmemCols = NV == 64 ? 256 : 128;
-    static_assert(kStAQ % 1024 == 0 && kStageBytes % 1024 == 0, "stage images must stay 1 KB aligned");
+    // D_S buffers [0, NV), [NV, 2 NV); D_O buffers [2 NV, 3 NV), [3 NV, 4 NV)
+    static constexpr uint32_t kTmemCols = 4 * NV;
+    static_assert(kStageBytes % 1024 == 0, "stage images must stay 1 KB aligned");
     static_assert(BYTES <= 232448, "recurrence shared memory exceeds 227 KB");
     // byte offset of 16-byte chunk `ch` of row `row` in an S image / the output staging
     __device__ static __forceinline__ uint32_t s_off(uint32_t row, uint32_t ch) {
@@ -834,18 +893,74 @@ struct RecCfg {
     }
 };
 
+// Loader of the recurrence kernels (one thread): every chunk's record (the first head_bytes
+// as stored, then `tail_bytes` from tail_off) into stage kk % 2 once the products of chunk
+// kk - 2 have released it; the records a few chunks ahead go to L2 first.  Never leaves with
+// copies in flight.
+template <typename RecordAt>
+__device__ __forceinline__ void load_record_stages(uint32_t sb, uint32_t stage_bytes, uint32_t full0,
+                                                   uint32_t empty0, int nchunks, volatile int* abort_flag,
+                                                   RecordAt record, uint32_t head_bytes, uint32_t tail_off,
+                                                   uint32_t tail_bytes) {
+    auto prefetch = [&](int kk) {
+        bulk_prefetch_l2(record(kk), head_bytes);
+        if (tail_bytes) bulk_prefetch_l2(record(kk) + tail_off, tail_bytes);
+    };
+    for (int kk = 0; kk < nchunks && kk < kPrefetchAhead; ++kk) prefetch(kk);
+    int issued = 0;
+    for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
+        const int st = kk % kStages, use = kk / kStages;
+        if (use > 0 && !mbar_wait(empty0 + 8 * st, (use - 1) & 1)) {
+            kda_set_status(KDA_ERR_TIMEOUT);
+            *abort_flag = 1;
+            break;
+        }
+        const uint32_t fb = full0 + 8 * st, dst = sb + st * stage_bytes;
+        mbar_arrive_expect_tx(fb, head_bytes + tail_bytes);
+        bulk_g2s(dst, record(kk), head_bytes, fb);
+        if (tail_bytes) bulk_g2s(dst + head_bytes, record(kk) + tail_off, tail_bytes, fb);
+        if (kk + kPrefetchAhead < nchunks) prefetch(kk + kPrefetchAhead);
+        ++issued;
+    }
+    for (int kk = max(0, issued - kStages); kk < issued; ++kk)
+        mbar_wait(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
+}
+
+// Segments of the chunk-parallel scan (seg_tab non-null): CTA (segment s, head h, slice) runs
+// the segment's chunks from S_in(s) (the initial state for a sequence's first segment) and
+// writes the final state only from the sequence's last segment.
 template <int NV>
 __global__ void __launch_bounds__(kRecThreads, 1)
 rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __restrict__ tab,
            const uint8_t* __restrict__ records, const float* initial_state, float* final_state,
-           __nv_bfloat16* __restrict__ out, const int32_t* __restrict__ etab, float* emit_states) {
+           __nv_bfloat16* __restrict__ out, const int32_t* __restrict__ etab, float* emit_states,
+           const int4* __restrict__ seg_tab, const int32_t* __restrict__ seg_count,
+           const float* __restrict__ seg_states) {
     using S = RecCfg<NV>;
     constexpr int NSL = S::NSL;
+    (void)num_seqs;
     const int sl = blockIdx.x % NSL;
     const int h = (blockIdx.x / NSL) % H;
-    const int n = blockIdx.x / (NSL * H);
-    const int c_begin = off[n], nchunks = off[n + 1] - c_begin;
-    (void)num_seqs;
+    const int unit = blockIdx.x / (NSL * H);   // sequence, or scan segment
+    int n, c_begin, nchunks;
+    bool write_final = final_state != nullptr;
+    const float* s_init;
+    if (seg_tab) {
+        if (unit >= *seg_count) return;   // the whole CTA, before any barrier
+        const int4 sg = seg_tab[unit];    // (sequence, first chunk, chunks, index | last << 16)
+        n = sg.x;
+        c_begin = sg.y;
+        nchunks = sg.z;
+        write_final = write_final && (sg.w >> 16) != 0;
+        s_init = (sg.w & 0xFFFF) == 0
+                     ? (initial_state ? initial_state + ((size_t)n * H + h) * D * D : nullptr)
+                     : seg_states + ((size_t)unit * H + h) * (kSegStateBytes / sizeof(float)) + 2 * D * D;
+    } else {
+        n = unit;
+        c_begin = off[n];
+        nchunks = off[n + 1] - c_begin;
+        s_init = initial_state ? initial_state + ((size_t)n * H + h) * D * D : nullptr;
+    }
     auto record = [&](int kk) { return records + ((size_t)(c_begin + kk) * H + h) * kRecBytes; };
 
     extern __shared__ uint8_t smem_raw[];
@@ -853,8 +968,8 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
     const uint32_t sb = smem_u32(sm);
     // Each barrier's waiters can never fall two phases behind: its next phase needs an
     // arrival that every waiter of the current phase precedes.
-    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 16, mma_s = full0 + 32, mma_o = full0 + 40;
-    const uint32_t ofree = full0 + 56, sbr0 = full0 + 72;
+    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 16, mma_s = full0 + 32, mma_o = full0 + 48;
+    const uint32_t ofree = full0 + 64, sbr0 = full0 + 80, sdrain = full0 + 96, fin = full0 + 112;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + S::FLAG);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -863,11 +978,13 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
         for (int b2 = 0; b2 < 2; ++b2) {
             mbar_init(full0 + 8 * b2, 1);
             mbar_init(empty0 + 8 * b2, 2);    // tcgen05.commit of both products that read it
+            mbar_init(mma_s + 8 * b2, 1);
             mbar_init(mma_o + 8 * b2, 1);
-            mbar_init(ofree + 8 * b2, kRecComputeWarps);
-            mbar_init(sbr0 + 8 * b2, kRecComputeWarps);
+            mbar_init(ofree + 8 * b2, kRecStateWarps);
+            mbar_init(sbr0 + 8 * b2, kRecStateWarps);
+            mbar_init(sdrain + 8 * b2, kRecStateWarps);
+            mbar_init(fin + 8 * b2, 1);
         }
-        mbar_init(mma_s, 1);
         fence_mbar_init();
         *abort_flag = 0;
     }
@@ -876,103 +993,78 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
     tc_fence_after();
     const uint32_t tS = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
 
-    if (warp == kLoaderWarp) {
-        // ---------------- loader ------------------------------------------------------------
-        if (lane == 0) {
-            // everything this CTA reads of a record goes to L2 kPrefetchAhead chunks early
-            auto prefetch = [&](int kk) {
-                const uint8_t* rec = record(kk);
-                bulk_prefetch_l2(rec, 65536);
-                bulk_prefetch_l2(rec + kRecU + sl * S::kUBytes, S::kUBytes);
-                bulk_prefetch_l2(rec + kRecAQ, 8192 + 512);
-            };
-            for (int kk = 0; kk < nchunks && kk < kPrefetchAhead; ++kk) prefetch(kk);
-            int issued = 0;
-            for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
-                const int st = kk % kStages, use = kk / kStages;
-                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 0);
-                if (use > 0 && !mbar_wait(empty0 + 8 * st, (use - 1) & 1)) {
-                    kda_set_status(KDA_ERR_TIMEOUT);
-                    *abort_flag = 1;
-                    break;
-                }
-                const uint8_t* rec = record(kk);
-                const uint32_t dst = sb + st * S::kStageBytes, fb = full0 + 8 * st;
-                mbar_arrive_expect_tx(fb, S::kStageBytes);
-#pragma unroll
-                for (int part = 0; part < 4; ++part)   // P, M, K_res: the record's first 64 KB
-                    bulk_g2s(dst + part * 16384, rec + part * 16384, 16384, fb);
-                bulk_g2s(dst + S::kStU, rec + kRecU + sl * S::kUBytes, S::kUBytes, fb);
-                bulk_g2s(dst + S::kStAQ, rec + kRecAQ, 8192, fb);
-                if (kk + kPrefetchAhead < nchunks) prefetch(kk + kPrefetchAhead);
-                KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 1);
-                ++issued;
-            }
-            // never leave with copies in flight: wait (bounded) for the last stages filled
-            for (int kk = max(0, issued - kStages); kk < issued; ++kk)
-                mbar_wait(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
-        }
+    if (warp == kRecLoaderWarp) {
+        if (lane == 0)
+            load_record_stages(sb, S::kStageBytes, full0, empty0, nchunks, abort_flag, record, kRecHead,
+                               kRecU + sl * S::kUBytes, S::kUBytes);
     } else if (warp == kIssuerWarp || warp == kIssuerOWarp) {
-        // ---------------- issuers: D_S (warp 9) and D_O into buffer kk % 2 (warp 10) -------
-        // D_O(kk) also waits until the output rows of chunk kk - 2 have left its buffer.  The
-        // image of S_in stays put until D_O is done: the state warps overwrite it only after
-        // they have drained D_O.
+        // ---------------- issuers: D_S (warp 9) and D_O (warp 10) into buffer kk % 2 ----------
+        // The U term first (its buffer drained by chunk kk - 2), then, once the image of S_in is
+        // in, the S term.  The image of S_in stays put until both products of the chunk are
+        // done: the state warps overwrite it only after they have drained D_O.
         if (lane == 0) {
             const bool is_s = warp == kIssuerWarp;
-            constexpr uint32_t idS = idesc_bf16(128, NV, false, true);
-            constexpr uint32_t idSx = idesc_bf16(128, NV, true, true);    // A = K_res^T (MN-major)
-            constexpr uint32_t idO = idesc_bf16(64, NV, false, true);
+            constexpr uint32_t idSU = idesc_bf16(128, NV, true, true);     // K_res^T (MN-major) U (MN-major)
+            constexpr uint32_t idSS = idesc_bf16(128, NV, false, true);    // M (K-major) S (MN-major)
+            constexpr uint32_t idOU = idesc_bf16(64, NV, false, true);     // Aqk (K-major) U
+            constexpr uint32_t idOS = idesc_bf16(64, NV, false, true);     // P (K-major) S
+            bool ok = true;
             for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
-                const int st = kk % kStages, so = kk & 1;
-                const uint32_t sbuf = sb + S::SB + (kk & 1) * S::kSImg;
+                const int st = kk % kStages, b = kk & 1, use = kk >> 1;
+                const uint32_t stage = sb + st * S::kStageBytes;
+                const uint32_t sbuf = sb + S::SB + b * S::kSImg;
+                const uint32_t tD = tS + (is_s ? 0u : 2u * NV) + NV * b;
                 if (!mbar_wait(full0 + 8 * st, (kk / kStages) & 1) ||
-                    !mbar_wait(sbr0 + 8 * (kk & 1), (kk >> 1) & 1) ||
-                    (!is_s && kk >= 2 && !mbar_wait(ofree + 8 * so, ((kk - 2) >> 1) & 1))) {
-                    kda_set_status(KDA_ERR_TIMEOUT);
-                    *abort_flag = 1;
+                    (use > 0 && !mbar_wait((is_s ? sdrain : ofree) + 8 * b, (use - 1) & 1))) {
+                    ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t stage = sb + st * S::kStageBytes;
-                if (is_s) {
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks)
-                        umma_bf16(tS, smem_desc(stage + S::kStM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128),
-                                  smem_desc(sbuf + ks * 2 * S::kSSbo, 16, S::kSSbo, S::kSSwz), idS, ks > 0);
-#pragma unroll
-                    for (int ks = 0; ks < C / 16; ++ks)
-                        umma_bf16(tS, smem_desc(stage + S::kStKR + ks * 2048, 8192, 1024, kSwizzle128),
-                                  smem_desc(stage + S::kStU + ks * 1024, kUSlice, 512, kSwizzle64), idSx, 1);
-                    umma_commit(mma_s);
-                    KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 2);
-                } else {
-                    const uint32_t tO = tS + NV + NV * so;
-#pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks)
-                        umma_bf16(tO, smem_desc(stage + S::kStP + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128),
-                                  smem_desc(sbuf + ks * 2 * S::kSSbo, 16, S::kSSbo, S::kSSwz), idO, ks > 0);
-#pragma unroll
-                    for (int ks = 0; ks < C / 16; ++ks)
-                        umma_bf16(tO, smem_desc(stage + S::kStAQ + ks * 32, 16, 1024, kSwizzle128),
-                                  smem_desc(stage + S::kStU + ks * 1024, kUSlice, 512, kSwizzle64), idO, 1);
-                    umma_commit(mma_o + 8 * so);
-                    KDA_TRACE_POINT(blockIdx.x == 0 && kk < 256, 4096 + kk * 4 + 3);
+                for (int ks = 0; ks < C / 16; ++ks) {
+                    const uint64_t bu = smem_desc(stage + S::kStU + ks * 1024, kUSlice, 512, kSwizzle64);
+                    if (is_s)
+                        umma_bf16(tD, smem_desc(stage + kRecUB + ks * 2048, 8192, 1024, kSwizzle128), bu, idSU, ks > 0);
+                    else
+                        umma_bf16(tD, smem_desc(stage + kRecAQ + ks * 32, 16, 1024, kSwizzle128), bu, idOU, ks > 0);
                 }
+                if (!mbar_wait(sbr0 + 8 * b, use & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (is_s) KDA_TRACE_POINT(blockIdx.x == 0 && kk < 512, 16 * kk + 8);
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t bs = smem_desc(sbuf + ks * 2 * S::kSSbo, 16, S::kSSbo, S::kSSwz);
+                    const uint32_t a = stage + kRecSB + (ks >> 2) * kRecSBHalf + (ks & 3) * 32 + (is_s ? 0u : kRecP);
+                    umma_bf16(tD, smem_desc(a, 16, 1024, kSwizzle128), bs, is_s ? idSS : idOS, 1);
+                }
+                umma_commit((is_s ? mma_s : mma_o) + 8 * b);
                 umma_commit(empty0 + 8 * st);
+                if (is_s) KDA_TRACE_POINT(blockIdx.x == 0 && kk < 512, 16 * kk + 9);
             }
+            if (!ok) {
+                kda_set_status(KDA_ERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            // nothing may still run on the tensor pipe when Tensor Memory is released
+            const uint32_t fb = fin + 8 * (is_s ? 0 : 1);
+            umma_commit(fb);
+            mbar_wait(fb, 0);
         }
-    } else if (warp < kRecComputeWarps) {
+    } else {
         // ---------------- state: row i, columns NC cw .. NC cw + NC - 1 of the slice -------
         constexpr int NC = S::NC;
         const int q4 = warp & 3, i = 32 * q4 + lane, cw = warp >> 2;
         const uint32_t taw = (uint32_t)(32 * q4) << 16;
-        const size_t sbase = (((size_t)n * H + h) * D + i) * D + (size_t)sl * NV + NC * cw;
+        const size_t col0 = (size_t)sl * NV + NC * cw;
         const int r_out = 16 * q4 + lane;   // output row of this lane (lanes 0-15)
         float Sr[NC];
-        if (initial_state) {
+        if (s_init) {
 #pragma unroll
             for (int j4 = 0; j4 < NC / 4; ++j4) {
-                const float4 t = reinterpret_cast<const float4*>(initial_state + sbase)[j4];
+                const float4 t = reinterpret_cast<const float4*>(s_init + (size_t)i * D + col0)[j4];
                 Sr[4 * j4] = t.x; Sr[4 * j4 + 1] = t.y; Sr[4 * j4 + 2] = t.z; Sr[4 * j4 + 3] = t.w;
             }
         } else {
@@ -980,76 +1072,77 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
             for (int j = 0; j < NC; ++j) Sr[j] = 0.f;
         }
         // bf16 image of the state entering the next chunk (B operand of both products)
-        auto put_state = [&](uint32_t buf) {
+        auto put_state = [&](int b) {
 #pragma unroll
             for (int cb = 0; cb < NC / 8; ++cb)
-                *reinterpret_cast<uint4*>(sm + buf + S::s_off(i, (NC / 8) * cw + cb)) = pack_bf16x8(&Sr[8 * cb]);
+                *reinterpret_cast<uint4*>(sm + S::SB + b * S::kSImg + S::s_off(i, (NC / 8) * cw + cb)) =
+                    pack_bf16x8(&Sr[8 * cb]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sbr0 + 8 * b);
         };
-        // gamma of row i and the (first token, rows) of a chunk, loaded one chunk ahead
-        float gam = 0.f;
-        int2 ce = make_int2(0, 0);
+        // gamma of row i, the (first token, rows) and the emission slot of a chunk, loaded a
+        // chunk ahead so that their global-load latency stays off the chain
+        float gam_next = 0.f;
+        int2 ce_next = make_int2(0, 0);
+        int e_next = -1;
         if (nchunks > 0) {
-            gam = __ldg(reinterpret_cast<const float*>(record(0) + kRecGamma) + i);
-            ce = tab[c_begin];
-            put_state(S::SB);
+            gam_next = __ldg(reinterpret_cast<const float*>(record(0) + kRecGamma) + i);
+            ce_next = tab[c_begin];
+            if (etab) e_next = etab[c_begin];
+            put_state(0);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sbr0);
-
         bool ok = true;
         for (int kk = 0; kk < nchunks; ++kk) {
-            const int so = kk & 1;
+            const int b = kk & 1, use = kk >> 1;
             const bool more = kk + 1 < nchunks;
-            const bool tr = blockIdx.x == 0 && tid == 0 && kk < 256;
+            const float gam = gam_next;
+            const int2 ce = ce_next;
+            const int e_slot = e_next;
+            if (more) {
+                gam_next = __ldg(reinterpret_cast<const float*>(record(kk + 1) + kRecGamma) + i);
+                ce_next = tab[c_begin + kk + 1];
+                if (etab) e_next = etab[c_begin + kk + 1];
+            }
+            const bool tr = blockIdx.x == 0 && tid == 0 && kk < 512;
             (void)tr;
-            KDA_TRACE_POINT(tr, kk * 8 + 0);
-            ok = __all_sync(0xffffffffu, mbar_wait(mma_s, kk & 1));
+            KDA_TRACE_POINT(tr, 16 * kk + 0);
+            ok = __all_sync(0xffffffffu, mbar_wait(mma_s + 8 * b, use & 1));
             if (!ok || *abort_flag) { ok = false; break; }
-            KDA_TRACE_POINT(tr, kk * 8 + 3);
+            KDA_TRACE_POINT(tr, 16 * kk + 1);
             tc_fence_after();
             {
                 float dsv[NC];
-                tmem_ld_cols(tS + taw + NC * cw, dsv);
+                tmem_ld_cols(tS + taw + NV * b + NC * cw, dsv);
                 tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sdrain + 8 * b);
 #pragma unroll
                 for (int j = 0; j < NC; ++j) Sr[j] = fmaf(gam, Sr[j], dsv[j]);
             }
-            KDA_TRACE_POINT(tr, kk * 8 + 4);
-            if (etab) {   // emission boundary at the end of this chunk: the fp32 state as it is
-                const int e = etab[c_begin + kk];
-                if (e >= 0) {
-                    float* dst = emit_states + ((((size_t)e * H + h) * D + i) * D + (size_t)sl * NV + NC * cw);
-#pragma unroll
-                    for (int j4 = 0; j4 < NC / 4; ++j4)
-                        reinterpret_cast<float4*>(dst)[j4] =
-                            make_float4(Sr[4 * j4], Sr[4 * j4 + 1], Sr[4 * j4 + 2], Sr[4 * j4 + 3]);
-                }
-            }
+            KDA_TRACE_POINT(tr, 16 * kk + 2);
             // the image of S_{kk+1} replaces that of S_{kk-1}, whose products (D_S(kk-1), and
             // D_O(kk-1), drained below in the previous pass) are complete
-            if (more) put_state(S::SB + ((kk + 1) & 1) * S::kSImg);
-            tc_fence_before();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sbr0 + 8 * ((kk + 1) & 1));
-            const int t0 = ce.x, nrow = ce.y;
-            if (more) {
-                gam = __ldg(reinterpret_cast<const float*>(record(kk + 1) + kRecGamma) + i);
-                ce = tab[c_begin + kk + 1];
+            if (more) put_state((kk + 1) & 1);
+            KDA_TRACE_POINT(tr, 16 * kk + 4);
+            if (e_slot >= 0) {   // emission boundary at the end of this chunk: the fp32 state as it is
+                float* dst = emit_states + ((size_t)e_slot * H + h) * D * D + (size_t)i * D + col0;
+#pragma unroll
+                for (int j4 = 0; j4 < NC / 4; ++j4)
+                    reinterpret_cast<float4*>(dst)[j4] =
+                        make_float4(Sr[4 * j4], Sr[4 * j4 + 1], Sr[4 * j4 + 2], Sr[4 * j4 + 3]);
             }
-            KDA_TRACE_POINT(tr, kk * 8 + 5);
             // output rows 16 q4 .. 16 q4 + 15, columns NC cw .. of the slice
-            ok = __all_sync(0xffffffffu, mbar_wait(mma_o + 8 * so, (kk >> 1) & 1));
+            ok = __all_sync(0xffffffffu, mbar_wait(mma_o + 8 * b, use & 1));
             if (!ok) break;
-            KDA_TRACE_POINT(tr, kk * 8 + 7);
             tc_fence_after();
             float dov[NC];
-            tmem_ld_cols(tS + taw + NV + NV * so + NC * cw, dov);
+            tmem_ld_cols(tS + taw + 2 * NV + NV * b + NC * cw, dov);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(ofree + 8 * so);
+            if (lane == 0) mbar_arrive(ofree + 8 * b);
             // lane l (< 16) holds row 16 q4 + l: stage the bf16 rows, then re-read them so that
             // NC / 8 lanes store one row's 2 NC contiguous bytes
             uint8_t* os = sm + S::OST;
@@ -1069,21 +1162,22 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
 #pragma unroll
                 for (int g = 0; g < 16 / RPI; ++g) {
                     const int rr = 16 * q4 + RPI * g + lane / LPR;
-                    if (rr < nrow)
-                        *reinterpret_cast<uint4*>(out + ((size_t)(t0 + rr) * H + h) * D + sl * NV + NC * cw +
+                    if (rr < ce.y)
+                        *reinterpret_cast<uint4*>(out + ((size_t)(ce.x + rr) * H + h) * D + sl * NV + NC * cw +
                                                   8 * (lane % LPR)) = ov[g];
                 }
             }
             __syncwarp();   // the staging rows are rewritten by the next chunk
-            KDA_TRACE_POINT(tr, kk * 8 + 6);
+            KDA_TRACE_POINT(tr, 16 * kk + 7);
         }
         if (!ok) {
             if (lane == 0) kda_set_status(KDA_ERR_TIMEOUT);
             *abort_flag = 1;
-        } else if (final_state) {
+        } else if (write_final) {
+            float* dst = final_state + ((size_t)n * H + h) * D * D + (size_t)i * D + col0;
 #pragma unroll
             for (int j4 = 0; j4 < NC / 4; ++j4)
-                reinterpret_cast<float4*>(final_state + sbase)[j4] =
+                reinterpret_cast<float4*>(dst)[j4] =
                     make_float4(Sr[4 * j4], Sr[4 * j4 + 1], Sr[4 * j4 + 2], Sr[4 * j4 + 3]);
         }
     }
@@ -1092,6 +1186,293 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tS, S::kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ chunk-parallel scan
+// Scan segments from the chunk offsets: sequence n gets max(1, ceil(chunks_n / seg))
+// segments (an empty sequence one segment without chunks, so that its final state is still
+// written); seg_tab[s] = (n, first chunk, chunks, index | last << 16), seg_off[n] the first
+// segment of sequence n, *seg_count the total.  Single CTA of 1024 threads.
+__global__ void __launch_bounds__(1024)
+segment_index_kernel(int num_seqs, const int32_t* __restrict__ off, int seg,
+                     int32_t* __restrict__ seg_off, int32_t* __restrict__ seg_count,
+                     int4* __restrict__ seg_tab) {
+    __shared__ int32_t warp_tot[32];
+    __shared__ int32_t carry;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < num_seqs; base += 1024) {
+        const int n = base + tid;
+        const int cnt = n < num_seqs ? max(1, (off[n + 1] - off[n] + seg - 1) / seg) : 0;
+        int x = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_tot[w] = x;
+        __syncthreads();
+        if (w == 0) {
+            int t = warp_tot[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, t, o);
+                if (lane >= o) t += y;
+            }
+            warp_tot[lane] = t;
+        }
+        __syncthreads();
+        if (n < num_seqs) seg_off[n] = carry + (w > 0 ? warp_tot[w - 1] : 0) + x - cnt;
+        __syncthreads();
+        if (tid == 0) carry += warp_tot[31];
+        __syncthreads();
+    }
+    if (tid == 0) {
+        seg_off[num_seqs] = carry;
+        *seg_count = carry;
+    }
+    __syncthreads();
+    for (int sgi = tid; sgi < carry; sgi += 1024) {
+        const int n = find_seq(seg_off, num_seqs, sgi);
+        const int p = sgi - seg_off[n], last = seg_off[n + 1] - 1 == sgi;
+        const int chunks = off[n + 1] - off[n];
+        seg_tab[sgi] = make_int4(n, off[n] + p * seg, max(0, min(seg, chunks - p * seg)), p | (last << 16));
+    }
+}
+
+// Pass 1 of the chunk-parallel scan: CTA (segment s, head h), for every segment but the last
+// of its sequence, runs the segment's chunks from a zero state (S_local) and composes the
+// segment's transition T = prod (diag(gamma) + M) beside it; both go to the segment states.
+// In the transposed form of rec_kernel, X = T^T evolves like S^T without the U term,
+//   X <- X diag(gamma) + X M^T  from X = I,
+// so the chain step is two products with the same B operand (M, the first 128 rows of the
+// record's [M ; P]).  warps 0-7: S^T and X (rows j = 32 (w % 4) + lane, columns 64 (w / 4) ..),
+// warp 8: loader, warp 9: issuer.  Tensor Memory: D_S [0, 128), D_X [128, 256), S^T images
+// [256, 320) [320, 384), X images [384, 448) [448, 512).
+constexpr int kSegThreads = 320, kSegStateWarps = 8, kSegLoaderWarp = 8, kSegIssuerWarp = 9;
+struct SegSmem {
+    static constexpr uint32_t kStage = (kRecBytes + 1023) / 1024 * 1024;   // one record, as stored
+    // full[2] empty[2] mma sready[2] sdrain fin
+    static constexpr uint32_t BAR = kStages * kStage;
+    static constexpr uint32_t TMEM = BAR + 16 * 8;
+    static constexpr uint32_t FLAG = TMEM + 4;
+    static constexpr uint32_t BYTES = FLAG + 4 + 1024;
+    static_assert(BYTES <= 232448, "scan shared memory exceeds 227 KB");
+};
+constexpr uint32_t kSegTmemCols = 512;
+// operand descriptors of the transposed products, K step ks: [M ; P] (K-major B), K_res
+// (MN-major B) and U^T (MN-major A, four 32-column atoms)
+__device__ __forceinline__ uint64_t seg_m_desc(uint32_t stage, int ks) {
+    return smem_desc(stage + kRecSB + (ks >> 2) * kRecSBHalf + (ks & 3) * 32, 16, 1024, kSwizzle128);
+}
+__device__ __forceinline__ uint64_t seg_kres_desc(uint32_t stage, int ks) {
+    return smem_desc(stage + kRecUB + ks * 2048, 8192, 1024, kSwizzle128);
+}
+__device__ __forceinline__ uint64_t seg_u_desc(uint32_t stage, int ks) {
+    return smem_desc(stage + kRecU + ks * 1024, kUSlice, 512, kSwizzle64);
+}
+__global__ void __launch_bounds__(kSegThreads, 1)
+seg_kernel(int H, const uint8_t* __restrict__ records, const int4* __restrict__ seg_tab,
+           const int32_t* __restrict__ seg_count, float* __restrict__ seg_states) {
+    using S = SegSmem;
+    const int h = blockIdx.x % H, sgi = blockIdx.x / H;
+    if (sgi >= *seg_count) return;   // the whole CTA, before any barrier
+    const int4 sg = seg_tab[sgi];
+    if ((sg.w >> 16) != 0) return;   // a sequence's last segment needs no transition
+    const int c_begin = sg.y, nchunks = sg.z;
+    auto record = [&](int kk) { return records + ((size_t)(c_begin + kk) * H + h) * kRecBytes; };
+    constexpr uint32_t kDX = 128, kSTi = 256, kXTi = 384;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+    const uint32_t sb = smem_u32(sm);
+    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 16, mmas = full0 + 32, sready0 = full0 + 64;
+    const uint32_t sdrain = full0 + 80, finbar = full0 + 112;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + S::FLAG);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (warp == 0) tmem_alloc(sb + S::TMEM, kSegTmemCols);
+    if (tid == 0) {
+        for (int b2 = 0; b2 < 2; ++b2) {
+            mbar_init(full0 + 8 * b2, 1);
+            mbar_init(empty0 + 8 * b2, 1 + kSegStateWarps);
+            mbar_init(sready0 + 8 * b2, kSegStateWarps);
+        }
+        mbar_init(mmas, 1);
+        mbar_init(sdrain, kSegStateWarps);
+        mbar_init(finbar, 1);
+        fence_mbar_init();
+        *abort_flag = 0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *reinterpret_cast<volatile uint32_t*>(sm + S::TMEM);
+
+    if (warp == kSegLoaderWarp) {
+        if (lane == 0)
+            load_record_stages(sb, S::kStage, full0, empty0, nchunks, abort_flag, record, kRecU, kRecU,
+                               kRecBytes - kRecU);
+    } else if (warp == kSegIssuerWarp) {
+        if (lane == 0) {
+            constexpr uint32_t idSU = idesc_bf16(128, 128, true, true);    // U^T (MN-major) K_res (MN-major)
+            constexpr uint32_t idSS = idesc_bf16(128, 128, false, false);  // S^T / X (TMEM) M (K-major)
+            bool ok = true;
+            for (int kk = 0; kk < nchunks && !*abort_flag; ++kk) {
+                const int st = kk % kStages, b = kk & 1;
+                const uint32_t stage = sb + st * S::kStage;
+                // the record is in; D_S and D_X of chunk kk - 1 have been drained
+                if (!mbar_wait(full0 + 8 * st, (kk / kStages) & 1) ||
+                    (kk > 0 && !mbar_wait(sdrain, (kk - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks) umma_bf16(tm, seg_u_desc(stage, ks), seg_kres_desc(stage, ks), idSU, ks > 0);
+                if (!mbar_wait(sready0 + 8 * b, (kk >> 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t bm = seg_m_desc(stage, ks);
+                    umma_bf16_tmem_a(tm, tm + kSTi + 64 * b + 8 * ks, bm, idSS, 1);
+                    umma_bf16_tmem_a(tm + kDX, tm + kXTi + 64 * b + 8 * ks, bm, idSS, ks > 0);
+                }
+                umma_commit(mmas);
+                umma_commit(empty0 + 8 * st);
+            }
+            if (!ok) {
+                kda_set_status(KDA_ERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            umma_commit(finbar);
+            mbar_wait(finbar, 0);
+        }
+    } else {
+        const int q4 = warp & 3, j = 32 * q4 + lane, c = warp >> 2;
+        const uint32_t lanes = (uint32_t)(32 * q4) << 16;
+        float Sr[64], Xr[64];
+#pragma unroll
+        for (int u = 0; u < 64; ++u) {
+            Sr[u] = 0.f;
+            Xr[u] = (64 * c + u == j) ? 1.f : 0.f;
+        }
+        auto put = [&](int b) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t r[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) r[u] = pack_bf16x2(Sr[32 * hf + 2 * u], Sr[32 * hf + 2 * u + 1]);
+                tmem_st16(tm + lanes + kSTi + 64 * b + 32 * c + 16 * hf, r);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) r[u] = pack_bf16x2(Xr[32 * hf + 2 * u], Xr[32 * hf + 2 * u + 1]);
+                tmem_st16(tm + lanes + kXTi + 64 * b + 32 * c + 16 * hf, r);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sready0 + 8 * b);
+        };
+        if (nchunks > 0) put(0);
+        bool ok = true;
+        for (int kk = 0; kk < nchunks; ++kk) {
+            const int st = kk % kStages;
+            ok = __all_sync(0xffffffffu, mbar_wait(mmas, kk & 1));
+            if (!ok || *abort_flag) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float4* gam = reinterpret_cast<const float4*>(sm + st * S::kStage + kRecGamma) + 16 * c;
+            // x[16 q ..] = gamma x + D for one 16-column quarter of D_S (into Sr) or D_X (into Xr);
+            // quarters keep the live registers within the 168 a 320-thread CTA may use
+            auto update = [&](float(&x)[64], uint32_t dcol, int qt) {
+                float d[16];
+                tmem_ld16(tm + lanes + dcol + 64 * c + 16 * qt, d);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u4 = 0; u4 < 4; ++u4) {
+                    const float4 g4 = gam[4 * qt + u4];
+                    x[16 * qt + 4 * u4 + 0] = fmaf(g4.x, x[16 * qt + 4 * u4 + 0], d[4 * u4 + 0]);
+                    x[16 * qt + 4 * u4 + 1] = fmaf(g4.y, x[16 * qt + 4 * u4 + 1], d[4 * u4 + 1]);
+                    x[16 * qt + 4 * u4 + 2] = fmaf(g4.z, x[16 * qt + 4 * u4 + 2], d[4 * u4 + 2]);
+                    x[16 * qt + 4 * u4 + 3] = fmaf(g4.w, x[16 * qt + 4 * u4 + 3], d[4 * u4 + 3]);
+                }
+            };
+#pragma unroll
+            for (int qt = 0; qt < 4; ++qt) update(Sr, 0u, qt);
+#pragma unroll
+            for (int qt = 0; qt < 4; ++qt) update(Xr, kDX, qt);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(sdrain);
+                mbar_arrive(empty0 + 8 * st);   // gamma of this stage read
+            }
+            if (kk + 1 < nchunks) put((kk + 1) & 1);
+        }
+        if (!ok) {
+            if (lane == 0) kda_set_status(KDA_ERR_TIMEOUT);
+            *abort_flag = 1;
+        } else {
+            float* dst = seg_states + ((size_t)sgi * H + h) * (kSegStateBytes / sizeof(float));
+#pragma unroll
+            for (int u = 0; u < 64; ++u) {
+                dst[(size_t)(64 * c + u) * D + j] = Sr[u];            // S_local[i][j]
+                dst[D * D + (size_t)(64 * c + u) * D + j] = Xr[u];    // T[i][j] = X[j][i]
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, kSegTmemCols);
+    }
+}
+
+// The segments' starting states along each sequence, S_in(p+1) = T_p S_in(p) + S_local(p)
+// from S_in(0) = the initial state (or 0), in fp32 on CUDA cores; S_in(p) is stored for
+// p > 0.  One CTA of 512 threads per (sequence, head), S_in(p) in shared memory (64 KB).
+constexpr int kCombineThreads = 512;
+constexpr size_t kCombineSmem = sizeof(float) * D * D;
+__global__ void __launch_bounds__(kCombineThreads)
+combine_kernel(int H, const float* __restrict__ initial_state, const int32_t* __restrict__ seg_off,
+               float* __restrict__ seg_states) {
+    extern __shared__ __align__(16) float sS[];
+    const int h = blockIdx.x % H, n = blockIdx.x / H, tid = threadIdx.x;
+    const int s0 = seg_off[n], ns = seg_off[n + 1] - s0;
+    if (ns <= 1) return;
+    constexpr size_t kWords = kSegStateBytes / sizeof(float);
+    for (int e = tid; e < D * D; e += kCombineThreads)
+        sS[e] = initial_state ? initial_state[((size_t)n * H + h) * D * D + e] : 0.f;
+    __syncthreads();
+    // thread: row i = tid / 4, columns j = tid % 4 + 4 z (z < 32)
+    const int i = tid >> 2, j0 = tid & 3;
+    for (int p = 0; p + 1 < ns; ++p) {
+        const float* seg = seg_states + ((size_t)(s0 + p) * H + h) * kWords;
+        const float* Trow = seg + D * D + (size_t)i * D;
+        float acc[32];
+#pragma unroll
+        for (int z = 0; z < 32; ++z) acc[z] = seg[(size_t)i * D + j0 + 4 * z];   // S_local
+        for (int kx = 0; kx < D; ++kx) {
+            const float t = Trow[kx];
+#pragma unroll
+            for (int z = 0; z < 32; ++z) acc[z] = fmaf(t, sS[kx * D + j0 + 4 * z], acc[z]);
+        }
+        __syncthreads();   // every read of S_in(p) done
+        float* dst = seg_states + ((size_t)(s0 + p + 1) * H + h) * kWords + 2 * D * D;
+#pragma unroll
+        for (int z = 0; z < 32; ++z) {
+            sS[i * D + j0 + 4 * z] = acc[z];
+            dst[(size_t)i * D + j0 + 4 * z] = acc[z];
+        }
+        __syncthreads();
     }
 }
 
@@ -1132,13 +1513,34 @@ struct Workspace {
     int32_t* off;
     int2* tab;
     int32_t* etab;
+    int32_t* strong_count;
+    int2* strong_units;
+    int seg;                 // chunks per scan segment, 0 without segments
+    int64_t max_segs;
+    int32_t* seg_off;
+    int32_t* seg_count;
+    int4* seg_tab;
+    float* seg_states;
     uint8_t* records;
 };
-inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs) {
+inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs, int H) {
     uint8_t* base = static_cast<uint8_t*>(workspace);
-    return {reinterpret_cast<int32_t*>(base), reinterpret_cast<int2*>(base + ws_table_offset(num_seqs)),
-            reinterpret_cast<int32_t*>(base + ws_emit_offset(total, num_seqs)),
-            base + ws_records_offset(total, num_seqs)};
+    uint8_t* strong = base + ws_strong_offset(total, num_seqs);
+    Workspace w{reinterpret_cast<int32_t*>(base), reinterpret_cast<int2*>(base + ws_table_offset(num_seqs)),
+                reinterpret_cast<int32_t*>(base + ws_emit_offset(total, num_seqs)),
+                reinterpret_cast<int32_t*>(strong), reinterpret_cast<int2*>(strong + 16),
+                scan_segment_chunks(total, num_seqs, H), 0, nullptr, nullptr, nullptr, nullptr,
+                base + ws_records_offset(total, num_seqs, H)};
+    if (w.seg > 0) {
+        uint8_t* sc = base + ws_scan_offset(total, num_seqs, H);
+        w.max_segs = max_segments(total, num_seqs, w.seg);
+        w.seg_off = reinterpret_cast<int32_t*>(sc);
+        sc += align_up(sizeof(int32_t) * (num_seqs + 1), 16);
+        w.seg_count = reinterpret_cast<int32_t*>(sc);
+        w.seg_tab = reinterpret_cast<int4*>(sc + 16);
+        w.seg_states = reinterpret_cast<float*>(sc + 16 + align_up(sizeof(int4) * w.max_segs, 1024));
+    }
+    return w;
 }
 
 // SMs of the current device (cached per device; 0 when the query fails).  Host threads
@@ -1155,27 +1557,26 @@ inline int device_sm_count() {
     return n;
 }
 
-// Chunk table (+ emission slots when emit_pos is given) + chunk-parallel preparation.
+// Chunk table (+ emission slots when emit_pos is given) + chunk-parallel preparation, then
+// the CUDA-core preparation of the chunks prep_kernel listed for their strong decay.
 inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, const int32_t* cu, int num_seqs,
                                   int64_t total, int H, void* workspace, cudaStream_t stream,
                                   const int64_t* emit_pos = nullptr, int num_emit = 0,
                                   uint32_t in_flags = 0) {
     const bool g_scalar = (in_flags & kInGScalar) != 0;
-    const Workspace w = split_workspace(workspace, total, num_seqs);
-    const bool pro = (in_flags & ~(kInGScalar | kInStrongDecay)) != 0;
-    const bool strong = (in_flags & kInStrongDecay) != 0;
-    auto pick = [&](auto sc) {
-        constexpr bool kSc = decltype(sc)::value;
-        return strong ? (pro ? prep_kernel<kSc, true, true> : prep_kernel<kSc, false, true>)
-                      : (pro ? prep_kernel<kSc, true, false> : prep_kernel<kSc, false, false>);
-    };
-    auto prep = g_scalar ? pick(std::true_type{}) : pick(std::false_type{});
+    const Workspace w = split_workspace(workspace, total, num_seqs, H);
+    const bool pro = (in_flags & (kInNormQK | kInGLogits | kInBetaLogits)) != 0;
+    auto prep = g_scalar ? (pro ? prep_kernel<true, true> : prep_kernel<true, false>)
+                         : (pro ? prep_kernel<false, true> : prep_kernel<false, false>);
+    auto strong = g_scalar ? prep_strong_kernel<true> : prep_strong_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepSmem::BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(strong, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StrongSmem::BYTES);
     if (e != cudaSuccess) return e;
     chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off, w.tab,
-                                               num_emit > 0 ? w.etab : nullptr);
+                                               num_emit > 0 ? w.etab : nullptr, w.strong_count);
     if (num_emit > 0)
         emit_index_kernel<<<(num_emit + 255) / 256, 256, 0, stream>>>(cu, num_seqs, w.off, emit_pos,
                                                                        num_emit, w.etab);
@@ -1188,38 +1589,59 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
              !make_tmap(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE)))
             return cudaErrorInvalidValue;
         if (g_scalar) tg = tq;   // a scalar gate is read with plain loads: this map goes unused
-        dim3 grid((unsigned)max_chunks(total, num_seqs), (unsigned)H);
+        const int64_t units = max_chunks(total, num_seqs);
+        dim3 grid((unsigned)units, (unsigned)H);
         prep<<<grid, kPrepThreads, PrepSmem::BYTES, stream>>>(tq, tk, tv, tg, g_scalar ? g : nullptr,
                                                               beta, num_seqs, H, w.off, w.tab, w.records,
+                                                              w.strong_count, w.strong_units,
                                                               in_flags, total);
+        const int sms = device_sm_count();
+        const int64_t sgrid = std::min<int64_t>(units * H, sms > 0 ? sms : 148);
+        strong<<<(unsigned)sgrid, kStrongThreads, StrongSmem::BYTES, stream>>>(
+            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+            static_cast<const __nv_bfloat16*>(v), g, beta, num_seqs, H, w.tab, w.records, w.strong_count,
+            w.strong_units, in_flags, total);
     }
     return cudaGetLastError();
 }
 
-template <int NV>
-inline cudaError_t launch_scan_nv(const float* s0, float* sf, void* out, int num_seqs, const Workspace& w,
-                                  int H, float* emit_states, cudaStream_t stream) {
-    using R = RecCfg<NV>;
-    cudaError_t e = cudaFuncSetAttribute(rec_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)R::BYTES);
-    if (e != cudaSuccess) return e;
-    rec_kernel<NV><<<(unsigned)num_seqs * H * R::NSL, kRecThreads, R::BYTES, stream>>>(
-        num_seqs, H, w.off, w.tab, w.records, s0, sf, static_cast<__nv_bfloat16*>(out),
-        emit_states ? w.etab : nullptr, emit_states);
-    return cudaGetLastError();
-}
-
-// Chunk-serial recurrence and the chunk outputs, over every (sequence, head, value slice):
-// 32-channel slices while 4 CTAs per (sequence, head) fit on the SMs at once, else 64.
+// Chunk-serial recurrence and the chunk outputs: one CTA per (sequence, head), or, when a few
+// long chains would leave most SMs idle, the chunk-parallel scan over segments (segment
+// table, transitions, starting states, then the recurrence per segment).
 // emit_states (nullable) receives the states at the emission slots launch_prepare recorded.
 inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_seqs, int64_t total,
                                int H, void* workspace, cudaStream_t stream,
-                               float* emit_states = nullptr) {
-    const Workspace w = split_workspace(workspace, total, num_seqs);
+                               float* emit_states = nullptr, uint32_t in_flags = 0) {
+    const Workspace w = split_workspace(workspace, total, num_seqs, H);
+    if ((int64_t)num_seqs * H == 0) return cudaSuccess;
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+    const int32_t* et = emit_states ? w.etab : nullptr;
+    const bool scan = w.seg > 0 && !(in_flags & kInSerialChains);
+    const int64_t units = scan ? w.max_segs : num_seqs;   // chains: sequences, or scan segments
+    // 32-channel value slices while four CTAs per chain fit on the SMs at once, else 64
     const int sms = device_sm_count();
-    if ((int64_t)num_seqs * H * RecCfg<32>::NSL <= (int64_t)sms)
-        return launch_scan_nv<32>(s0, sf, out, num_seqs, w, H, emit_states, stream);
-    return launch_scan_nv<64>(s0, sf, out, num_seqs, w, H, emit_states, stream);
+    const bool narrow = units * H * RecCfg<32>::NSL <= (int64_t)(sms > 0 ? sms : 148);
+    auto rec = narrow ? rec_kernel<32> : rec_kernel<64>;
+    const uint32_t rec_smem = narrow ? RecCfg<32>::BYTES : RecCfg<64>::BYTES;
+    const int nsl = narrow ? RecCfg<32>::NSL : RecCfg<64>::NSL;
+    cudaError_t e = cudaFuncSetAttribute(rec, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rec_smem);
+    if (e != cudaSuccess) return e;
+    if (!scan) {
+        rec<<<(unsigned)(num_seqs * H * nsl), kRecThreads, rec_smem, stream>>>(
+            num_seqs, H, w.off, w.tab, w.records, s0, sf, o, et, emit_states, nullptr, nullptr, nullptr);
+        return cudaGetLastError();
+    }
+    e = cudaFuncSetAttribute(seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SegSmem::BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombineSmem);
+    if (e != cudaSuccess) return e;
+    segment_index_kernel<<<1, 1024, 0, stream>>>(num_seqs, w.off, w.seg, w.seg_off, w.seg_count, w.seg_tab);
+    seg_kernel<<<(unsigned)(w.max_segs * H), kSegThreads, SegSmem::BYTES, stream>>>(H, w.records, w.seg_tab,
+                                                                                    w.seg_count, w.seg_states);
+    combine_kernel<<<(unsigned)num_seqs * H, kCombineThreads, kCombineSmem, stream>>>(H, s0, w.seg_off, w.seg_states);
+    rec<<<(unsigned)(w.max_segs * H * nsl), kRecThreads, rec_smem, stream>>>(
+        num_seqs, H, w.off, w.tab, w.records, s0, sf, o, et, emit_states, w.seg_tab, w.seg_count, w.seg_states);
+    return cudaGetLastError();
 }
 
 inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* g,
@@ -1232,7 +1654,7 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
                                    emit_pos, num_emit, in_flags);
     if (e == cudaSuccess)
         e = launch_scan(s0, sf, out, num_seqs, total, H, workspace, stream,
-                        num_emit > 0 ? emit_states : nullptr);
+                        num_emit > 0 ? emit_states : nullptr, in_flags);
     return e;
 }
 

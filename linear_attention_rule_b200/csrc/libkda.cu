@@ -45,7 +45,7 @@ cudaError_t dispatch_simt(int32_t dk, int32_t C, const void* q, const void* k, c
 
 extern "C" {
 
-int32_t kda_abi_version(void) { return 6; }
+int32_t kda_abi_version(void) { return 7; }
 
 const char* kda_status_string(kda_status s) {
     switch (s) {
@@ -66,7 +66,28 @@ size_t kda_prefill_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_
         !valid_chunk(dt, C))
         return 0;
     if (!tensor_core_path(dt, dk)) return 0;
-    return kda::tc::workspace_bytes(total_tokens, num_seqs, H);
+    size_t bytes = 0;
+    return kda::tc::workspace_bytes_checked(total_tokens, num_seqs, H, &bytes) ? bytes : 0;
+}
+
+int32_t kda_prefill_launches(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
+                             int32_t dv, int32_t C, kda_dtype dt, uint32_t in_flags, int32_t num_emit) {
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0 || !supported_dim(dk, dv) || !valid_chunk(dt, C))
+        return -1;
+    if (num_seqs == 0) return 0;
+    if (!tensor_core_path(dt, dk)) return 1;
+    // chunk table, [emission slots], preparation, strongly decayed chunks, recurrence
+    int32_t n = 1 + (num_emit > 0 ? 1 : 0) + (total_tokens > 0 ? 2 : 0) + 1;
+    if (!(in_flags & KDA_IN_SERIAL_CHAINS) && kda::tc::scan_segment_chunks(total_tokens, num_seqs, H) > 0)
+        n += 3;   // segment table, segment transitions, starting states
+    return n;
+}
+
+// A tensor-core problem whose workspace or launch grids cannot be addressed (see
+// workspace_bytes_checked) is rejected before anything is launched.
+static bool tc_problem_fits(int64_t total_tokens, int32_t num_seqs, int32_t H) {
+    size_t bytes = 0;
+    return kda::tc::workspace_bytes_checked(total_tokens, num_seqs, H, &bytes);
 }
 
 static kda_status prefill_common(const void* q, const void* k, const void* v, const float* g,
@@ -79,7 +100,7 @@ static kda_status prefill_common(const void* q, const void* k, const void* v, co
     if (num_seqs < 0 || total_tokens < 0 || H <= 0 || dk <= 0 || dv <= 0 || num_emit < 0)
         return KDA_ERR_INVALID_ARG;
     if (in_flags & ~(uint32_t)(KDA_IN_NORMALIZE_QK | KDA_IN_G_LOGITS | KDA_IN_BETA_LOGITS |
-                               KDA_IN_G_SCALAR | KDA_IN_STRONG_DECAY))
+                               KDA_IN_G_SCALAR | KDA_IN_STRONG_DECAY | KDA_IN_SERIAL_CHAINS))
         return KDA_ERR_INVALID_ARG;
     if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (total_tokens > INT32_MAX) return KDA_ERR_UNSUPPORTED;  // cu_seqlens is int32
@@ -90,6 +111,7 @@ static kda_status prefill_common(const void* q, const void* k, const void* v, co
             return KDA_ERR_INVALID_ARG;
         if (!tensor_core_path(dt, dk)) return KDA_ERR_UNSUPPORTED;
     }
+    if (tensor_core_path(dt, dk) && !tc_problem_fits(total_tokens, num_seqs, H)) return KDA_ERR_UNSUPPORTED;
     if (num_seqs == 0) return KDA_OK;
     if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
@@ -169,6 +191,7 @@ static kda_status check_staged(const int32_t* cu_seqlens, int32_t num_seqs, int6
     if (total_tokens > INT32_MAX) return KDA_ERR_UNSUPPORTED;
     if (!tensor_core_path(dt, dk) || !supported_dim(dk, dv) || !valid_chunk(dt, C))
         return KDA_ERR_UNSUPPORTED;
+    if (!tc_problem_fits(total_tokens, num_seqs, H)) return KDA_ERR_UNSUPPORTED;
     if (num_seqs > 0 && (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0))
         return KDA_ERR_INVALID_ARG;
     const size_t need = kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, dt);
@@ -218,9 +241,9 @@ static kda_status decode_common(const void* q, const void* k, const void* v, con
                                 int32_t dk, int32_t dv, kda_dtype dt, kda_stream_t stream, uint32_t in_flags) {
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (in_flags & ~(uint32_t)(KDA_IN_NORMALIZE_QK | KDA_IN_G_LOGITS | KDA_IN_BETA_LOGITS |
-                               KDA_IN_G_SCALAR | KDA_IN_STRONG_DECAY))
+                               KDA_IN_G_SCALAR | KDA_IN_STRONG_DECAY | KDA_IN_SERIAL_CHAINS))
         return KDA_ERR_INVALID_ARG;
-    in_flags &= ~(uint32_t)KDA_IN_STRONG_DECAY;   // one token's decay is applied directly
+    in_flags &= ~(uint32_t)(KDA_IN_STRONG_DECAY | KDA_IN_SERIAL_CHAINS);   // no effect on one token
     if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (!supported_dim(dk, dv)) return KDA_ERR_UNSUPPORTED;
     if (N == 0) return KDA_OK;
@@ -291,25 +314,67 @@ kda_status kda_get_device_status(kda_stream_t stream) {
 static __device__ __align__(256) uint8_t g_kda_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 256;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 
-// Device address of the scratch array on the current device, looked up once per device.
-// The array's name is only a host-side stand-in; the kernels must get this address.
-cudaError_t noalloc_scratch(void** ptr) {
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess) return err;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+// cuCtxGetCurrent through the runtime's driver entry point (no link against libcuda).
+CtxGetCurrentFn ctx_get_current() {
+    static const CtxGetCurrentFn fn = [] {
         void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<CtxGetCurrentFn>(p);
+        return static_cast<CtxGetCurrentFn>(nullptr);
+    }();
+    return fn;
+}
+
+// Last looked-up scratch address per CUDA context.  The array's name is only a host-side
+// stand-in; the kernels must get the device address, which belongs to the context that
+// loaded the module: a new primary context after cudaDeviceReset, or another context made
+// current, has its own.
+struct ScratchEntry {
+    CUcontext ctx;
+    void* ptr;
+};
+constexpr int kMaxContexts = 64;
+std::mutex g_noalloc_mutex;
+ScratchEntry g_noalloc_cache[kMaxContexts] = {};
+
+// Device address of the scratch array in the current context.  Outside stream capture the
+// address is looked up on every call (cudaGetSymbolAddress, a host-side query once the
+// module is loaded) and the cache refreshed; while `stream` is capturing only the cache
+// of this context is used, so the first call in a context must come before any capture.
+cudaError_t noalloc_scratch(cudaStream_t stream, void** ptr) {
+    CtxGetCurrentFn get = ctx_get_current();
+    if (!get) return cudaErrorNotSupported;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t err = cudaStreamIsCapturing(stream, &cap);
+    if (err != cudaSuccess) return err;
+    void* p = nullptr;
+    if (cap == cudaStreamCaptureStatusNone) {
+        // also makes the device's primary context current if nothing was yet
         err = cudaGetSymbolAddress(&p, g_kda_noalloc_scratch);
         if (err != cudaSuccess) return err;
-        g_noalloc_ptr[dev] = p;
     }
-    *ptr = g_noalloc_ptr[dev];
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    int slot = -1;
+    for (int i = 0; i < kMaxContexts; ++i)
+        if (g_noalloc_cache[i].ctx == ctx) { slot = i; break; }
+    if (cap != cudaStreamCaptureStatusNone) {
+        if (slot < 0) return cudaErrorStreamCaptureUnsupported;
+        *ptr = g_noalloc_cache[slot].ptr;
+        return cudaSuccess;
+    }
+    if (slot < 0) {
+        for (int i = 0; i < kMaxContexts && slot < 0; ++i)
+            if (g_noalloc_cache[i].ctx == nullptr) slot = i;
+        if (slot < 0) slot = 0;   // table full: reuse the first entry
+    }
+    g_noalloc_cache[slot] = {ctx, p};
+    *ptr = p;
     return cudaSuccess;
 }
 }  // namespace
@@ -321,12 +386,15 @@ extern "C" kda_status kda_prefill_noalloc(const void* q, const void* k, const vo
                                           int32_t dk, int32_t dv, kda_dtype dt, void* out,
                                           float* final_state, int32_t C, kda_stream_t stream) {
     if (num_seqs < 0 || total_tokens < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (dt != KDA_BF16 || dk != 128 || dv != 128 || C != 64) return KDA_ERR_UNSUPPORTED;
+    if (total_tokens > INT32_MAX || !tc_problem_fits(total_tokens, num_seqs, H)) return KDA_ERR_UNSUPPORTED;
     const size_t need = kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, dt);
-    if (need > KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_UNSUPPORTED;
+    if (need == 0 || need > KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_UNSUPPORTED;
     if (num_seqs == 0) return KDA_OK;
     void* scratch = nullptr;
-    if (noalloc_scratch(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
+    if (noalloc_scratch(reinterpret_cast<cudaStream_t>(stream), &scratch) != cudaSuccess)
+        return KDA_ERR_CUDA;
     return kda_prefill(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_tokens, H,
                        dk, dv, dt, out, final_state, C, scratch, KDA_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -29,6 +29,7 @@ KDA_IN_G_LOGITS = 2
 KDA_IN_BETA_LOGITS = 4
 KDA_IN_G_SCALAR = 8
 KDA_IN_STRONG_DECAY = 16
+KDA_IN_SERIAL_CHAINS = 32
 KDA_F32 = 0
 KDA_BF16 = 1
 
@@ -37,7 +38,7 @@ EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_stat
             "kda_get_device_status", "kda_abi_version", "kda_prefill_noalloc",
             "kda_prefill_prepare", "kda_prefill_scan", "kda_selftest_bounded_wait",
             "kda_prefill_emit", "kda_prefill_gdn", "kda_decode_gdn", "kda_prefill_ex",
-            "kda_decode_ex")
+            "kda_decode_ex", "kda_prefill_launches")
 
 # Size of the library-owned scratch behind kda_prefill_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -94,6 +95,8 @@ def load() -> ctypes.CDLL:
     lib.kda_prefill_emit.argtypes = [P, P, P, P, P, P, P, I32, I64, I32, I32, I32, ctypes.c_int, P, P,
                                      I32, P, I32, P, P, SZ, P]
     lib.kda_prefill_emit.restype = ctypes.c_int
+    lib.kda_prefill_launches.argtypes = [I64, I32, I32, I32, I32, I32, ctypes.c_int, U32, I32]
+    lib.kda_prefill_launches.restype = I32
     lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P]
     lib.kda_selftest_bounded_wait.restype = ctypes.c_int
     _lib = lib
@@ -403,18 +406,20 @@ def kda_get_device_status(stream=None) -> int:
     return int(load().kda_get_device_status(_stream(stream)))
 
 
-def _tensor_core_path(dtype: torch.dtype, D: int) -> bool:
+def tensor_core_path(dtype: torch.dtype, D: int) -> bool:
     # mirrors tensor_core_path() in csrc/libkda.cu
     return dtype == torch.bfloat16 and D == 128
 
 
-def prefill_launches(dtype: torch.dtype, D: int = 128) -> int:
-    """Kernel launches one kda_prefill call makes: chunk index, preparation and
-    recurrence on the tensor-core path; one chunk-serial kernel on the CUDA-core path."""
-    return 3 if _tensor_core_path(dtype, D) else 1
+def kda_prefill_launches(total_tokens: int, num_seqs: int, H: int, dk: int, dv: int, C: int,
+                         dtype: torch.dtype, in_flags: int = 0, num_emit: int = 0) -> int:
+    """Kernels one kda_prefill_ex call with these sizes launches (kda_prefill_launches in
+    include/libkda.h)."""
+    code = KDA_F32 if dtype == torch.float32 else KDA_BF16
+    return int(load().kda_prefill_launches(total_tokens, num_seqs, H, dk, dv, C, code, in_flags, num_emit))
 
 
 def prefill_compute_dtype(dtype: torch.dtype, D: int = 128) -> str:
     """Operand type of the prefill contractions (accumulation and the state are fp32
     on every path)."""
-    return "bf16" if _tensor_core_path(dtype, D) else "f32"
+    return "bf16" if tensor_core_path(dtype, D) else "f32"

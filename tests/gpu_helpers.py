@@ -48,9 +48,11 @@ def oracle_prefill(inp: dict, heads=None, initial=True):
                           s0=s0, heads=heads)
 
 
-def check_prefill(inp: dict, out, final, heads=None, tol=None, initial=True):
+def check_prefill(inp: dict, out, final, heads=None, tol=None, initial=True, chunk=None):
     """Compare GPU results (all heads) with the oracle on `heads` (default all).
-    Returns (max output error, max final-state error)."""
+    With `chunk` (the chunk size C), every chunk of C rows of every (sequence, head) slice
+    is also held to the tolerance on its own, so that a few wrong rows cannot hide in a
+    long slice.  Returns (max output error, max final-state error)."""
     tol = TOL[inp["q"].dtype] if tol is None else tol
     o_ref, f_ref = oracle_prefill(inp, heads, initial=initial)
     hs = list(range(inp["q"].shape[1])) if heads is None else list(heads)
@@ -59,4 +61,8 @@ def check_prefill(inp: dict, out, final, heads=None, tol=None, initial=True):
     assert np.isfinite(out[:, hs]).all()
     assert e_out <= tol, ("output", e_out, tol)
     assert e_fin <= tol, ("final state", e_fin, tol)
+    if chunk is not None:
+        e_chunk = oracle.max_rel_frobenius_per_chunk(out[:, hs], o_ref, inp["cu_seqlens"], chunk)
+        print("worst chunk rel err %.3g" % e_chunk)
+        assert e_chunk <= tol, ("output chunk", e_chunk, tol)
     return e_out, e_fin

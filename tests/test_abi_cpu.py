@@ -46,7 +46,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert kda.kda_abi_version() == 6
+    assert kda.kda_abi_version() == 7
     for code in range(7):
         s = kda.kda_status_string(code)
         assert s and s != "unknown status"
@@ -172,15 +172,32 @@ def test_prologue_entry_points_reject_unknown_flags(lib):
     ex = lambda flags: lib.kda_prefill_ex(P(4096), P(4096), P(4096), P(4096), P(4096), None, P(4096), 1, 256,
                                           2, 128, 128, kda.KDA_BF16, P(4096), None, 64, flags, None, 0, None,
                                           P(1 << 20), need, None)
-    assert ex(32) == kda.KDA_ERR_INVALID_ARG
+    assert ex(64) == kda.KDA_ERR_INVALID_ARG
     assert ex(1 << 31) == kda.KDA_ERR_INVALID_ARG
     dec = lambda flags: lib.kda_decode_ex(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), 2,
                                           2, 128, 128, kda.KDA_BF16, flags, None)
-    assert dec(32) == kda.KDA_ERR_INVALID_ARG
+    assert dec(64) == kda.KDA_ERR_INVALID_ARG
     assert lib.kda_decode_ex(P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), P(4096), 0, 2, 128, 128,
-                             kda.KDA_BF16, 31, None) == kda.KDA_OK   # every known bit, N = 0
+                             kda.KDA_BF16, 63, None) == kda.KDA_OK   # every known bit, N = 0
 
 
 def test_selftest_rejects_out_of_range_limits(lib):
     assert lib.kda_selftest_bounded_wait(10, None) == kda.KDA_ERR_INVALID_ARG
     assert lib.kda_selftest_bounded_wait(3_000_000_000, None) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_prefill_launch_count(lib):
+    """Host-side count of the kernels one prefill call launches (no device needed)."""
+    bf, f32 = kda.KDA_BF16, kda.KDA_F32
+    n = lambda T, N, H, dt=bf, flags=0, emit=0, d=128: lib.kda_prefill_launches(T, N, H, d, d, 64, dt, flags, emit)
+    assert n(8192, 1, 32) == 4                    # 128 chunks per chain: segments too short
+    assert n(1 << 20, 1, 32) == 4                 # 32 chains x 4 slices already fill the SMs
+    assert n(1 << 20, 1, 8) == 7                  # 8 long chains: chunk-parallel scan (+3)
+    assert n(1 << 20, 1, 8, flags=kda.KDA_IN_SERIAL_CHAINS) == 4
+    assert n(8192, 16, 32) == 4                   # 512 chains fill the SMs: no scan
+    assert n(300, 1, 2) == 4                      # 5 chunks per chain: segments too short
+    assert n(8192, 1, 32, emit=2) == 5
+    assert n(0, 1, 32) == 2                       # chunk table and recurrence only
+    assert n(8192, 0, 32) == 0
+    assert n(256, 1, 2, dt=f32, d=64) == 1        # CUDA-core path: one kernel
+    assert n(256, 1, 2, d=96) == -1

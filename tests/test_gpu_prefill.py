@@ -35,12 +35,12 @@ def test_bf16_ragged_varlen_small():
     lens = [1000, 64, 63, 65, 1, 0, 300]
     inp = _inputs(lens, 4, 128, torch.bfloat16, seed=11)
     out, fin = run_prefill(inp, C=64)
-    check_prefill(inp, out, fin)
+    check_prefill(inp, out, fin, chunk=64)
 
 
 def test_bf16_many_sequence_heads():
-    """More (sequence, head) pairs than SMs / 4: the recurrence takes 64-channel value slices
-    (the other tests here run 32-channel slices).  Ragged and empty sequences included."""
+    """More (sequence, head) pairs than the recurrence can run at once on the SMs (192 CTAs),
+    ragged and empty sequences included."""
     lens = [100, 64, 1, 300, 0, 129]
     inp = _inputs(lens, 32, 128, torch.bfloat16, seed=13)
     out, fin = run_prefill(inp, C=64)
@@ -49,21 +49,65 @@ def test_bf16_many_sequence_heads():
 
 @pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.bfloat16, 64), (torch.float32, 64),
                                      (torch.float32, 128)])
-def test_strong_decay_beyond_fp32_exponent_range(dtype, D):
-    """Gates logsigmoid(N(-1.5, 1)): a full chunk's total log-decay is about -115 per channel,
-    so e^{-a} alone would overflow fp32 (and bf16); exponents relative to half the chunk's
-    decay (KDA_IN_STRONG_DECAY on the tensor-core path, always on the CUDA-core paths) keep
-    every factor within e^{|a_last| / 2}."""
-    inp = _inputs([200, 64, 70], 2, D, dtype, seed=17, g_mean=-1.5)
-    assert float(inp["g"][:64].sum(0).min()) < -100      # the premise: far beyond e^{88}
-    out, fin = run_prefill(inp, C=64, in_flags=kda.KDA_IN_STRONG_DECAY)
-    check_prefill(inp, out, fin)
+@pytest.mark.parametrize("g_mean", [-3.0, -8.0])
+def test_strong_decay_by_default(dtype, D, g_mean):
+    """Gates logsigmoid(N(-3, 1)) (a full chunk's log-decay near -190 per channel, so e^{-a}
+    alone would overflow fp32 and bf16) and logsigmoid(N(-8, 1)) (near -8 per token: even 16
+    tokens pass -88), with no flag: every path matches the oracle."""
+    inp = _inputs([200, 64, 70, 1], 2, D, dtype, seed=17, g_mean=g_mean)
+    assert float(inp["g"][:64].sum(0).max()) < -150      # the premise: far beyond e^{88}
+    out, fin = run_prefill(inp, C=64)
+    check_prefill(inp, out, fin, chunk=64)
+
+
+def test_strong_and_mild_chunks_in_one_call():
+    """Sequences whose chunks take the tensor-core preparation and sequences whose chunks are
+    too strongly decayed for it, packed together (and one chunk with a single strong channel
+    among mild ones): the records of both preparations meet in one recurrence."""
+    lens = [300, 130, 64, 200]
+    inp = _inputs(lens, 3, 128, torch.bfloat16, seed=71, g_mean=3.0)
+    strong = _inputs(lens, 3, 128, torch.bfloat16, seed=72, g_mean=-4.0)
+    cu = inp["cu_seqlens"].tolist()
+    inp["g"][cu[1]:cu[2]] = strong["g"][cu[1]:cu[2]]          # sequence 1 strong everywhere
+    inp["g"][cu[3] + 64:cu[3] + 128, 1, 5] = -3.0              # one channel of one chunk of head 1
+    out, fin = run_prefill(inp, C=64)
+    check_prefill(inp, out, fin, chunk=64)
+
+
+def test_strong_decay_with_prologue_and_scalar_gate():
+    """Strong decay through the Gated DeltaNet scalar gate and through gate logits."""
+    import oracle
+    lens = [150, 64]
+    inp = _inputs(lens, 2, 128, torch.bfloat16, seed=73, g_mean=-4.0)
+    gs = inp["g"][:, :, 0].contiguous()                        # one gate per (token, head)
+    d = to_device(inp)
+    out = torch.full_like(d["v"], float("nan"))
+    fin = torch.full((2, 2, 128, 128), float("nan"), device="cuda")
+    kda.kda_prefill_gdn(d["q"], d["k"], d["v"], gs.cuda(), d["beta"], d["cu_seqlens"], out,
+                        initial_state=d["s0"], final_state=fin)
+    assert kda.kda_get_device_status() == kda.KDA_OK
+    g_full = gs[..., None].expand(-1, -1, 128).contiguous()
+    o_ref, f_ref = oracle.prefill(inp["q"], inp["k"], inp["v"], g_full, inp["beta"], inp["cu_seqlens"],
+                                  s0=inp["s0"])
+    tol = TOL[torch.bfloat16]
+    assert oracle.max_rel_frobenius_per_slice(out.double().cpu().numpy(), o_ref, inp["cu_seqlens"]) <= tol
+    assert oracle.max_rel_frobenius_states(fin.double().cpu().numpy(), f_ref) <= tol
+    # gate logits N(-3, 1): logsigmoid applied inside, strong decay in every chunk
+    logits = -3.0 + torch.randn(inp["g"].shape, generator=torch.Generator().manual_seed(74))
+    out2 = torch.full_like(d["v"], float("nan"))
+    kda.kda_prefill_ex(d["q"], d["k"], d["v"], logits.cuda(), d["beta"], d["cu_seqlens"], out2,
+                       kda.KDA_IN_G_LOGITS, initial_state=d["s0"], final_state=fin)
+    assert kda.kda_get_device_status() == kda.KDA_OK
+    g2 = torch.from_numpy(oracle.logsigmoid(logits)).float()
+    o_ref2, f_ref2 = oracle.prefill(inp["q"], inp["k"], inp["v"], g2, inp["beta"], inp["cu_seqlens"],
+                                    s0=inp["s0"])
+    assert oracle.max_rel_frobenius_per_slice(out2.double().cpu().numpy(), o_ref2, inp["cu_seqlens"]) <= tol
+    assert oracle.max_rel_frobenius_states(fin.double().cpu().numpy(), f_ref2) <= tol
 
 
 @pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.float32, 64)])
 def test_strong_decay_flag_is_bit_identical_on_mild_decay(dtype, D):
-    """Channels whose chunk total stays above -64 keep the chunk-start reference: the flag
-    changes nothing there, bit for bit (and the CUDA-core paths ignore it)."""
+    """KDA_IN_STRONG_DECAY is accepted and ignored: results are the same bit for bit."""
     inp = _inputs([300, 64, 1, 129], 3, D, dtype, seed=19, g_mean=3.0)
     assert float(inp["g"][:64].sum(0).min()) > -64
     o0, f0 = run_prefill(inp, C=64)
@@ -132,7 +176,7 @@ def test_config1_full_size_sampled_heads():
     configuration; the oracle checks every output and the final state of 3 heads."""
     inp = synthetic.make_config_inputs(1)
     out, fin = run_prefill(inp, C=64)
-    e_o, e_f = check_prefill(inp, out, fin, heads=[0, 13, 31])
+    e_o, e_f = check_prefill(inp, out, fin, heads=[0, 13, 31], chunk=64)
     print("config1 max rel err out %.3g final %.3g" % (e_o, e_f))
 
 
@@ -140,7 +184,7 @@ def test_config2_full_size_sampled_heads():
     """Config 2 at full size (16 sequences, lengths U[1024, 32768], S0 ~ N(0, 0.02^2))."""
     inp = synthetic.make_config_inputs(2)
     out, fin = run_prefill(inp, C=64)
-    e_o, e_f = check_prefill(inp, out, fin, heads=[5, 30])
+    e_o, e_f = check_prefill(inp, out, fin, heads=[5, 30], chunk=64)
     print("config2 max rel err out %.3g final %.3g" % (e_o, e_f))
 
 
@@ -246,8 +290,10 @@ def test_config4_long_context_full_size_sampled_heads():
                                   nthreads=len(heads))
     e_o = oracle.max_rel_frobenius_per_slice(o, o_ref, c["cu_seqlens"])
     e_f = oracle.max_rel_frobenius_states(f, f_ref)
-    print("config4 max rel err out %.3g final %.3g" % (e_o, e_f))
+    e_c = oracle.max_rel_frobenius_per_chunk(o, o_ref, c["cu_seqlens"], cfg.C)
+    print("config4 max rel err out %.3g final %.3g worst chunk %.3g" % (e_o, e_f, e_c))
     assert e_o <= TOL[torch.bfloat16] and e_f <= TOL[torch.bfloat16]
+    assert e_c <= TOL[torch.bfloat16]
     # windows along the sequence (early, middle, end) stay within tolerance too
     for a in (0, T // 2, T - 65536):
         e_w = oracle.rel_frobenius(o[a:a + 65536], o_ref[a:a + 65536])
