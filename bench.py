@@ -97,8 +97,10 @@ def prefill_stage_page_bytes(lengths, H, D, C):
 
 # CUDA sources each kernel's recorded counters depend on (its own file and the helpers it uses)
 KERNEL_SOURCES = {
-    "prep_kernel": ("kda_common.cuh", "kda_sm100.cuh", "kda_prefill_tc.cuh"),
-    "rec_kernel": ("kda_common.cuh", "kda_sm100.cuh", "kda_prefill_tc.cuh"),
+    "prep_kernel": ("kda_common.cuh", "kda_sm100.cuh", "kda_prefill_tc.cuh",
+                    "kda_prep_strong.cuh", "kda_chunk_simt.cuh"),
+    "rec_kernel": ("kda_common.cuh", "kda_sm100.cuh", "kda_prefill_tc.cuh",
+                   "kda_prep_strong.cuh", "kda_chunk_simt.cuh"),
     "decode_kernel": ("kda_common.cuh", "kda_decode.cuh"),
 }
 
