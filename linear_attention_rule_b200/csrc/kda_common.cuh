@@ -12,6 +12,16 @@ __device__ int g_kda_status;
 
 __device__ __forceinline__ void kda_set_status(int s) { atomicCAS(&g_kda_status, 0, s); }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization
+// may start before the kernel ahead of it in the stream has finished: it waits for that
+// kernel's completion (and its memory) at kda_grid_wait, before its first access to anything
+// that kernel writes or reads.  Every kernel of such a chain waits on every path, so each
+// one completing implies that all before it have completed.  Without the attribute both
+// calls do nothing.
+__device__ __forceinline__ void kda_grid_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel of the stream be scheduled (its blocks wait at kda_grid_wait).
+__device__ __forceinline__ void kda_grid_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Input prologue (the layer's elementwise steps in front of KDA, fused into the kernels):
 // bit flags as in include/libkda.h (KDA_IN_*).
 constexpr uint32_t kInNormQK = 1u, kInGLogits = 2u, kInBetaLogits = 4u, kInGScalar = 8u,

@@ -40,6 +40,7 @@
 #include <algorithm>
 #include <atomic>
 #include <type_traits>
+#include <utility>
 
 #include "kda_common.cuh"
 #include "kda_sm100.cuh"
@@ -172,6 +173,7 @@ chunk_index_kernel(const int32_t* __restrict__ cu, int num_seqs, int64_t total,
     __shared__ int32_t carry;
     __shared__ int bad;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    kda_grid_launch_next();   // the preparation's blocks may start loading their inputs
     if (tid == 0) { carry = 0; bad = 0; *strong_count = 0; }
     __syncthreads();
     for (int base = 0; base < num_seqs; base += 1024) {
@@ -320,18 +322,26 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t in_flags = kPrologue ? in_flags_arg : 0u;
     using S = PrepSmem;
     const int c = blockIdx.x, h = blockIdx.y;
+    kda_grid_launch_next();
+    // One sequence: chunk c is tokens 64 c .., and the input copies are issued before the wait
+    // for the chunk table (whose kernel also resets the strong-decay count used below).
+    const bool one_seq = num_seqs == 1;
     int total_chunks, t0, nrow;
-    if (num_seqs == 1) {   // one sequence: chunk c is tokens 64 c .., no table load before the TMA
+    if (one_seq) {
         total_chunks = (int)((total + C - 1) / C);
         t0 = c * C;
         nrow = (int)(total - t0 < C ? total - t0 : C);
     } else {
+        kda_grid_wait();
         total_chunks = off[num_seqs];
         const int2 e = tab[c];   // in bounds for every c < max_chunks; meaningful for c < total
         t0 = e.x;
         nrow = e.y;
     }
-    if (c >= total_chunks) return;
+    if (c >= total_chunks) {
+        if (one_seq) kda_grid_wait();
+        return;
+    }
     uint8_t* rec = records + ((size_t)c * H + h) * kRecBytes;
 
     extern __shared__ uint8_t smem_raw[];
@@ -383,6 +393,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const float x = r < nrow ? g_scalar[(size_t)(t0 + r) * H + h] : 0.f;
         reinterpret_cast<float*>(sm + S::GR)[r] = r < nrow && (in_flags & kInGLogits) ? kda_logsigmoid(x) : x;
     }
+    if (one_seq) kda_grid_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -939,6 +950,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
     using S = RecCfg<NV>;
     constexpr int NSL = S::NSL;
     (void)num_seqs;
+    kda_grid_wait();   // the chunk table and the records
     const int sl = blockIdx.x % NSL;
     const int h = (blockIdx.x / NSL) % H;
     const int unit = blockIdx.x / (NSL * H);   // sequence, or scan segment
@@ -1545,6 +1557,24 @@ inline Workspace split_workspace(void* workspace, int64_t total, int num_seqs, i
 
 // SMs of the current device (cached per device; 0 when the query fails).  Host threads
 // may race on the first query of a device: they store the same value, atomically.
+// Launch with programmatic stream serialization: the kernel's blocks may be scheduled while
+// the kernel ahead of it in the stream is still running; they wait for it in kda_grid_wait.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_after(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 inline int device_sm_count() {
     static std::atomic<int> cached[64];
     int dev = 0;
@@ -1591,16 +1621,17 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
         if (g_scalar) tg = tq;   // a scalar gate is read with plain loads: this map goes unused
         const int64_t units = max_chunks(total, num_seqs);
         dim3 grid((unsigned)units, (unsigned)H);
-        prep<<<grid, kPrepThreads, PrepSmem::BYTES, stream>>>(tq, tk, tv, tg, g_scalar ? g : nullptr,
-                                                              beta, num_seqs, H, w.off, w.tab, w.records,
-                                                              w.strong_count, w.strong_units,
-                                                              in_flags, total);
+        e = launch_after(prep, grid, dim3(kPrepThreads), PrepSmem::BYTES, stream, tq, tk, tv, tg,
+                         g_scalar ? g : nullptr, beta, num_seqs, H, (const int32_t*)w.off, (const int2*)w.tab,
+                         w.records, w.strong_count, w.strong_units, in_flags, total);
+        if (e != cudaSuccess) return e;
         const int sms = device_sm_count();
         const int64_t sgrid = std::min<int64_t>(units * H, sms > 0 ? sms : 148);
-        strong<<<(unsigned)sgrid, kStrongThreads, StrongSmem::BYTES, stream>>>(
-            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-            static_cast<const __nv_bfloat16*>(v), g, beta, num_seqs, H, w.tab, w.records, w.strong_count,
-            w.strong_units, in_flags, total);
+        e = launch_after(strong, dim3((unsigned)sgrid), dim3(kStrongThreads), StrongSmem::BYTES, stream,
+                         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                         static_cast<const __nv_bfloat16*>(v), g, beta, num_seqs, H, (const int2*)w.tab,
+                         w.records, (const int32_t*)w.strong_count, (const int2*)w.strong_units, in_flags, total);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
@@ -1626,11 +1657,11 @@ inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_se
     const int nsl = narrow ? RecCfg<32>::NSL : RecCfg<64>::NSL;
     cudaError_t e = cudaFuncSetAttribute(rec, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rec_smem);
     if (e != cudaSuccess) return e;
-    if (!scan) {
-        rec<<<(unsigned)(num_seqs * H * nsl), kRecThreads, rec_smem, stream>>>(
-            num_seqs, H, w.off, w.tab, w.records, s0, sf, o, et, emit_states, nullptr, nullptr, nullptr);
-        return cudaGetLastError();
-    }
+    if (!scan)
+        return launch_after(rec, dim3((unsigned)(num_seqs * H * nsl)), dim3(kRecThreads), rec_smem, stream,
+                            num_seqs, H, (const int32_t*)w.off, (const int2*)w.tab, (const uint8_t*)w.records, s0,
+                            sf, o, et, emit_states, (const int4*)nullptr, (const int32_t*)nullptr,
+                            (const float*)nullptr);
     e = cudaFuncSetAttribute(seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SegSmem::BYTES);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombineSmem);
@@ -1639,9 +1670,12 @@ inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_se
     seg_kernel<<<(unsigned)(w.max_segs * H), kSegThreads, SegSmem::BYTES, stream>>>(H, w.records, w.seg_tab,
                                                                                     w.seg_count, w.seg_states);
     combine_kernel<<<(unsigned)num_seqs * H, kCombineThreads, kCombineSmem, stream>>>(H, s0, w.seg_off, w.seg_states);
-    rec<<<(unsigned)(w.max_segs * H * nsl), kRecThreads, rec_smem, stream>>>(
-        num_seqs, H, w.off, w.tab, w.records, s0, sf, o, et, emit_states, w.seg_tab, w.seg_count, w.seg_states);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_after(rec, dim3((unsigned)(w.max_segs * H * nsl)), dim3(kRecThreads), rec_smem, stream,
+                        num_seqs, H, (const int32_t*)w.off, (const int2*)w.tab, (const uint8_t*)w.records, s0, sf,
+                        o, et, emit_states, (const int4*)w.seg_tab, (const int32_t*)w.seg_count,
+                        (const float*)w.seg_states);
 }
 
 inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* g,

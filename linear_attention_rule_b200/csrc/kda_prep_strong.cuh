@@ -48,6 +48,8 @@ prep_strong_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
     float* sNq = smf + S::NQ;
     float* sNk = smf + S::NK;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    kda_grid_launch_next();
+    kda_grid_wait();   // the list the preparation wrote
     const int count = *strong_count;
 
     for (int item = blockIdx.x; item < count; item += gridDim.x) {
