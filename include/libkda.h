@@ -85,10 +85,20 @@ typedef enum {
  *   final_state   [num_seqs, H, dk, dv]   fp32, or NULL to skip; may alias initial_state
  *   C             chunk size: 64 for bf16; 16, 32 or 64 for fp32.  Chunks never straddle
  *                 sequences; the last chunk of a sequence may be partial.
- *   workspace     device scratch of at least kda_prefill_workspace_size(...) bytes,
- *                 256-byte aligned (may be NULL when that size is 0).  Its contents on
- *                 entry do not matter; it is clobbered.  Two calls in flight at once need
- *                 two workspaces.
+ *   workspace     device scratch, 256-byte aligned (may be NULL when the size needed is
+ *                 0), of ws_bytes bytes: kda_prefill_workspace_size(...) for the fastest
+ *                 run, or anything down to kda_prefill_workspace_size_min(...), with which
+ *                 the chunks run in windows (below).  Its contents on entry do not matter;
+ *                 it is clobbered.  Two calls in flight at once need two workspaces.
+ * Windows: the full workspace holds a record of about 88.5 KB per chunk of 64 tokens and
+ * head (the chunk tensors the recurrence reads).  With less, the call prepares and runs the
+ * chunks in windows of W consecutive chunks of the packed problem, as many as the workspace
+ * holds (at least 8): each window is prepared, then its recurrence runs, and a sequence
+ * that crosses a window boundary carries its fp32 state to the next window through the
+ * workspace.  The results are the same, bit for bit; the cost is three more kernel
+ * launches per window and, within a window, no chunk-parallel scan.  The workspace is then
+ * bounded by the window, not by total_tokens: about W x H x 88.5 KB + 2 x H x 64 KB + 16
+ * bytes per chunk.
  * Supported: dk == dv, both 64 or 128.  num_seqs == 0 or total_tokens == 0 are valid.
  * Decay range: any.  The chunk products need e^{a_r - a_s} (a the cumulative log-decay in
  * the chunk, s <= r), which is at most 1, but the factor e^{-a} of K_inv overflows once a
@@ -206,6 +216,21 @@ size_t kda_prefill_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_
                                   int32_t dk, int32_t dv, int32_t C, kda_dtype dt);
 
 /*
+ * The least workspace kda_prefill accepts for this problem: windows of 8 chunks, or the
+ * full size when that is smaller (0 when it needs none).  Depends only on the arguments.
+ */
+size_t kda_prefill_workspace_size_min(int64_t total_tokens, int32_t num_seqs, int32_t H,
+                                      int32_t dk, int32_t dv, int32_t C, kda_dtype dt);
+
+/*
+ * Windows a kda_prefill call with a workspace of ws_bytes runs in: 1 with the full
+ * workspace (or on a path that needs none), more below it, -1 for invalid or unsupported
+ * arguments or a workspace below kda_prefill_workspace_size_min.
+ */
+int64_t kda_prefill_windows(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
+                            int32_t dv, int32_t C, kda_dtype dt, size_t ws_bytes);
+
+/*
  * Number of kernels one kda_prefill_ex call with these arguments launches (for capturing
  * the call in a CUDA graph or counting launches), -1 for arguments kda_prefill_ex rejects
  * as unsupported.  On the tensor-core path that is the chunk table, the emission slots
@@ -214,6 +239,9 @@ size_t kda_prefill_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_
  * that runs, unless in_flags holds KDA_IN_SERIAL_CHAINS, when few (sequence, head) chains
  * are long: when the recurrence's four value-slice CTAs per chain would leave at least half
  * of 148 SMs idle (18 chains or fewer) and segments of 64 chunks or more result.
+ * That count is for the full workspace; a call that runs in n > 1 windows
+ * (kda_prefill_windows) launches the chunk table, the emission slots when num_emit > 0,
+ * and three kernels per window (preparation, strongly decayed chunks, recurrence).
  * Depends on the sizes only.
  */
 int32_t kda_prefill_launches(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
@@ -289,9 +317,11 @@ kda_status kda_selftest_bounded_wait(uint64_t limit_ns, kda_stream_t stream);
  *     problem returns KDA_ERR_UNSUPPORTED (the CUDA-core path needs no scratch: call
  *     kda_prefill with a NULL workspace instead).  A dtype that is neither KDA_F32 nor
  *     KDA_BF16 is KDA_ERR_INVALID_ARG, as for every entry point.
- *   - A problem whose kda_prefill_workspace_size exceeds KDA_NOALLOC_SCRATCH_BYTES returns
- *     KDA_ERR_UNSUPPORTED before anything is launched (with H = 32 and one sequence that
- *     is anything beyond 1,471 tokens).
+ *   - The scratch array is the call's workspace: problems up to its size run in one
+ *     window, larger ones in windows (kda_prefill, Windows), with the same results.  A
+ *     problem whose kda_prefill_workspace_size_min exceeds KDA_NOALLOC_SCRATCH_BYTES returns
+ *     KDA_ERR_UNSUPPORTED before anything is launched (windows of 8 chunks need about
+ *     H x 0.8 MB, so that is more than about 72 heads).
  *   - The scratch address belongs to the CUDA context that loaded the library's module on
  *     that device.  Every call made while `stream` is not capturing looks it up again in
  *     the current context (cudaGetSymbolAddress), so a new primary context after
@@ -323,7 +353,7 @@ const char *kda_status_string(kda_status s);
  */
 kda_status kda_get_device_status(kda_stream_t stream);
 
-/* ABI version of this header: 7. */
+/* ABI version of this header: 8. */
 int32_t kda_abi_version(void);
 
 #ifdef __cplusplus

@@ -150,6 +150,47 @@ __host__ inline bool workspace_bytes_checked(int64_t total_tokens, int num_seqs,
     return true;
 }
 
+// Windowed workspace: when the caller's workspace is smaller than workspace_bytes, the chunks
+// run in windows of W global chunks, each prepared and then run through the recurrence
+// before the next; a sequence crossing a window boundary carries its fp32 state from one
+// window to the next through one of two slots per head.
+// [chunk offsets (N+1)] [chunk table (max_chunks)] [emission slot per chunk] [strong-decay
+// count per window (max_chunks)] [strong-decay units (W x H)] [carry 2 x H x D x D fp32]
+// [records (W x H)]
+constexpr int64_t kMinWindowChunks = 8;
+struct WindowLayout {
+    size_t counts, list, carry, records, bytes;
+};
+__host__ inline WindowLayout window_layout(int64_t total_tokens, int num_seqs, int H, int64_t W) {
+    const size_t mc = (size_t)max_chunks(total_tokens, num_seqs);
+    WindowLayout l;
+    l.counts = align_up(ws_emit_offset(total_tokens, num_seqs) + sizeof(int32_t) * mc, 16);
+    l.list = align_up(l.counts + sizeof(int32_t) * mc, 16);
+    l.carry = align_up(l.list + sizeof(int2) * (size_t)W * H, 1024);
+    l.records = align_up(l.carry + 2 * sizeof(float) * (size_t)H * D * D, 1024);
+    l.bytes = l.records + (size_t)W * H * kRecBytes;
+    return l;
+}
+// Chunks per window for a workspace of ws_bytes: max_chunks (one window, the layout of
+// workspace_bytes) when that fits, else the most that fit, 0 when not even kMinWindowChunks do.
+__host__ inline int64_t window_chunks(int64_t total_tokens, int num_seqs, int H, size_t ws_bytes) {
+    const int64_t mc = max_chunks(total_tokens, num_seqs);
+    if (ws_bytes >= workspace_bytes(total_tokens, num_seqs, H)) return mc;
+    const WindowLayout l0 = window_layout(total_tokens, num_seqs, H, 0);
+    if (ws_bytes < l0.bytes) return 0;
+    int64_t W = (int64_t)((ws_bytes - l0.bytes) / ((size_t)H * (kRecBytes + sizeof(int2))));
+    if (W >= mc) W = mc - 1;   // a full window takes the one-window layout, which did not fit
+    while (W >= kMinWindowChunks && window_layout(total_tokens, num_seqs, H, W).bytes > ws_bytes) --W;
+    return W >= kMinWindowChunks ? W : 0;
+}
+// The least workspace the prefill accepts (a window of kMinWindowChunks, or one window when
+// the whole problem is not larger than that).
+__host__ inline size_t workspace_bytes_min(int64_t total_tokens, int num_seqs, int H) {
+    const size_t full = workspace_bytes(total_tokens, num_seqs, H);
+    const size_t win = window_layout(total_tokens, num_seqs, H, kMinWindowChunks).bytes;
+    return win < full ? win : full;
+}
+
 // ------------------------------------------------------------------ chunk index
 // Sequence containing global chunk c: the largest n with off[n] <= c.
 __device__ __forceinline__ int find_seq(const int32_t* off, int num_seqs, int c) {
@@ -168,13 +209,14 @@ __device__ __forceinline__ int find_seq(const int32_t* off, int num_seqs, int c)
 __global__ void __launch_bounds__(1024)
 chunk_index_kernel(const int32_t* __restrict__ cu, int num_seqs, int64_t total,
                    int32_t* __restrict__ off, int2* __restrict__ tab, int32_t* __restrict__ etab,
-                   int32_t* __restrict__ strong_count) {
+                   int32_t* __restrict__ strong_count, int num_counts) {
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t carry;
     __shared__ int bad;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     kda_grid_launch_next();   // the preparation's blocks may start loading their inputs
-    if (tid == 0) { carry = 0; bad = 0; *strong_count = 0; }
+    if (tid == 0) { carry = 0; bad = 0; }
+    for (int i = tid; i < num_counts; i += blockDim.x) strong_count[i] = 0;   // one per window
     __syncthreads();
     for (int base = 0; base < num_seqs; base += 1024) {
         const int n = base + tid;
@@ -318,10 +360,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float* __restrict__ g_scalar, const float* __restrict__ beta, int num_seqs, int H,
             const int32_t* __restrict__ off, const int2* __restrict__ tab, uint8_t* __restrict__ records,
             int32_t* __restrict__ strong_count, int2* __restrict__ strong_units,
-            uint32_t in_flags_arg, int64_t total) {
+            uint32_t in_flags_arg, int64_t total, int c_base) {
     const uint32_t in_flags = kPrologue ? in_flags_arg : 0u;
     using S = PrepSmem;
-    const int c = blockIdx.x, h = blockIdx.y;
+    // chunk c of the problem; records are indexed from the window's first chunk c_base
+    const int c = c_base + (int)blockIdx.x, h = blockIdx.y;
     kda_grid_launch_next();
     // One sequence: chunk c is tokens 64 c .., and the input copies are issued before the wait
     // for the chunk table (whose kernel also resets the strong-decay count used below).
@@ -334,15 +377,18 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     } else {
         kda_grid_wait();
         total_chunks = off[num_seqs];
-        const int2 e = tab[c];   // in bounds for every c < max_chunks; meaningful for c < total
-        t0 = e.x;
-        nrow = e.y;
+        t0 = nrow = 0;
+        if (c < total_chunks) {
+            const int2 e = tab[c];
+            t0 = e.x;
+            nrow = e.y;
+        }
     }
     if (c >= total_chunks) {
         if (one_seq) kda_grid_wait();
         return;
     }
-    uint8_t* rec = records + ((size_t)c * H + h) * kRecBytes;
+    uint8_t* rec = records + ((size_t)(c - c_base) * H + h) * kRecBytes;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
@@ -940,13 +986,25 @@ __device__ __forceinline__ void load_record_stages(uint32_t sb, uint32_t stage_b
 // Segments of the chunk-parallel scan (seg_tab non-null): CTA (segment s, head h, slice) runs
 // the segment's chunks from S_in(s) (the initial state for a sequence's first segment) and
 // writes the final state only from the sequence's last segment.
+// The window of chunks one recurrence launch covers: chunks [c_lo, c_hi) of the problem,
+// whose records start at records[0]; a sequence that began before c_lo starts from
+// carry_in, one that continues past c_hi leaves its state in carry_out (both [H][D][D]
+// fp32).  One window from 0 to INT32_MAX is the whole problem.
+struct RecWindow {
+    int c_lo, c_hi;
+    int last;   // the last window: it also owns empty sequences that sit at its end
+    const float* carry_in;
+    float* carry_out;
+};
+constexpr RecWindow kWholeProblem = {0, INT32_MAX, 1, nullptr, nullptr};
+
 template <int NV>
 __global__ void __launch_bounds__(kRecThreads, 1)
 rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __restrict__ tab,
            const uint8_t* __restrict__ records, const float* initial_state, float* final_state,
            __nv_bfloat16* __restrict__ out, const int32_t* __restrict__ etab, float* emit_states,
            const int4* __restrict__ seg_tab, const int32_t* __restrict__ seg_count,
-           const float* __restrict__ seg_states) {
+           const float* __restrict__ seg_states, RecWindow win) {
     using S = RecCfg<NV>;
     constexpr int NSL = S::NSL;
     (void)num_seqs;
@@ -957,6 +1015,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
     int n, c_begin, nchunks;
     bool write_final = final_state != nullptr;
     const float* s_init;
+    float* s_carry = nullptr;   // where the state goes when the sequence continues past the window
     if (seg_tab) {
         if (unit >= *seg_count) return;   // the whole CTA, before any barrier
         const int4 sg = seg_tab[unit];    // (sequence, first chunk, chunks, index | last << 16)
@@ -968,12 +1027,27 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
                      ? (initial_state ? initial_state + ((size_t)n * H + h) * D * D : nullptr)
                      : seg_states + ((size_t)unit * H + h) * (kSegStateBytes / sizeof(float)) + 2 * D * D;
     } else {
+        // this sequence's chunks inside the window [c_lo, c_hi)
         n = unit;
-        c_begin = off[n];
-        nchunks = off[n + 1] - c_begin;
-        s_init = initial_state ? initial_state + ((size_t)n * H + h) * D * D : nullptr;
+        const int a = off[n], b = off[n + 1];
+        c_begin = max(a, win.c_lo);
+        nchunks = min(b, win.c_hi) - c_begin;
+        if (nchunks <= 0) {
+            // an empty sequence belongs to the window at its position (the last window takes
+            // those at the very end); a sequence outside the window has nothing to do here
+            const bool owner = a == b && a >= win.c_lo && (a < win.c_hi || win.last);
+            if (!owner) return;   // the whole CTA, before any barrier
+            nchunks = 0;
+        }
+        const bool starts_here = a >= win.c_lo;
+        s_init = starts_here ? (initial_state ? initial_state + ((size_t)n * H + h) * D * D : nullptr)
+                             : win.carry_in + (size_t)h * D * D;
+        if (b > win.c_hi) {
+            write_final = false;
+            s_carry = win.carry_out + (size_t)h * D * D;
+        }
     }
-    auto record = [&](int kk) { return records + ((size_t)(c_begin + kk) * H + h) * kRecBytes; };
+    auto record = [&](int kk) { return records + ((size_t)(c_begin + kk - win.c_lo) * H + h) * kRecBytes; };
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
@@ -1185,8 +1259,8 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
         if (!ok) {
             if (lane == 0) kda_set_status(KDA_ERR_TIMEOUT);
             *abort_flag = 1;
-        } else if (write_final) {
-            float* dst = final_state + ((size_t)n * H + h) * D * D + (size_t)i * D + col0;
+        } else if (write_final || s_carry) {
+            float* dst = (s_carry ? s_carry : final_state + ((size_t)n * H + h) * D * D) + (size_t)i * D + col0;
 #pragma unroll
             for (int j4 = 0; j4 < NC / 4; ++j4)
                 reinterpret_cast<float4*>(dst)[j4] =
@@ -1589,14 +1663,40 @@ inline int device_sm_count() {
 
 // Chunk table (+ emission slots when emit_pos is given) + chunk-parallel preparation, then
 // the CUDA-core preparation of the chunks prep_kernel listed for their strong decay.
-inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, const float* g,
-                                  const float* beta, const int32_t* cu, int num_seqs,
-                                  int64_t total, int H, void* workspace, cudaStream_t stream,
-                                  const int64_t* emit_pos = nullptr, int num_emit = 0,
-                                  uint32_t in_flags = 0) {
+// What the preparation of any range of chunks needs: the inputs, their tensor maps and the
+// chunk table.
+struct PrepInputs {
+    CUtensorMap tq, tk, tv, tg;
+    const void *q, *k, *v;
+    const float *g, *beta;
+    int num_seqs, H;
+    int64_t total;
+    const int32_t* off;
+    const int2* tab;
+    uint32_t in_flags;
+};
+inline cudaError_t make_prep_inputs(PrepInputs* p, const void* q, const void* k, const void* v, const float* g,
+                                    const float* beta, int num_seqs, int64_t total, int H, const Workspace& w,
+                                    uint32_t in_flags) {
     const bool g_scalar = (in_flags & kInGScalar) != 0;
-    const Workspace w = split_workspace(workspace, total, num_seqs, H);
-    const bool pro = (in_flags & (kInNormQK | kInGLogits | kInBetaLogits)) != 0;
+    *p = PrepInputs{};
+    p->q = q; p->k = k; p->v = v; p->g = g; p->beta = beta;
+    p->num_seqs = num_seqs; p->H = H; p->total = total; p->off = w.off; p->tab = w.tab; p->in_flags = in_flags;
+    if (!make_tmap(&p->tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap(&p->tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap(&p->tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        (!g_scalar && !make_tmap(&p->tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE)))
+        return cudaErrorInvalidValue;
+    if (g_scalar) p->tg = p->tq;   // a scalar gate is read with plain loads: this map goes unused
+    return cudaSuccess;
+}
+// Prepares chunks c_base .. c_base + nchunks - 1 (those that exist) into records[0 ..]:
+// the tensor-core preparation, then the CUDA-core one for the chunks it listed in
+// (count, list), which the chunk-table kernel zeroed.
+inline cudaError_t launch_prep_chunks(const PrepInputs& p, int64_t c_base, int64_t nchunks, uint8_t* records,
+                                      int32_t* count, int2* list, cudaStream_t stream) {
+    const bool g_scalar = (p.in_flags & kInGScalar) != 0;
+    const bool pro = (p.in_flags & (kInNormQK | kInGLogits | kInBetaLogits)) != 0;
     auto prep = g_scalar ? (pro ? prep_kernel<true, true> : prep_kernel<true, false>)
                          : (pro ? prep_kernel<false, true> : prep_kernel<false, false>);
     auto strong = g_scalar ? prep_strong_kernel<true> : prep_strong_kernel<false>;
@@ -1605,41 +1705,37 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(strong, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StrongSmem::BYTES);
     if (e != cudaSuccess) return e;
+    e = launch_after(prep, dim3((unsigned)nchunks, (unsigned)p.H), dim3(kPrepThreads), PrepSmem::BYTES, stream,
+                     p.tq, p.tk, p.tv, p.tg, g_scalar ? p.g : nullptr, p.beta, p.num_seqs, p.H, p.off, p.tab,
+                     records, count, list, p.in_flags, p.total, (int)c_base);
+    if (e != cudaSuccess) return e;
+    const int sms = device_sm_count();
+    const int64_t sgrid = std::min<int64_t>(nchunks * p.H, sms > 0 ? sms : 148);
+    return launch_after(strong, dim3((unsigned)sgrid), dim3(kStrongThreads), StrongSmem::BYTES, stream,
+                        static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
+                        static_cast<const __nv_bfloat16*>(p.v), p.g, p.beta, p.num_seqs, p.H, p.tab, records,
+                        (const int32_t*)count, (const int2*)list, p.in_flags, p.total, (int)c_base);
+}
+
+inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const int32_t* cu, int num_seqs,
+                                  int64_t total, int H, void* workspace, cudaStream_t stream,
+                                  const int64_t* emit_pos = nullptr, int num_emit = 0,
+                                  uint32_t in_flags = 0) {
+    const Workspace w = split_workspace(workspace, total, num_seqs, H);
     chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off, w.tab,
-                                               num_emit > 0 ? w.etab : nullptr, w.strong_count);
+                                               num_emit > 0 ? w.etab : nullptr, w.strong_count, 1);
     if (num_emit > 0)
         emit_index_kernel<<<(num_emit + 255) / 256, 256, 0, stream>>>(cu, num_seqs, w.off, emit_pos,
                                                                        num_emit, w.etab);
-    if (total > 0) {
-        CUtensorMap tq, tk, tv, tg;
-        if (!make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tmap(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tmap(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            (!g_scalar &&
-             !make_tmap(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE)))
-            return cudaErrorInvalidValue;
-        if (g_scalar) tg = tq;   // a scalar gate is read with plain loads: this map goes unused
-        const int64_t units = max_chunks(total, num_seqs);
-        dim3 grid((unsigned)units, (unsigned)H);
-        e = launch_after(prep, grid, dim3(kPrepThreads), PrepSmem::BYTES, stream, tq, tk, tv, tg,
-                         g_scalar ? g : nullptr, beta, num_seqs, H, (const int32_t*)w.off, (const int2*)w.tab,
-                         w.records, w.strong_count, w.strong_units, in_flags, total);
-        if (e != cudaSuccess) return e;
-        const int sms = device_sm_count();
-        const int64_t sgrid = std::min<int64_t>(units * H, sms > 0 ? sms : 148);
-        e = launch_after(strong, dim3((unsigned)sgrid), dim3(kStrongThreads), StrongSmem::BYTES, stream,
-                         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                         static_cast<const __nv_bfloat16*>(v), g, beta, num_seqs, H, (const int2*)w.tab,
-                         w.records, (const int32_t*)w.strong_count, (const int2*)w.strong_units, in_flags, total);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || total == 0) return e;
+    PrepInputs p;
+    e = make_prep_inputs(&p, q, k, v, g, beta, num_seqs, total, H, w, in_flags);
+    if (e != cudaSuccess) return e;
+    return launch_prep_chunks(p, 0, max_chunks(total, num_seqs), w.records, w.strong_count, w.strong_units, stream);
 }
 
-// Chunk-serial recurrence and the chunk outputs: one CTA per (sequence, head), or, when a few
-// long chains would leave most SMs idle, the chunk-parallel scan over segments (segment
-// table, transitions, starting states, then the recurrence per segment).
-// emit_states (nullable) receives the states at the emission slots launch_prepare recorded.
 inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_seqs, int64_t total,
                                int H, void* workspace, cudaStream_t stream,
                                float* emit_states = nullptr, uint32_t in_flags = 0) {
@@ -1661,7 +1757,7 @@ inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_se
         return launch_after(rec, dim3((unsigned)(num_seqs * H * nsl)), dim3(kRecThreads), rec_smem, stream,
                             num_seqs, H, (const int32_t*)w.off, (const int2*)w.tab, (const uint8_t*)w.records, s0,
                             sf, o, et, emit_states, (const int4*)nullptr, (const int32_t*)nullptr,
-                            (const float*)nullptr);
+                            (const float*)nullptr, kWholeProblem);
     e = cudaFuncSetAttribute(seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SegSmem::BYTES);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombineSmem);
@@ -1675,21 +1771,68 @@ inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_se
     return launch_after(rec, dim3((unsigned)(w.max_segs * H * nsl)), dim3(kRecThreads), rec_smem, stream,
                         num_seqs, H, (const int32_t*)w.off, (const int2*)w.tab, (const uint8_t*)w.records, s0, sf,
                         o, et, emit_states, (const int4*)w.seg_tab, (const int32_t*)w.seg_count,
-                        (const float*)w.seg_states);
+                        (const float*)w.seg_states, kWholeProblem);
 }
 
+// The whole prefill.  window: chunks per window when the workspace holds fewer records than
+// the problem has chunks (window_chunks); the chunk-parallel scan runs only in one window.
 inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, const float* s0, const int32_t* cu,
                                   int num_seqs, int64_t total, int H, void* out, float* sf,
                                   void* workspace, cudaStream_t stream,
                                   const int64_t* emit_pos = nullptr, int num_emit = 0,
-                                  float* emit_states = nullptr, uint32_t in_flags = 0) {
-    cudaError_t e = launch_prepare(q, k, v, g, beta, cu, num_seqs, total, H, workspace, stream,
-                                   emit_pos, num_emit, in_flags);
-    if (e == cudaSuccess)
-        e = launch_scan(s0, sf, out, num_seqs, total, H, workspace, stream,
-                        num_emit > 0 ? emit_states : nullptr, in_flags);
-    return e;
+                                  float* emit_states = nullptr, uint32_t in_flags = 0,
+                                  int64_t window = INT64_MAX) {
+    const int64_t mc = max_chunks(total, num_seqs);
+    if (window >= mc) {
+        cudaError_t e = launch_prepare(q, k, v, g, beta, cu, num_seqs, total, H, workspace, stream,
+                                       emit_pos, num_emit, in_flags);
+        if (e == cudaSuccess)
+            e = launch_scan(s0, sf, out, num_seqs, total, H, workspace, stream,
+                            num_emit > 0 ? emit_states : nullptr, in_flags);
+        return e;
+    }
+    if (window <= 0 || num_seqs == 0) return cudaErrorInvalidValue;
+    const Workspace w = split_workspace(workspace, total, num_seqs, H);   // chunk offsets, table, slots
+    const WindowLayout l = window_layout(total, num_seqs, H, window);
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    int32_t* counts = reinterpret_cast<int32_t*>(base + l.counts);
+    int2* list = reinterpret_cast<int2*>(base + l.list);
+    float* carry = reinterpret_cast<float*>(base + l.carry);
+    uint8_t* records = base + l.records;
+    const int64_t nw = (mc + window - 1) / window;
+    chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off, w.tab,
+                                               num_emit > 0 ? w.etab : nullptr, counts, (int)nw);
+    if (num_emit > 0)
+        emit_index_kernel<<<(num_emit + 255) / 256, 256, 0, stream>>>(cu, num_seqs, w.off, emit_pos,
+                                                                       num_emit, w.etab);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    PrepInputs p;
+    if (total > 0 && (e = make_prep_inputs(&p, q, k, v, g, beta, num_seqs, total, H, w, in_flags)) != cudaSuccess)
+        return e;
+    const int sms = device_sm_count();
+    const bool narrow = (int64_t)num_seqs * H * RecCfg<32>::NSL <= (int64_t)(sms > 0 ? sms : 148);
+    auto rec = narrow ? rec_kernel<32> : rec_kernel<64>;
+    const uint32_t rec_smem = narrow ? RecCfg<32>::BYTES : RecCfg<64>::BYTES;
+    const int nsl = narrow ? RecCfg<32>::NSL : RecCfg<64>::NSL;
+    if ((e = cudaFuncSetAttribute(rec, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rec_smem)) != cudaSuccess)
+        return e;
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+    const size_t slot = (size_t)H * D * D;
+    for (int64_t wi = 0; wi < nw; ++wi) {
+        const int64_t c_lo = wi * window;
+        if (total > 0 && (e = launch_prep_chunks(p, c_lo, window, records, counts + wi, list, stream)) != cudaSuccess)
+            return e;
+        const RecWindow rw = {(int)c_lo, (int)std::min<int64_t>(c_lo + window, INT32_MAX), wi == nw - 1 ? 1 : 0,
+                              carry + (size_t)(wi & 1) * slot, carry + (size_t)((wi + 1) & 1) * slot};
+        e = launch_after(rec, dim3((unsigned)(num_seqs * H * nsl)), dim3(kRecThreads), rec_smem, stream, num_seqs,
+                         H, (const int32_t*)w.off, (const int2*)w.tab, (const uint8_t*)records, s0, sf, o,
+                         (const int32_t*)(num_emit > 0 ? w.etab : nullptr), num_emit > 0 ? emit_states : nullptr,
+                         (const int4*)nullptr, (const int32_t*)nullptr, (const float*)nullptr, rw);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 // One thread waits (bounded) on a barrier nothing arrives on and reports the expiry.

@@ -31,7 +31,7 @@ prep_strong_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
                    const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
                    const float* __restrict__ beta, int num_seqs, int H, const int2* __restrict__ tab,
                    uint8_t* __restrict__ records, const int32_t* __restrict__ strong_count,
-                   const int2* __restrict__ strong_units, uint32_t in_flags, int64_t total) {
+                   const int2* __restrict__ strong_units, uint32_t in_flags, int64_t total, int c_base) {
     using S = StrongSmem;
     constexpr int PK = S::PK, PC = S::PC;
     extern __shared__ __align__(16) float smf[];
@@ -64,7 +64,7 @@ prep_strong_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
             t0 = e.x;
             nrow = e.y;
         }
-        uint8_t* rec = records + ((size_t)c * H + h) * kRecBytes;
+        uint8_t* rec = records + ((size_t)(c - c_base) * H + h) * kRecBytes;   // the window's records
         auto at = [&](int r) { return ((size_t)(t0 + r) * H + h) * D; };
         __syncthreads();   // the previous unit is done with every buffer
 

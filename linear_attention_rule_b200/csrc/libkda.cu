@@ -45,7 +45,7 @@ cudaError_t dispatch_simt(int32_t dk, int32_t C, const void* q, const void* k, c
 
 extern "C" {
 
-int32_t kda_abi_version(void) { return 7; }
+int32_t kda_abi_version(void) { return 8; }
 
 const char* kda_status_string(kda_status s) {
     switch (s) {
@@ -68,6 +68,24 @@ size_t kda_prefill_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_
     if (!tensor_core_path(dt, dk)) return 0;
     size_t bytes = 0;
     return kda::tc::workspace_bytes_checked(total_tokens, num_seqs, H, &bytes) ? bytes : 0;
+}
+
+size_t kda_prefill_workspace_size_min(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
+                                      int32_t dv, int32_t C, kda_dtype dt) {
+    if (kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, dt) == 0) return 0;
+    return kda::tc::workspace_bytes_min(total_tokens, num_seqs, H);
+}
+
+int64_t kda_prefill_windows(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk, int32_t dv,
+                            int32_t C, kda_dtype dt, size_t ws_bytes) {
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0 || !supported_dim(dk, dv) || !valid_chunk(dt, C))
+        return -1;
+    if (!tensor_core_path(dt, dk) || num_seqs == 0) return 1;
+    if (kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, dt) == 0) return -1;
+    const int64_t w = kda::tc::window_chunks(total_tokens, num_seqs, H, ws_bytes);
+    if (w <= 0) return -1;
+    const int64_t mc = kda::tc::max_chunks(total_tokens, num_seqs);
+    return w >= mc ? 1 : (mc + w - 1) / w;
 }
 
 int32_t kda_prefill_launches(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
@@ -119,17 +137,24 @@ static kda_status prefill_common(const void* q, const void* k, const void* v, co
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return KDA_ERR_INVALID_ARG;
-    const size_t need = kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, dt);
+    // A workspace below the full size runs the chunks in windows (window_chunks), down to
+    // kda_prefill_workspace_size_min.
+    const size_t need = kda_prefill_workspace_size_min(total_tokens, num_seqs, H, dk, dv, C, dt);
     if (ws_bytes < need || (need > 0 && (!workspace ||
                                          (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)))
         return KDA_ERR_INVALID_ARG;
+    int64_t window = INT64_MAX;
+    if (tensor_core_path(dt, dk) && need > 0) {
+        window = kda::tc::window_chunks(total_tokens, num_seqs, H, ws_bytes);
+        if (window <= 0) return KDA_ERR_INVALID_ARG;
+    }
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t err;
     if (tensor_core_path(dt, dk))
         err = kda::tc::launch_prefill(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
                                       total_tokens, H, out, final_state, workspace, st, emit_pos,
-                                      num_emit, emit_states, in_flags);
+                                      num_emit, emit_states, in_flags, window);
     else if (dt == KDA_F32)
         err = dispatch_simt<float>(dk, C, q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
                                    total_tokens, H, out, final_state, st, in_flags);
@@ -389,7 +414,7 @@ extern "C" kda_status kda_prefill_noalloc(const void* q, const void* k, const vo
     if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (dt != KDA_BF16 || dk != 128 || dv != 128 || C != 64) return KDA_ERR_UNSUPPORTED;
     if (total_tokens > INT32_MAX || !tc_problem_fits(total_tokens, num_seqs, H)) return KDA_ERR_UNSUPPORTED;
-    const size_t need = kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, dt);
+    const size_t need = kda_prefill_workspace_size_min(total_tokens, num_seqs, H, dk, dv, C, dt);
     if (need == 0 || need > KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_UNSUPPORTED;
     if (num_seqs == 0) return KDA_OK;
     void* scratch = nullptr;

@@ -38,7 +38,8 @@ EXPORTED = ("kda_prefill", "kda_prefill_workspace_size", "kda_decode", "kda_stat
             "kda_get_device_status", "kda_abi_version", "kda_prefill_noalloc",
             "kda_prefill_prepare", "kda_prefill_scan", "kda_selftest_bounded_wait",
             "kda_prefill_emit", "kda_prefill_gdn", "kda_decode_gdn", "kda_prefill_ex",
-            "kda_decode_ex", "kda_prefill_launches")
+            "kda_decode_ex", "kda_prefill_launches", "kda_prefill_workspace_size_min",
+            "kda_prefill_windows")
 
 # Size of the library-owned scratch behind kda_prefill_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -66,6 +67,10 @@ def load() -> ctypes.CDLL:
     lib.kda_prefill.restype = ctypes.c_int
     lib.kda_prefill_workspace_size.argtypes = [I64, I32, I32, I32, I32, I32, ctypes.c_int]
     lib.kda_prefill_workspace_size.restype = SZ
+    lib.kda_prefill_workspace_size_min.argtypes = [I64, I32, I32, I32, I32, I32, ctypes.c_int]
+    lib.kda_prefill_workspace_size_min.restype = SZ
+    lib.kda_prefill_windows.argtypes = [I64, I32, I32, I32, I32, I32, ctypes.c_int, SZ]
+    lib.kda_prefill_windows.restype = I64
     lib.kda_decode.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, ctypes.c_int, P]
     lib.kda_decode.restype = ctypes.c_int
     lib.kda_status_string.argtypes = [ctypes.c_int]
@@ -199,6 +204,22 @@ def kda_prefill_workspace_size(total_tokens: int, num_seqs: int, H: int, dk: int
                                C: int, dtype: torch.dtype) -> int:
     code = KDA_F32 if dtype == torch.float32 else KDA_BF16
     return int(load().kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, C, code))
+
+
+def kda_prefill_workspace_size_min(total_tokens: int, num_seqs: int, H: int, dk: int, dv: int,
+                                   C: int, dtype: torch.dtype) -> int:
+    """The least workspace the prefill accepts; below kda_prefill_workspace_size it runs the
+    chunks in windows (kda_prefill_workspace_size_min in include/libkda.h)."""
+    code = KDA_F32 if dtype == torch.float32 else KDA_BF16
+    return int(load().kda_prefill_workspace_size_min(total_tokens, num_seqs, H, dk, dv, C, code))
+
+
+def kda_prefill_windows(total_tokens: int, num_seqs: int, H: int, dk: int, dv: int, C: int,
+                        dtype: torch.dtype, ws_bytes: int) -> int:
+    """Windows a prefill with a workspace of ws_bytes runs in (kda_prefill_windows in
+    include/libkda.h); -1 when the workspace is too small or the problem unsupported."""
+    code = KDA_F32 if dtype == torch.float32 else KDA_BF16
+    return int(load().kda_prefill_windows(total_tokens, num_seqs, H, dk, dv, C, code, ws_bytes))
 
 
 def kda_prefill(q, k, v, g, beta, cu_seqlens, out, initial_state=None, final_state=None,

@@ -46,7 +46,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert kda.kda_abi_version() == 7
+    assert kda.kda_abi_version() == 8
     for code in range(7):
         s = kda.kda_status_string(code)
         assert s and s != "unknown status"
@@ -86,7 +86,7 @@ def test_prefill_rejects_bad_arguments(lib):
 
 
 def test_prefill_workspace_check(lib):
-    need = lib.kda_prefill_workspace_size(8192, 1, 32, 128, 128, 64, kda.KDA_BF16)
+    need = lib.kda_prefill_workspace_size_min(8192, 1, 32, 128, 128, 64, kda.KDA_BF16)
     if need > 0:
         assert _prefill(lib, dk=128, dv=128, H=32, T=8192, dt=kda.KDA_BF16,
                         ws=ctypes.c_void_p(4096), ws_bytes=need - 1) == kda.KDA_ERR_INVALID_ARG
@@ -201,3 +201,39 @@ def test_prefill_launch_count(lib):
     assert n(8192, 0, 32) == 0
     assert n(256, 1, 2, dt=f32, d=64) == 1        # CUDA-core path: one kernel
     assert n(256, 1, 2, d=96) == -1
+
+
+REC = 90624   # bytes of one chunk record (one chunk of 64 tokens, one head)
+
+
+def test_window_workspace_sizes(lib):
+    """Below the full workspace the prefill runs in windows of W chunks: the least
+    workspace is windows of 8 chunks, and the count of windows follows from the bytes."""
+    bf = kda.KDA_BF16
+    full = lambda T, N, H: lib.kda_prefill_workspace_size(T, N, H, 128, 128, 64, bf)
+    least = lambda T, N, H: lib.kda_prefill_workspace_size_min(T, N, H, 128, 128, 64, bf)
+    win = lambda T, N, H, ws: lib.kda_prefill_windows(T, N, H, 128, 128, 64, bf, ws)
+    T, N, H = 8192, 1, 32
+    mc = T // 64 + N                                   # chunks the layout reserves
+    assert win(T, N, H, full(T, N, H)) == 1
+    lo = least(T, N, H)
+    # 8 chunks of records, two carried states per head, and per-chunk tables (16 B each)
+    records, carry = 8 * H * REC, 2 * H * 128 * 128 * 4
+    assert records + carry < lo < records + carry + 16 * mc + 64 * 1024
+    assert win(T, N, H, lo) == -(-mc // 8)
+    assert win(T, N, H, lo - 1) == -1
+    prev = None
+    for ws in (lo, lo + 5 * H * REC, lo + 40 * H * REC, full(T, N, H) - 1, full(T, N, H)):
+        n = win(T, N, H, ws)
+        assert n >= 1 and (prev is None or n <= prev)
+        prev = n
+    assert win(T, N, H, full(T, N, H) - 1) >= 2
+    # a problem of at most 8 chunks needs its full workspace
+    assert least(300, 1, 2) == full(300, 1, 2) and win(300, 1, 2, full(300, 1, 2)) == 1
+    # the full size grows with T, the least almost not (16 bytes per chunk)
+    assert full(1 << 20, 1, 32) > 40 * 10**9
+    assert least(1 << 20, 1, 32) - least(8192, 1, 32) == 16 * ((1 << 20) // 64 - 8192 // 64)
+    # paths that need no workspace
+    assert lib.kda_prefill_workspace_size_min(256, 1, 2, 64, 64, 64, kda.KDA_F32) == 0
+    assert lib.kda_prefill_windows(256, 1, 2, 64, 64, 64, kda.KDA_F32, 0) == 1
+    assert lib.kda_prefill_windows(256, 1, 2, 96, 96, 64, bf, 1 << 30) == -1
