@@ -477,6 +477,42 @@ def bench_crossover(args, dev, stream):
     return {"crossover": rows}
 
 
+def bench_windows(args, dev, stream):
+    """The cost of a bounded workspace: the prefill of configs 1 and 4 with workspaces from
+    the full size down to the allocation-free scratch (64 MiB), the chunks then running in
+    windows (kda_prefill_windows); bitwise the same results."""
+    import torch
+    from linear_attention_rule_b200 import kda
+    rows = []
+    for cfg_id in (1, 4):
+        P = setup_prefill(dev, 0, cfg_id)
+        d, T, N, H, D, C = P["d"], P["T"], P["N"], P["H"], P["D"], P["C"]
+        full = kda.kda_prefill_workspace_size(T, N, H, D, D, C, P["cfg"].dtype)
+        budgets = [full, 4 << 30, 1 << 30, 256 << 20, kda.NOALLOC_SCRATCH_BYTES]
+        P["ws"] = None
+        torch.cuda.empty_cache()
+        ws = torch.empty(full, dtype=torch.uint8, device=dev)
+        for b in budgets:
+            if b > full:
+                continue
+            n = kda.kda_prefill_windows(T, N, H, D, D, C, P["cfg"].dtype, b)
+            view = ws[:b]
+
+            def step():
+                kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], P["out"],
+                                initial_state=d["s0"], final_state=P["fin"], C=C, workspace=view, stream=stream)
+            for _ in range(args.warmup):
+                step()
+            steps = max(2, min(args.steps, int(2e7 // T) + 2))
+            ms, _, _ = timed(stream, dev, 1, steps, step)
+            assert kda.kda_get_device_status(stream) == kda.KDA_OK
+            rows.append({"workload": P["cfg"].name, "workspace_bytes": b, "windows": n, "ms": round(ms, 4),
+                         "tokens_per_s": round(T / (ms * 1e-3), 1)})
+        del P, ws, view
+        torch.cuda.empty_cache()
+    return {"windows": rows}
+
+
 def bench_gpu(args):
     import torch
     from linear_attention_rule_b200 import kda
@@ -512,6 +548,8 @@ def bench_gpu(args):
     line = {}
     if args.workload == "crossover":
         line = bench_crossover(args, dev, stream)
+    elif args.workload == "windows":
+        line = bench_windows(args, dev, stream)
     elif args.workload in ("config2", "config4"):
         P = setup_prefill(dev, rank, int(args.workload[-1]))
         pre = bench_prefill(args, P, dev, stream, world, peaks)
@@ -616,7 +654,7 @@ def main(argv=None):
     ap.add_argument("--no-extra-configs", action="store_true",
                     help="skip the varlen (config 2) and long-context (config 4) prefill entries")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--workload", choices=["all", "prefill", "decode", "config2", "config4", "crossover"],
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "config2", "config4", "crossover", "windows"],
                     default="all",
                     help="restrict the run (profiling) or measure another prefill config; "
                          "the driver's JSON line is 'all'")
