@@ -62,8 +62,10 @@ typedef enum {
 
 typedef enum {
     KDA_F32 = 0,   /* q, k, v, out in fp32: the CUDA-core (FFMA) chunked path */
-    KDA_BF16 = 1   /* q, k, v, out in bf16: the tensor-core (tcgen05) chunked path at
-                      dk = dv = 128, the CUDA-core path at 64 */
+    KDA_BF16 = 1   /* q, k, v, out in bf16: the tensor-core (tcgen05) chunked path; at
+                      dk = dv = 64 it runs as the first 64 channels of a 128-channel
+                      problem whose other channels are zero (same results, the cost of
+                      d = 128) */
 } kda_dtype;
 
 /*
@@ -196,7 +198,7 @@ kda_status kda_decode_gdn(const void *q, const void *k, const void *v, const flo
  * A position that is not such a boundary is reported on the device as KDA_ERR_BAD_EMIT_POS
  * and its slot is left as it was (with inconsistent cu_seqlens nothing is emitted).
  * num_seqs = 0 with num_emit > 0 is KDA_ERR_INVALID_ARG.
- * Tensor-core problems only (bf16, dk = dv = 128, C = 64): others return
+ * Tensor-core problems only (bf16, dk = dv = 128 or 64, C = 64): others return
  * KDA_ERR_UNSUPPORTED when num_emit > 0.  The workspace is kda_prefill's.
  */
 kda_status kda_prefill_emit(const void *q, const void *k, const void *v, const float *g,
@@ -268,7 +270,7 @@ kda_status kda_decode(const void *q, const void *k, const void *v, const float *
  * The chunkwise prefill as its two stages, for callers that schedule them separately
  * (for instance, preparing the next segment on one stream while another stream runs
  * the recurrence of the current one).  kda_prefill runs exactly these two in order.
- * Tensor-core problems only (bf16, dk = dv = 128, C = 64); anything else returns
+ * Tensor-core problems only (bf16, dk = dv = 128 or 64, C = 64); anything else returns
  * KDA_ERR_UNSUPPORTED.  Both take the same problem description and the same workspace,
  * which carries the chunk table and the chunk records from the first stage to the
  * second, and must run in this order (stream order, or events between streams):
@@ -313,7 +315,7 @@ kda_status kda_selftest_bounded_wait(uint64_t limit_ns, kda_stream_t stream);
  * cudaMalloc, cudaFree or any other allocating routine.
  *
  *   - Arguments and layouts are those of kda_prefill without workspace / ws_bytes.
- *   - Only the tensor-core problem (bf16, dk = dv = 128, C = 64) is served; any other
+ *   - Only tensor-core problems (bf16, dk = dv = 128 or 64, C = 64) are served; any other
  *     problem returns KDA_ERR_UNSUPPORTED (the CUDA-core path needs no scratch: call
  *     kda_prefill with a NULL workspace instead).  A dtype that is neither KDA_F32 nor
  *     KDA_BF16 is KDA_ERR_INVALID_ARG, as for every entry point.

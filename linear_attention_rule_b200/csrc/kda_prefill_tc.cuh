@@ -316,7 +316,8 @@ struct PrepSmem {
     static constexpr uint32_t ABAR = GR, AQK = GR + 8192, LI = GR + 16384;   // LI: [64][68]
     static constexpr uint32_t XCH = GR + 33792;      // decay partials [8][128]; later T [32][36]
     static constexpr uint32_t BETA = XCH + 4608;     // [64]
-    static constexpr uint32_t BAR = BETA + 256;       // g's TMA, then the products in order
+    static constexpr uint32_t DIAG = BETA + 256;      // [64] q_r . k_r in fp32 (Aqk's diagonal)
+    static constexpr uint32_t BAR = DIAG + 256;       // g's TMA, then the products in order
     static constexpr uint32_t BAR2 = BAR + 8;         // the last product (Aqk W)
     static constexpr uint32_t BARQK = BAR2 + 8;       // TMA of q and k
     static constexpr uint32_t BARV = BARQK + 8;       // TMA of v
@@ -353,7 +354,11 @@ constexpr float kStrongDecay = -64.f;
 // (token, head), g [T, H] (Gated DeltaNet, the scalar forget gate that KDA makes diagonal):
 // the same decay on every channel, loaded like beta instead of through the g tensor map.
 // kPrologue: in_flags may hold KDA_IN_* prologue bits (the plain path compiles without them).
-template <bool kScalarG, bool kPrologue>
+// DIN: channels per head of q, k, v and g, 128 or 64.  With 64 the chunk is prepared as the
+// first 64 channels of a 128-channel one whose other channels are zero (q = k = v = 0 and no
+// decay there): those channels add nothing to any product, so the records are the 128-channel
+// ones with zero halves, and the state's rows and columns from 64 on stay zero.
+template <bool kScalarG, bool kPrologue, int DIN>
 __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -415,19 +420,20 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(barv, 1);
         fence_mbar_init();
         *strong_flag = 0;
-        const int x0 = h * D;
-        if (!kScalarG) {
-            mbar_arrive_expect_tx(bar, kPrepTxG);
+        constexpr uint32_t halves = DIN / 64;   // 64-channel boxes per tensor
+        const int x0 = h * DIN;
+        if (!kScalarG) {   // the g tile lands as [64 rows][DIN] fp32
+            mbar_arrive_expect_tx(bar, kPrepTxG / 2 * halves);
             tma_load_2d(sb + S::GR, &tm_g, x0, t0, bar);
         }
-        mbar_arrive_expect_tx(barqk, kPrepTxQK);
+        mbar_arrive_expect_tx(barqk, kPrepTxQK / 2 * halves);
         tma_load_2d(sb + S::QD0, &tm_q, x0, t0, barqk);
-        tma_load_2d(sb + S::QD1, &tm_q, x0 + 64, t0, barqk);
+        if (DIN == 128) tma_load_2d(sb + S::QD1, &tm_q, x0 + 64, t0, barqk);
         tma_load_2d(sb + S::KD0, &tm_k, x0, t0, barqk);
-        tma_load_2d(sb + S::KD1, &tm_k, x0 + 64, t0, barqk);
-        mbar_arrive_expect_tx(barv, kPrepTxV);
+        if (DIN == 128) tma_load_2d(sb + S::KD1, &tm_k, x0 + 64, t0, barqk);
+        mbar_arrive_expect_tx(barv, kPrepTxV / 2 * halves);
         tma_load_2d(sb + S::V0, &tm_v, x0, t0, barv);
-        tma_load_2d(sb + S::V1, &tm_v, x0 + 64, t0, barv);
+        if (DIN == 128) tma_load_2d(sb + S::V1, &tm_v, x0 + 64, t0, barv);
     }
     if (warp == 1) tmem_alloc(sb + S::TMEM, kPrepTmemCols);
     if (tid < C) {
@@ -470,15 +476,18 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if constexpr (kScalarG) {
 #pragma unroll
                 for (int u = 0; u < 8; ++u) gv[u] = gt[r];
-            } else {
-                const float4 g0 = *reinterpret_cast<const float4*>(gt + r * D + 8 * cg);
-                const float4 g1 = *reinterpret_cast<const float4*>(gt + r * D + 8 * cg + 4);
+            } else if (DIN == 128 || cg < 8) {
+                const float4 g0 = *reinterpret_cast<const float4*>(gt + r * DIN + 8 * cg);
+                const float4 g1 = *reinterpret_cast<const float4*>(gt + r * DIN + 8 * cg + 4);
                 gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w;
                 gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
                 if (in_flags & kInGLogits) {
 #pragma unroll
                     for (int u = 0; u < 8; ++u) gv[u] = kda_logsigmoid(gv[u]);
                 }
+            } else {   // channels without input: no decay
+#pragma unroll
+                for (int u = 0; u < 8; ++u) gv[u] = 0.f;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -534,8 +543,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int r = 4 * rb + rr;
             const uint32_t o = kb * S::BLK + sw128_off(r, c8);
             float qv[8], kv[8], qd[8], kd[8], ki[8];
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + o), qv);
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::KD0 + o), kv);
+            if (DIN == 128 || kb == 0) {
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::QD0 + o), qv);
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + S::KD0 + o), kv);
+            } else {   // channels 64..127 of a 64-channel input: zero, and so is v there
+#pragma unroll
+                for (int u = 0; u < 8; ++u) qv[u] = kv[u] = 0.f;
+                *reinterpret_cast<uint4*>(sm + S::V0 + o) = make_uint4(0u, 0u, 0u, 0u);
+            }
             if (in_flags & kInNormQK) {   // the 16 lanes of this half-warp hold the row's 128 channels
                 float sq = 0.f, sk = 0.f;
 #pragma unroll
@@ -550,6 +565,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 for (int u = 0; u < 8; ++u) { qv[u] *= iq; kv[u] *= ik; }
             }
             const bool live = r < nrow;
+            {   // Aqk's diagonal needs no decay (e^{a_r - a_r} = 1): q_r . k_r in fp32 from the
+                // inputs, where the bf16 images' roundings would spoil a q . k that cancels
+                float dg = 0.f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) dg = fmaf(qv[u], kv[u], dg);
+#pragma unroll
+                for (int o2 = 1; o2 < 16; o2 <<= 1) dg += __shfl_xor_sync(0xffffffffu, dg, o2);
+                if (cg == 0) reinterpret_cast<float*>(sm + S::DIAG)[r] = live ? dg : 0.f;
+            }
             // a scalar gate gives every channel the same decay: two exponentials per row
             const float ep0 = __expf(base[0] + loc[rr][0]), em0 = __expf(-(base[0] + loc[rr][0]));
 #pragma unroll
@@ -609,15 +633,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     *reinterpret_cast<float4*>(sLI + r * kLP + 32 * wh + 4 * u4) =
                         make_float4(e[0], e[1], e[2], e[3]);
                 }
-            } else {        // Aqk[r][s] = (Q_dec K_inv^T)[r][s] for s <= r (bf16 image)
+            } else {        // Aqk[r][s] = (Q_dec K_inv^T)[r][s] for s < r, q_r . k_r for s = r (bf16 image)
                 const int r = 32 * (wq - 2) + lane;
+                const float dg = reinterpret_cast<const float*>(sm + S::DIAG)[r];
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
                     float e[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int s = 32 * wh + 8 * qq + u;
-                        e[u] = s <= r ? d[8 * qq + u] : 0.f;
+                        e[u] = s < r ? d[8 * qq + u] : (s == r ? dg : 0.f);
                     }
                     *reinterpret_cast<uint4*>(sm + S::AQK + sw128_off(r, 4 * wh + qq)) = pack_bf16x8(e);
                 }
@@ -998,7 +1023,10 @@ struct RecWindow {
 };
 constexpr RecWindow kWholeProblem = {0, INT32_MAX, 1, nullptr, nullptr};
 
-template <int NV>
+// DIN: channels per head of the caller's outputs and states (128, or 64 with the chunk
+// tensors of a 128-channel problem whose channels from 64 on are zero: only the value slices
+// of the first 64 columns run, and only the state's first 64 rows are read or written).
+template <int NV, int DIN>
 __global__ void __launch_bounds__(kRecThreads, 1)
 rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __restrict__ tab,
            const uint8_t* __restrict__ records, const float* initial_state, float* final_state,
@@ -1006,7 +1034,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
            const int4* __restrict__ seg_tab, const int32_t* __restrict__ seg_count,
            const float* __restrict__ seg_states, RecWindow win) {
     using S = RecCfg<NV>;
-    constexpr int NSL = S::NSL;
+    constexpr int NSL = DIN / NV;   // value slices of the caller's columns
     (void)num_seqs;
     kda_grid_wait();   // the chunk table and the records
     const int sl = blockIdx.x % NSL;
@@ -1015,6 +1043,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
     int n, c_begin, nchunks;
     bool write_final = final_state != nullptr;
     const float* s_init;
+    int s_ld = DIN;             // row length of s_init
     float* s_carry = nullptr;   // where the state goes when the sequence continues past the window
     if (seg_tab) {
         if (unit >= *seg_count) return;   // the whole CTA, before any barrier
@@ -1023,9 +1052,10 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
         c_begin = sg.y;
         nchunks = sg.z;
         write_final = write_final && (sg.w >> 16) != 0;
-        s_init = (sg.w & 0xFFFF) == 0
-                     ? (initial_state ? initial_state + ((size_t)n * H + h) * D * D : nullptr)
-                     : seg_states + ((size_t)unit * H + h) * (kSegStateBytes / sizeof(float)) + 2 * D * D;
+        const bool first = (sg.w & 0xFFFF) == 0;
+        s_init = first ? (initial_state ? initial_state + ((size_t)n * H + h) * DIN * DIN : nullptr)
+                       : seg_states + ((size_t)unit * H + h) * (kSegStateBytes / sizeof(float)) + 2 * D * D;
+        if (!first) s_ld = D;
     } else {
         // this sequence's chunks inside the window [c_lo, c_hi)
         n = unit;
@@ -1040,11 +1070,11 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
             nchunks = 0;
         }
         const bool starts_here = a >= win.c_lo;
-        s_init = starts_here ? (initial_state ? initial_state + ((size_t)n * H + h) * D * D : nullptr)
-                             : win.carry_in + (size_t)h * D * D;
+        s_init = starts_here ? (initial_state ? initial_state + ((size_t)n * H + h) * DIN * DIN : nullptr)
+                             : win.carry_in + (size_t)h * DIN * DIN;
         if (b > win.c_hi) {
             write_final = false;
-            s_carry = win.carry_out + (size_t)h * D * D;
+            s_carry = win.carry_out + (size_t)h * DIN * DIN;
         }
     }
     auto record = [&](int kk) { return records + ((size_t)(c_begin + kk - win.c_lo) * H + h) * kRecBytes; };
@@ -1147,10 +1177,10 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
         const size_t col0 = (size_t)sl * NV + NC * cw;
         const int r_out = 16 * q4 + lane;   // output row of this lane (lanes 0-15)
         float Sr[NC];
-        if (s_init) {
+        if (s_init && i < DIN) {
 #pragma unroll
             for (int j4 = 0; j4 < NC / 4; ++j4) {
-                const float4 t = reinterpret_cast<const float4*>(s_init + (size_t)i * D + col0)[j4];
+                const float4 t = reinterpret_cast<const float4*>(s_init + (size_t)i * s_ld + col0)[j4];
                 Sr[4 * j4] = t.x; Sr[4 * j4 + 1] = t.y; Sr[4 * j4 + 2] = t.z; Sr[4 * j4 + 3] = t.w;
             }
         } else {
@@ -1212,8 +1242,8 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
             // D_O(kk-1), drained below in the previous pass) are complete
             if (more) put_state((kk + 1) & 1);
             KDA_TRACE_POINT(tr, 16 * kk + 4);
-            if (e_slot >= 0) {   // emission boundary at the end of this chunk: the fp32 state as it is
-                float* dst = emit_states + ((size_t)e_slot * H + h) * D * D + (size_t)i * D + col0;
+            if (e_slot >= 0 && i < DIN) {   // emission boundary at the end of this chunk: the state as it is
+                float* dst = emit_states + ((size_t)e_slot * H + h) * DIN * DIN + (size_t)i * DIN + col0;
 #pragma unroll
                 for (int j4 = 0; j4 < NC / 4; ++j4)
                     reinterpret_cast<float4*>(dst)[j4] =
@@ -1249,7 +1279,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
                 for (int g = 0; g < 16 / RPI; ++g) {
                     const int rr = 16 * q4 + RPI * g + lane / LPR;
                     if (rr < ce.y)
-                        *reinterpret_cast<uint4*>(out + ((size_t)(ce.x + rr) * H + h) * D + sl * NV + NC * cw +
+                        *reinterpret_cast<uint4*>(out + ((size_t)(ce.x + rr) * H + h) * DIN + sl * NV + NC * cw +
                                                   8 * (lane % LPR)) = ov[g];
                 }
             }
@@ -1259,8 +1289,8 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
         if (!ok) {
             if (lane == 0) kda_set_status(KDA_ERR_TIMEOUT);
             *abort_flag = 1;
-        } else if (write_final || s_carry) {
-            float* dst = (s_carry ? s_carry : final_state + ((size_t)n * H + h) * D * D) + (size_t)i * D + col0;
+        } else if ((write_final || s_carry) && i < DIN) {
+            float* dst = (s_carry ? s_carry : final_state + ((size_t)n * H + h) * DIN * DIN) + (size_t)i * DIN + col0;
 #pragma unroll
             for (int j4 = 0; j4 < NC / 4; ++j4)
                 reinterpret_cast<float4*>(dst)[j4] =
@@ -1584,11 +1614,11 @@ inline EncodeTiledFn encode_tiled() {
 
 // Rows = tokens (T), columns = H*D elements; box = 64 tokens x `box_cols` columns.
 inline bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, size_t elem,
-                      int64_t T, int H, uint32_t box_cols, CUtensorMapSwizzle sw) {
+                      int64_t T, int H, uint32_t box_cols, CUtensorMapSwizzle sw, int din = D) {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)H * D, (cuuint64_t)T};
-    const cuuint64_t strides[1] = {(cuuint64_t)H * D * elem};
+    const cuuint64_t dims[2] = {(cuuint64_t)H * din, (cuuint64_t)T};
+    const cuuint64_t strides[1] = {(cuuint64_t)H * din * elem};
     const cuuint32_t box[2] = {box_cols, (cuuint32_t)C};
     const cuuint32_t es[2] = {1, 1};
     return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1674,18 +1704,22 @@ struct PrepInputs {
     const int32_t* off;
     const int2* tab;
     uint32_t in_flags;
+    int din;   // channels per head of q, k, v, g: 128 or 64
 };
 inline cudaError_t make_prep_inputs(PrepInputs* p, const void* q, const void* k, const void* v, const float* g,
                                     const float* beta, int num_seqs, int64_t total, int H, const Workspace& w,
-                                    uint32_t in_flags) {
+                                    uint32_t in_flags, int din) {
     const bool g_scalar = (in_flags & kInGScalar) != 0;
     *p = PrepInputs{};
     p->q = q; p->k = k; p->v = v; p->g = g; p->beta = beta;
     p->num_seqs = num_seqs; p->H = H; p->total = total; p->off = w.off; p->tab = w.tab; p->in_flags = in_flags;
-    if (!make_tmap(&p->tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap(&p->tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap(&p->tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        (!g_scalar && !make_tmap(&p->tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE)))
+    p->din = din;
+    const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_tmap(&p->tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, sw, din) ||
+        !make_tmap(&p->tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, sw, din) ||
+        !make_tmap(&p->tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64, sw, din) ||
+        (!g_scalar && !make_tmap(&p->tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, (uint32_t)din,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE, din)))
         return cudaErrorInvalidValue;
     if (g_scalar) p->tg = p->tq;   // a scalar gate is read with plain loads: this map goes unused
     return cudaSuccess;
@@ -1697,9 +1731,13 @@ inline cudaError_t launch_prep_chunks(const PrepInputs& p, int64_t c_base, int64
                                       int32_t* count, int2* list, cudaStream_t stream) {
     const bool g_scalar = (p.in_flags & kInGScalar) != 0;
     const bool pro = (p.in_flags & (kInNormQK | kInGLogits | kInBetaLogits)) != 0;
-    auto prep = g_scalar ? (pro ? prep_kernel<true, true> : prep_kernel<true, false>)
-                         : (pro ? prep_kernel<false, true> : prep_kernel<false, false>);
-    auto strong = g_scalar ? prep_strong_kernel<true> : prep_strong_kernel<false>;
+    const bool d64 = p.din == 64;
+    auto prep = d64 ? (g_scalar ? (pro ? prep_kernel<true, true, 64> : prep_kernel<true, false, 64>)
+                                : (pro ? prep_kernel<false, true, 64> : prep_kernel<false, false, 64>))
+                    : (g_scalar ? (pro ? prep_kernel<true, true, 128> : prep_kernel<true, false, 128>)
+                                : (pro ? prep_kernel<false, true, 128> : prep_kernel<false, false, 128>));
+    auto strong = d64 ? (g_scalar ? prep_strong_kernel<true, 64> : prep_strong_kernel<false, 64>)
+                      : (g_scalar ? prep_strong_kernel<true, 128> : prep_strong_kernel<false, 128>);
     cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PrepSmem::BYTES);
     if (e == cudaSuccess)
@@ -1717,11 +1755,28 @@ inline cudaError_t launch_prep_chunks(const PrepInputs& p, int64_t c_base, int64
                         (const int32_t*)count, (const int2*)list, p.in_flags, p.total, (int)c_base);
 }
 
+// The recurrence for `chains` (sequence or segment, head) chains of head width din: value
+// slices of 32 columns while all their CTAs fit on the SMs at once, else of 64.
+struct RecLaunch {
+    void (*kernel)(int, int, const int32_t*, const int2*, const uint8_t*, const float*, float*,
+                   __nv_bfloat16*, const int32_t*, float*, const int4*, const int32_t*, const float*,
+                   RecWindow);
+    uint32_t smem;
+    int nsl;   // CTAs per chain
+};
+inline RecLaunch pick_rec(int64_t chains, int din) {
+    const int sms = device_sm_count();
+    const bool narrow = chains * (din / 32) <= (int64_t)(sms > 0 ? sms : 148);
+    if (din == 64)
+        return narrow ? RecLaunch{rec_kernel<32, 64>, RecCfg<32>::BYTES, 2} : RecLaunch{rec_kernel<64, 64>, RecCfg<64>::BYTES, 1};
+    return narrow ? RecLaunch{rec_kernel<32, 128>, RecCfg<32>::BYTES, 4} : RecLaunch{rec_kernel<64, 128>, RecCfg<64>::BYTES, 2};
+}
+
 inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, const int32_t* cu, int num_seqs,
                                   int64_t total, int H, void* workspace, cudaStream_t stream,
                                   const int64_t* emit_pos = nullptr, int num_emit = 0,
-                                  uint32_t in_flags = 0) {
+                                  uint32_t in_flags = 0, int din = D) {
     const Workspace w = split_workspace(workspace, total, num_seqs, H);
     chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off, w.tab,
                                                num_emit > 0 ? w.etab : nullptr, w.strong_count, 1);
@@ -1731,26 +1786,25 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || total == 0) return e;
     PrepInputs p;
-    e = make_prep_inputs(&p, q, k, v, g, beta, num_seqs, total, H, w, in_flags);
+    e = make_prep_inputs(&p, q, k, v, g, beta, num_seqs, total, H, w, in_flags, din);
     if (e != cudaSuccess) return e;
     return launch_prep_chunks(p, 0, max_chunks(total, num_seqs), w.records, w.strong_count, w.strong_units, stream);
 }
 
 inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_seqs, int64_t total,
                                int H, void* workspace, cudaStream_t stream,
-                               float* emit_states = nullptr, uint32_t in_flags = 0) {
+                               float* emit_states = nullptr, uint32_t in_flags = 0, int din = D) {
     const Workspace w = split_workspace(workspace, total, num_seqs, H);
     if ((int64_t)num_seqs * H == 0) return cudaSuccess;
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
     const int32_t* et = emit_states ? w.etab : nullptr;
-    const bool scan = w.seg > 0 && !(in_flags & kInSerialChains);
+    // the chunk-parallel scan serves 128-channel heads only
+    const bool scan = w.seg > 0 && !(in_flags & kInSerialChains) && din == D;
     const int64_t units = scan ? w.max_segs : num_seqs;   // chains: sequences, or scan segments
-    // 32-channel value slices while four CTAs per chain fit on the SMs at once, else 64
-    const int sms = device_sm_count();
-    const bool narrow = units * H * RecCfg<32>::NSL <= (int64_t)(sms > 0 ? sms : 148);
-    auto rec = narrow ? rec_kernel<32> : rec_kernel<64>;
-    const uint32_t rec_smem = narrow ? RecCfg<32>::BYTES : RecCfg<64>::BYTES;
-    const int nsl = narrow ? RecCfg<32>::NSL : RecCfg<64>::NSL;
+    const RecLaunch rl = pick_rec(units * H, din);
+    auto rec = rl.kernel;
+    const uint32_t rec_smem = rl.smem;
+    const int nsl = rl.nsl;
     cudaError_t e = cudaFuncSetAttribute(rec, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rec_smem);
     if (e != cudaSuccess) return e;
     if (!scan)
@@ -1782,14 +1836,14 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
                                   void* workspace, cudaStream_t stream,
                                   const int64_t* emit_pos = nullptr, int num_emit = 0,
                                   float* emit_states = nullptr, uint32_t in_flags = 0,
-                                  int64_t window = INT64_MAX) {
+                                  int64_t window = INT64_MAX, int din = D) {
     const int64_t mc = max_chunks(total, num_seqs);
     if (window >= mc) {
         cudaError_t e = launch_prepare(q, k, v, g, beta, cu, num_seqs, total, H, workspace, stream,
-                                       emit_pos, num_emit, in_flags);
+                                       emit_pos, num_emit, in_flags, din);
         if (e == cudaSuccess)
             e = launch_scan(s0, sf, out, num_seqs, total, H, workspace, stream,
-                            num_emit > 0 ? emit_states : nullptr, in_flags);
+                            num_emit > 0 ? emit_states : nullptr, in_flags, din);
         return e;
     }
     if (window <= 0 || num_seqs == 0) return cudaErrorInvalidValue;
@@ -1809,17 +1863,16 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     PrepInputs p;
-    if (total > 0 && (e = make_prep_inputs(&p, q, k, v, g, beta, num_seqs, total, H, w, in_flags)) != cudaSuccess)
+    if (total > 0 && (e = make_prep_inputs(&p, q, k, v, g, beta, num_seqs, total, H, w, in_flags, din)) != cudaSuccess)
         return e;
-    const int sms = device_sm_count();
-    const bool narrow = (int64_t)num_seqs * H * RecCfg<32>::NSL <= (int64_t)(sms > 0 ? sms : 148);
-    auto rec = narrow ? rec_kernel<32> : rec_kernel<64>;
-    const uint32_t rec_smem = narrow ? RecCfg<32>::BYTES : RecCfg<64>::BYTES;
-    const int nsl = narrow ? RecCfg<32>::NSL : RecCfg<64>::NSL;
+    const RecLaunch rl = pick_rec((int64_t)num_seqs * H, din);
+    auto rec = rl.kernel;
+    const uint32_t rec_smem = rl.smem;
+    const int nsl = rl.nsl;
     if ((e = cudaFuncSetAttribute(rec, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rec_smem)) != cudaSuccess)
         return e;
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
-    const size_t slot = (size_t)H * D * D;
+    const size_t slot = (size_t)H * din * din;   // one carried state per head
     for (int64_t wi = 0; wi < nw; ++wi) {
         const int64_t c_lo = wi * window;
         if (total > 0 && (e = launch_prep_chunks(p, c_lo, window, records, counts + wi, list, stream)) != cudaSuccess)

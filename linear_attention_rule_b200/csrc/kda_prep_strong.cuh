@@ -24,8 +24,9 @@ struct StrongSmem {   // fp32 words
     static_assert(BYTES <= 232448, "strong-decay preparation shared memory exceeds 227 KB");
 };
 
-// Persistent over the listed (chunk, head) units.  kScalarG / in_flags as in prep_kernel.
-template <bool kScalarG>
+// Persistent over the listed (chunk, head) units.  kScalarG / in_flags as in prep_kernel;
+// DIN: channels per head of q, k, v and g (64: the channels from 64 on are zero).
+template <bool kScalarG, int DIN>
 __global__ void __launch_bounds__(kStrongThreads, 1)
 prep_strong_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                    const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
@@ -65,14 +66,14 @@ prep_strong_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
             nrow = e.y;
         }
         uint8_t* rec = records + ((size_t)(c - c_base) * H + h) * kRecBytes;   // the window's records
-        auto at = [&](int r) { return ((size_t)(t0 + r) * H + h) * D; };
+        auto at = [&](int r) { return ((size_t)(t0 + r) * H + h) * DIN; };
         __syncthreads();   // the previous unit is done with every buffer
 
         // (1) gate, beta and the row norms of the input prologue
         for (int e = tid; e < C * D; e += kStrongThreads) {
             const int r = e / D, ch = e % D;
             float x = 0.f;
-            if (r < nrow) {
+            if (r < nrow && (kScalarG || ch < DIN)) {
                 x = kScalarG ? g[(size_t)(t0 + r) * H + h] : g[at(r) + ch];
                 if (in_flags & kInGLogits) x = kda_logsigmoid(x);
             }
@@ -85,7 +86,7 @@ prep_strong_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
         for (int r = warp; r < C; r += kStrongThreads / 32) {
             float sq = 0.f, sk = 0.f;
             if (r < nrow && (in_flags & kInNormQK)) {
-                for (int ch = lane; ch < D; ch += 32) {
+                for (int ch = lane; ch < DIN; ch += 32) {
                     const float qq = __bfloat162float(q[at(r) + ch]), kk = __bfloat162float(k[at(r) + ch]);
                     sq += qq * qq;
                     sk += kk * kk;
@@ -102,13 +103,17 @@ prep_strong_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
             }
         }
         __syncthreads();
-        auto load_q = [&](int r, int ch) { return r < nrow ? __bfloat162float(q[at(r) + ch]) * sNq[r] : 0.f; };
-        auto load_k = [&](int r, int ch) { return r < nrow ? __bfloat162float(k[at(r) + ch]) * sNk[r] : 0.f; };
+        auto load_q = [&](int r, int ch) {
+            return r < nrow && ch < DIN ? __bfloat162float(q[at(r) + ch]) * sNq[r] : 0.f;
+        };
+        auto load_k = [&](int r, int ch) {
+            return r < nrow && ch < DIN ? __bfloat162float(k[at(r) + ch]) * sNk[r] : 0.f;
+        };
         for (int e = tid; e < C * D; e += kStrongThreads) {
             const int r = e / D, ch = e % D;
             sQ[r * PK + ch] = load_q(r, ch);
             sK[r * PK + ch] = load_k(r, ch);
-            sV[r * PK + ch] = r < nrow ? __bfloat162float(v[at(r) + ch]) : 0.f;
+            sV[r * PK + ch] = r < nrow && ch < DIN ? __bfloat162float(v[at(r) + ch]) : 0.f;
         }
         // (2) inclusive cumulative log-decay per channel, gamma = e^{a_last}
         for (int ch = tid; ch < D; ch += kStrongThreads) {

@@ -18,8 +18,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool supported_dim(int32_t dk, int32_t dv) { return dk == dv && (dk == 64 || dk == 128); }
 
-// bf16 with d = 128 runs on the tensor cores; fp32 (and bf16 with d = 64) on CUDA cores.
-bool tensor_core_path(kda_dtype dt, int32_t dk) { return dt == KDA_BF16 && dk == 128; }
+// bf16 runs on the tensor cores (d = 64 as the first 64 channels of a 128-channel problem);
+// fp32 on CUDA cores.
+bool tensor_core_path(kda_dtype dt, int32_t dk) { return dt == KDA_BF16 && (dk == 128 || dk == 64); }
 
 bool valid_chunk(kda_dtype dt, int32_t C) {
     if (dt == KDA_BF16) return C == 64;
@@ -96,7 +97,7 @@ int32_t kda_prefill_launches(int64_t total_tokens, int32_t num_seqs, int32_t H, 
     if (!tensor_core_path(dt, dk)) return 1;
     // chunk table, [emission slots], preparation, strongly decayed chunks, recurrence
     int32_t n = 1 + (num_emit > 0 ? 1 : 0) + (total_tokens > 0 ? 2 : 0) + 1;
-    if (!(in_flags & KDA_IN_SERIAL_CHAINS) && kda::tc::scan_segment_chunks(total_tokens, num_seqs, H) > 0)
+    if (!(in_flags & KDA_IN_SERIAL_CHAINS) && dk == 128 && kda::tc::scan_segment_chunks(total_tokens, num_seqs, H) > 0)
         n += 3;   // segment table, segment transitions, starting states
     return n;
 }
@@ -154,13 +155,12 @@ static kda_status prefill_common(const void* q, const void* k, const void* v, co
     if (tensor_core_path(dt, dk))
         err = kda::tc::launch_prefill(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
                                       total_tokens, H, out, final_state, workspace, st, emit_pos,
-                                      num_emit, emit_states, in_flags, window);
+                                      num_emit, emit_states, in_flags, window, dk);
     else if (dt == KDA_F32)
         err = dispatch_simt<float>(dk, C, q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
                                    total_tokens, H, out, final_state, st, in_flags);
     else
-        err = dispatch_simt<__nv_bfloat16>(dk, C, q, k, v, g, beta, initial_state, cu_seqlens,
-                                           num_seqs, total_tokens, H, out, final_state, st, in_flags);
+        return KDA_ERR_UNSUPPORTED;   // unreachable: every bf16 problem takes the tensor cores
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -237,7 +237,7 @@ kda_status kda_prefill_prepare(const void* q, const void* k, const void* v, cons
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
     return kda::tc::launch_prepare(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, H, workspace,
-                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                                   reinterpret_cast<cudaStream_t>(stream), nullptr, 0, 0u, dk) == cudaSuccess
                ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -251,7 +251,7 @@ kda_status kda_prefill_scan(const float* initial_state, float* final_state, void
         return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!out || !aligned16(out))) return KDA_ERR_INVALID_ARG;
     return kda::tc::launch_scan(initial_state, final_state, out, num_seqs, total_tokens, H,
-                                workspace, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                                workspace, reinterpret_cast<cudaStream_t>(stream), nullptr, 0u, dk) == cudaSuccess
                ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -412,7 +412,7 @@ extern "C" kda_status kda_prefill_noalloc(const void* q, const void* k, const vo
                                           float* final_state, int32_t C, kda_stream_t stream) {
     if (num_seqs < 0 || total_tokens < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
     if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
-    if (dt != KDA_BF16 || dk != 128 || dv != 128 || C != 64) return KDA_ERR_UNSUPPORTED;
+    if (dt != KDA_BF16 || !tensor_core_path(dt, dk) || dv != dk || C != 64) return KDA_ERR_UNSUPPORTED;
     if (total_tokens > INT32_MAX || !tc_problem_fits(total_tokens, num_seqs, H)) return KDA_ERR_UNSUPPORTED;
     const size_t need = kda_prefill_workspace_size_min(total_tokens, num_seqs, H, dk, dv, C, dt);
     if (need == 0 || need > KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_UNSUPPORTED;

@@ -150,7 +150,7 @@ def test_emit_entry_point_rejects_bad_arguments(lib):
     assert emit(st=P(8200)) == kda.KDA_ERR_INVALID_ARG        # emit_states 16-byte aligned
     assert emit(N=0) == kda.KDA_ERR_INVALID_ARG               # positions but no sequence
     assert emit(dt=kda.KDA_F32) == kda.KDA_ERR_UNSUPPORTED    # emission: tensor-core path only
-    assert emit(dk=64) == kda.KDA_ERR_UNSUPPORTED
+    assert emit(dk=96) == kda.KDA_ERR_UNSUPPORTED
     assert kda.kda_status_string(kda.KDA_ERR_BAD_EMIT_POS) != "unknown status"
 
 
@@ -200,6 +200,8 @@ def test_prefill_launch_count(lib):
     assert n(0, 1, 32) == 2                       # chunk table and recurrence only
     assert n(8192, 0, 32) == 0
     assert n(256, 1, 2, dt=f32, d=64) == 1        # CUDA-core path: one kernel
+    assert n(256, 1, 2, d=64) == 4                # bf16 at d = 64: the tensor-core kernels
+    assert n(1 << 20, 1, 8, d=64) == 4            # no chunk-parallel scan at d = 64
     assert n(256, 1, 2, d=96) == -1
 
 

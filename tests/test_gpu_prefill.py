@@ -171,6 +171,38 @@ def test_bf16_d64():
     check_prefill(inp, out, fin)
 
 
+def test_bf16_d64_tensor_core_path_windows_emission_strong_decay():
+    """bf16 at d = 64 runs on the tensor-core kernels as the first 64 channels of a
+    128-channel problem: against the oracle per slice and per chunk, with mild and strong
+    decay (g = logsigmoid(N(3, 1)) and logsigmoid(N(-3, 1))); in windows of chunks and with
+    state emission, bit for bit the same as in one window."""
+    lens, H = [700, 0, 333, 64, 1300], 3
+    for g_mean, seed in ((3.0, 31), (-3.0, 32)):
+        inp = synthetic.make_prefill_inputs(lens, H, 64, 64, torch.bfloat16, g_mean, 0.02, seed)
+        out, fin = run_prefill(inp, C=64, in_flags=kda.KDA_IN_SERIAL_CHAINS)
+        check_prefill(inp, out, fin, chunk=64)
+        T, N = sum(lens), len(lens)
+        least = kda.kda_prefill_workspace_size_min(T, N, H, 64, 64, 64, torch.bfloat16)
+        ws = torch.empty(least + 4 * H * (90624 + 8) + 2048, dtype=torch.uint8, device="cuda")
+        assert kda.kda_prefill_windows(T, N, H, 64, 64, 64, torch.bfloat16, ws.numel()) > 2
+        d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+        pos = torch.tensor([64, 700, 700 + 320, 1097, 1097 + 1280], dtype=torch.int64, device="cuda")
+        res = []
+        for workspace in (None, ws):
+            o = torch.full((T, H, 64), float("nan"), dtype=torch.bfloat16, device="cuda")
+            f = torch.full((N, H, 64, 64), float("nan"), device="cuda")
+            e = torch.full((pos.shape[0], H, 64, 64), float("nan"), device="cuda")
+            kda.kda_prefill_emit(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], o, pos, e,
+                                 initial_state=d["s0"], final_state=f, workspace=workspace)
+            assert kda.kda_get_device_status() == kda.KDA_OK
+            res.append([x.double().cpu().numpy() for x in (o, f, e)])
+        for a, b in zip(*res):
+            np.testing.assert_array_equal(b, a)
+        np.testing.assert_array_equal(res[0][0], out)
+        # the state after 700 tokens of sequence 0 is its final state
+        np.testing.assert_array_equal(res[0][2][1], res[0][1][0])
+
+
 def test_config1_full_size_sampled_heads():
     """Config 1 at full size (H=32, T=8192, D=128, bf16) in the benchmark's launch
     configuration; the oracle checks every output and the final state of 3 heads."""
