@@ -165,6 +165,19 @@ def test_degenerate_orthonormal_keys_retrieve_values_exactly(D):
     assert np.abs(out - v).max() <= 1e-4 * np.abs(v).max()
 
 
+@pytest.mark.parametrize("D", [128, 64])
+def test_many_one_and_two_token_sequences(D):
+    """Appends of one or two tokens (a prefill of a prompt's last tokens onto a cached
+    state): 400 short sequences x 4 heads, so that some q . k cancel to a small value; the
+    output of a one-token slice rests on that diagonal entry, which the preparation takes in
+    fp32 from the inputs.  Every slice must still meet the tolerance."""
+    lens = [1 + (i % 2) for i in range(400)]
+    inp = synthetic.make_prefill_inputs(lens, 4, D, D, torch.bfloat16, 3.0, 0.02, 41 + D)
+    out, fin = run_prefill(inp, C=64)
+    e_o, e_f = check_prefill(inp, out, fin)
+    print("short sequences D=%d: max rel err out %.3g final %.3g" % (D, e_o, e_f))
+
+
 def test_bf16_d64():
     inp = _inputs([130, 64, 7], 2, 64, torch.bfloat16, seed=12)
     out, fin = run_prefill(inp, C=64)
