@@ -1559,14 +1559,17 @@ constexpr int kCombineThreads = 512;
 constexpr size_t kCombineSmem = sizeof(float) * D * D;
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(int H, const float* __restrict__ initial_state, const int32_t* __restrict__ seg_off,
-               float* __restrict__ seg_states) {
+               float* __restrict__ seg_states, int din) {
     extern __shared__ __align__(16) float sS[];
     const int h = blockIdx.x % H, n = blockIdx.x / H, tid = threadIdx.x;
     const int s0 = seg_off[n], ns = seg_off[n + 1] - s0;
     if (ns <= 1) return;
     constexpr size_t kWords = kSegStateBytes / sizeof(float);
-    for (int e = tid; e < D * D; e += kCombineThreads)
-        sS[e] = initial_state ? initial_state[((size_t)n * H + h) * D * D + e] : 0.f;
+    for (int e = tid; e < D * D; e += kCombineThreads) {   // the caller's din x din state, top left
+        const int r = e / D, c = e % D;
+        sS[e] = initial_state && r < din && c < din ? initial_state[((size_t)n * H + h) * din * din + r * din + c]
+                                                    : 0.f;
+    }
     __syncthreads();
     // thread: row i = tid / 4, columns j = tid % 4 + 4 z (z < 32)
     const int i = tid >> 2, j0 = tid & 3;
@@ -1798,8 +1801,7 @@ inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_se
     if ((int64_t)num_seqs * H == 0) return cudaSuccess;
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
     const int32_t* et = emit_states ? w.etab : nullptr;
-    // the chunk-parallel scan serves 128-channel heads only
-    const bool scan = w.seg > 0 && !(in_flags & kInSerialChains) && din == D;
+    const bool scan = w.seg > 0 && !(in_flags & kInSerialChains);
     const int64_t units = scan ? w.max_segs : num_seqs;   // chains: sequences, or scan segments
     const RecLaunch rl = pick_rec(units * H, din);
     auto rec = rl.kernel;
@@ -1819,7 +1821,8 @@ inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_se
     segment_index_kernel<<<1, 1024, 0, stream>>>(num_seqs, w.off, w.seg, w.seg_off, w.seg_count, w.seg_tab);
     seg_kernel<<<(unsigned)(w.max_segs * H), kSegThreads, SegSmem::BYTES, stream>>>(H, w.records, w.seg_tab,
                                                                                     w.seg_count, w.seg_states);
-    combine_kernel<<<(unsigned)num_seqs * H, kCombineThreads, kCombineSmem, stream>>>(H, s0, w.seg_off, w.seg_states);
+    combine_kernel<<<(unsigned)num_seqs * H, kCombineThreads, kCombineSmem, stream>>>(H, s0, w.seg_off, w.seg_states,
+                                                                                   din);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_after(rec, dim3((unsigned)(w.max_segs * H * nsl)), dim3(kRecThreads), rec_smem, stream,

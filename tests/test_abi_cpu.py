@@ -201,7 +201,7 @@ def test_prefill_launch_count(lib):
     assert n(8192, 0, 32) == 0
     assert n(256, 1, 2, dt=f32, d=64) == 1        # CUDA-core path: one kernel
     assert n(256, 1, 2, d=64) == 4                # bf16 at d = 64: the tensor-core kernels
-    assert n(1 << 20, 1, 8, d=64) == 4            # no chunk-parallel scan at d = 64
+    assert n(1 << 20, 1, 8, d=64) == 7            # the chunk-parallel scan at d = 64 too
     assert n(256, 1, 2, d=96) == -1
 
 

@@ -36,6 +36,18 @@ def test_scan_few_heads_long_sequence(H):
     print("scan H=%d T=%d max rel err out %.3g final %.3g" % (H, T, e_o, e_f))
 
 
+def test_scan_d64():
+    """The scan at d = 64 (the tensor-core kernels on the first 64 channels of a
+    128-channel problem): T = 2^17, H = 4, with an initial state, against the oracle and
+    against the serial chains."""
+    T, H = 1 << 17, 4
+    assert kda.kda_prefill_launches(T, 1, H, 64, 64, 64, torch.bfloat16) == 7   # the scan runs
+    inp = synthetic.make_prefill_inputs([T], H, 64, 64, torch.bfloat16, 3.0, 0.02, 520)
+    out, fin = _serial_vs_scan(inp)
+    e_o, e_f = check_prefill(inp, out, fin, chunk=64)
+    print("scan d=64 H=%d T=%d max rel err out %.3g final %.3g" % (H, T, e_o, e_f))
+
+
 def test_scan_varlen_mixed_lengths_and_emission():
     """Sequences of 420000, 200000, 0 and 1 tokens at H = 1: the long ones are cut into
     segments, the empty and the one-token sequence are one segment each.  States emitted
