@@ -574,11 +574,7 @@ def bench_gpu(args):
             "ms_per_step": round(pre["ms"], 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": kda.prefill_compute_dtype(cfg.dtype, P["D"]),
             "data": "synthetic",
-            "config": {"workload": cfg.name, "T": P["T"], "H": P["H"], "D": P["D"], "C": P["C"],
-                       "l2": "inputs larger than L2 (%.0f MB resident per step)" % (
-                           sum(P["d"][k].numel() * P["d"][k].element_size()
-                               for k in ("q", "k", "v", "g", "beta")) / 1e6),
-                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "config": prefill_config_dict(cfg, P["T"], P["d"], world),
             "roofline": pre["roofline"], "stage_ms": pre.get("stage_ms"), "decode": decode,
             "e2e": e2e, "cpu_baseline": cpu, "clocks": pre["clocks"],
             "gpu_launches": pre["launches"],
@@ -596,6 +592,15 @@ def bench_gpu(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def prefill_config_dict(cfg, T, tensors, world):
+    """The prefill workload's config, the same for both arms (the input bytes from the
+    tensors of either arm: the same shapes and dtypes)."""
+    nbytes = sum(tensors[k].numel() * tensors[k].element_size() for k in ("q", "k", "v", "g", "beta"))
+    return {"workload": cfg.name, "T": T, "H": cfg.H, "D": cfg.D, "C": cfg.C,
+            "l2": "inputs larger than L2 (%.0f MB resident per step)" % (nbytes / 1e6),
+            "parallelism": "replicas" if world > 1 else "single GPU"}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -633,7 +638,7 @@ def bench_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(secs * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "T": sum(lengths), "H": H, "D": cfg.D, "C": cfg.C},
+        "config": prefill_config_dict(cfg, sum(lengths), inp, world),
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
