@@ -181,12 +181,23 @@ class ClockSampler:
 
     def __enter__(self):
         if self.ok:
+            # a short GIL switch interval, so that the sampling thread runs while the main
+            # thread issues launches (the default 5 ms left a few-ms region with one sample)
+            self._switch = sys.getswitchinterval()
+            sys.setswitchinterval(self.period / 2)
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
+            # the thread is sampling before the region starts (its start-up took a few ms,
+            # longer than a short timed region); what it took before then is dropped
+            t0 = time.perf_counter()
+            while len(self.samples) < 2 and time.perf_counter() - t0 < 1.0:
+                time.sleep(self.period)
+            del self.samples[:]
         return self
 
     def __exit__(self, *exc):
         if self.ok:
+            sys.setswitchinterval(self._switch)
             self._stop.set()
             self._t.join()
 
