@@ -524,6 +524,34 @@ def bench_windows(args, dev, stream):
     return {"windows": rows}
 
 
+def bench_d64(args, dev, stream):
+    """bf16 with d = 64 (the tensor-core kernels on the first 64 channels of a 128-channel
+    problem) against d = 128 on the same shape: T = 8,192 tokens, H = 32 and 64 heads."""
+    import torch
+    from linear_attention_rule_b200 import kda, synthetic
+    rows = []
+    for D, H in ((128, 32), (64, 32), (64, 64)):
+        T = 8192
+        d = synthetic.make_prefill_inputs_device([T], H, D, D, torch.bfloat16, 3.0, 0.0, 5, device=dev)
+        d.pop("cpu")
+        out = torch.empty(T, H, D, dtype=torch.bfloat16, device=dev)
+        fin = torch.empty(1, H, D, D, device=dev)
+        ws = torch.empty(kda.kda_prefill_workspace_size(T, 1, H, D, D, 64, torch.bfloat16), dtype=torch.uint8,
+                         device=dev)
+
+        def step():
+            kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out, final_state=fin,
+                            workspace=ws, stream=stream)
+        for _ in range(args.warmup):
+            step()
+        ms, _, _ = timed(stream, dev, 1, args.steps, step)
+        assert kda.kda_get_device_status(stream) == kda.KDA_OK
+        rows.append({"D": D, "H": H, "T": T, "ms": round(ms, 4), "tokens_per_s": round(T / (ms * 1e-3), 1)})
+        del d, out, fin, ws
+        torch.cuda.empty_cache()
+    return {"d64": rows}
+
+
 def bench_gpu(args):
     import torch
     from linear_attention_rule_b200 import kda
@@ -561,6 +589,8 @@ def bench_gpu(args):
         line = bench_crossover(args, dev, stream)
     elif args.workload == "windows":
         line = bench_windows(args, dev, stream)
+    elif args.workload == "d64":
+        line = bench_d64(args, dev, stream)
     elif args.workload in ("config2", "config4"):
         P = setup_prefill(dev, rank, int(args.workload[-1]))
         pre = bench_prefill(args, P, dev, stream, world, peaks)
@@ -670,7 +700,7 @@ def main(argv=None):
     ap.add_argument("--no-extra-configs", action="store_true",
                     help="skip the varlen (config 2) and long-context (config 4) prefill entries")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--workload", choices=["all", "prefill", "decode", "config2", "config4", "crossover", "windows"],
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "config2", "config4", "crossover", "windows", "d64"],
                     default="all",
                     help="restrict the run (profiling) or measure another prefill config; "
                          "the driver's JSON line is 'all'")
