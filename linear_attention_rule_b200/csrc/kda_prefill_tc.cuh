@@ -465,6 +465,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // ---- (1) decay: thread = (block of 4 tokens rb, group of 8 channels cg) ----
         const int cg = lane & 15, half = lane >> 4, rb = 2 * warp + half;
         const int kb = cg >> 3, c8 = cg & 7;
+        // fp32 rows of 8 channels per lane: the 8 lanes of a quarter warp sit 32 bytes apart,
+        // so a 16-byte access of the same half by all of them meets every other bank twice.
+        // Groups 4..7 of each eight take their upper half first (byte offsets o1, then o2):
+        // each access instruction then covers the 32 banks once.
+        const bool swp = (cg & 4) != 0;
+        const uint32_t o1 = swp ? 16u : 0u, o2 = 16u - o1;
         float loc[4][8], acc[8], gam[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) acc[u] = 0.f;
@@ -477,8 +483,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int u = 0; u < 8; ++u) gv[u] = gt[r];
             } else if (DIN == 128 || cg < 8) {
-                const float4 g0 = *reinterpret_cast<const float4*>(gt + r * DIN + 8 * cg);
-                const float4 g1 = *reinterpret_cast<const float4*>(gt + r * DIN + 8 * cg + 4);
+                const uint32_t ga = smem_u32(gt + r * DIN + 8 * cg);
+                const float4 f1 = lds_f4(ga + o1), f2 = lds_f4(ga + o2);
+                const float4 g0 = swp ? f2 : f1, g1 = swp ? f1 : f2;
                 gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w;
                 gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
                 if (in_flags & kInGLogits) {
@@ -498,29 +505,42 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         float other[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) other[u] = __shfl_xor_sync(0xffffffffu, acc[u], 16);
-        if (half == 0) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) sX[warp * D + 8 * cg + u] = acc[u] + other[u];
+        if (half == 0) {   // the same access order as the g reads
+            const float4 v0 = make_float4(acc[0] + other[0], acc[1] + other[1], acc[2] + other[2], acc[3] + other[3]);
+            const float4 v1 = make_float4(acc[4] + other[4], acc[5] + other[5], acc[6] + other[6], acc[7] + other[7]);
+            const uint32_t xa = smem_u32(sX + warp * D + 8 * cg);
+            sts_f4(xa + o1, swp ? v1 : v0);
+            sts_f4(xa + o2, swp ? v0 : v1);
         }
         KDA_TRACE_POINT(ptr_, 8192 + 20);
         __syncthreads();
         KDA_TRACE_POINT(ptr_, 8192 + 21);
-        float base[8], tot[8];
+        // sums over the warps' partials, held with the halves in access order (bp, tp), then
+        // put back in channel order
+        float base[8], tot[8], bp[8], tp[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            base[u] = half ? other[u] : 0.f;
-            tot[u] = 0.f;
+        for (int u = 0; u < 4; ++u) {
+            bp[u] = half ? (swp ? other[u + 4] : other[u]) : 0.f;
+            bp[u + 4] = half ? (swp ? other[u] : other[u + 4]) : 0.f;
+            tp[u] = tp[u + 4] = 0.f;
         }
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-            const float4 x0 = *reinterpret_cast<const float4*>(sX + w * D + 8 * cg);
-            const float4 x1 = *reinterpret_cast<const float4*>(sX + w * D + 8 * cg + 4);
-            const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            const uint32_t xa = smem_u32(sX + w * D + 8 * cg);
+            const float4 x1 = lds_f4(xa + o1), x2 = lds_f4(xa + o2);
+            const float xv[8] = {x1.x, x1.y, x1.z, x1.w, x2.x, x2.y, x2.z, x2.w};
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                tot[u] += xv[u];
-                if (w < warp) base[u] += xv[u];
+                tp[u] += xv[u];
+                if (w < warp) bp[u] += xv[u];
             }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            tot[u] = swp ? tp[u + 4] : tp[u];
+            tot[u + 4] = swp ? tp[u] : tp[u + 4];
+            base[u] = swp ? bp[u + 4] : bp[u];
+            base[u + 4] = swp ? bp[u] : bp[u + 4];
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) gam[u] = __expf(tot[u]);
