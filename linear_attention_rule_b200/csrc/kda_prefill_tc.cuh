@@ -24,7 +24,8 @@
 //                         [K_dec; Q_dec] K_inv^T                                      (MMA 128x64x128)
 //                         L = strict_tril(beta K_dec K_inv^T), Aqk = tril(Q_dec K_inv^T)
 //                         INV = (I + L)^-1: 16x16 diagonal blocks by forward substitution,
-//                                               then block doubling 16 -> 32 -> 64 (fp32)
+//                                               block doubling 16 -> 32 (fp32, CUDA cores),
+//                                               32 -> 64 as two chained products     (MMA tf32)
 //                         [W | U] = INV diag(beta) [K_dec | V]                       (MMA 128x256x64)
 //                         -M = K_res^T W                                             (MMA 128x128x64)
 //                         Aqk W -> P = Q_dec - Aqk W                                 (MMA 128x128x64)
@@ -315,19 +316,23 @@ struct PrepSmem {
     static constexpr uint32_t BLK = 16384;   // stride between the channel halves
     // g tile fp32 [64][128] (plain); after the decay: Abar image, Aqk image, L / INV fp32
     static constexpr uint32_t GR = 65536;
-    static constexpr uint32_t ABAR = GR, AQK = GR + 8192, LI = GR + 16384;   // LI: [64][68]
+    // L / INV as 32 x 32 fp32 tiles with 128-byte swizzled rows (the tf32 K-major operand
+    // layout): TB the lower-right block (L22, then B^{-1}), T10 the lower-left block of L
+    // stored transposed (L21^T), T00 the upper-left block (L11, then A^{-1}), TAT = A^{-T}.
+    // The upper-right block is zero and not stored.
+    static constexpr uint32_t ABAR = GR, AQK = GR + 8192, LI = GR + 16384;
+    static constexpr uint32_t TB = LI, T10 = LI + 4096, T00 = LI + 8192, TAT = LI + 12288;
     static constexpr uint32_t XCH = GR + 33792;      // decay partials [8][128]; later T [32][36]
     static constexpr uint32_t BETA = XCH + 4608;     // [64]
     static constexpr uint32_t DIAG = BETA + 256;      // [64] q_r . k_r in fp32 (Aqk's diagonal)
     static constexpr uint32_t BAR = DIAG + 256;       // g's TMA, then the products in order
-    static constexpr uint32_t BAR2 = BAR + 8;         // the last product (Aqk W)
+    static constexpr uint32_t BAR2 = BAR + 8;         // the UT's first product, then the last (Aqk W)
     static constexpr uint32_t BARQK = BAR2 + 8;       // TMA of q and k
     static constexpr uint32_t BARV = BARQK + 8;       // TMA of v
     static constexpr uint32_t TMEM = BARV + 8;
     static constexpr uint32_t STRONG = TMEM + 4;       // some channel's chunk decay is below kStrongDecay
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;  // + alignment slack
 };
-constexpr int kLP = 68;                                   // row pitch of L / INV (16-byte rows)
 constexpr int kTP = 36;                                   // row pitch of the product scratch
 constexpr uint32_t kPrepTmemCols = 256;
 constexpr uint32_t kPrepTxG = 32768, kPrepTxQK = 2 * 16384, kPrepTxV = 16384;   // bytes per barrier
@@ -403,7 +408,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t bar = sb + S::BAR;
     float* sBeta = reinterpret_cast<float*>(sm + S::BETA);
     float* sX = reinterpret_cast<float*>(sm + S::XCH);
-    float* sLI = reinterpret_cast<float*>(sm + S::LI);
+    // element (r, c) of a tile of L / INV, and 4 of them from a column c divisible by 4
+    auto lt = [&](uint32_t tile, int r, int c) -> float& {
+        return *reinterpret_cast<float*>(sm + tile + sw128_off(r, c >> 2) + (c & 3) * 4);
+    };
+    auto lt4 = [&](uint32_t tile, int r, int c) -> float4& {
+        return *reinterpret_cast<float4*>(sm + tile + sw128_off(r, c >> 2));
+    };
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wh = warp >> 2;   // TMEM lane quarter, column half
     bool ok = true, v_ok = true;
@@ -661,23 +672,26 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr)   // the first product has read K_inv
             *reinterpret_cast<uint4*>(sm + S::KI0 + kb * S::BLK + sw128_off(4 * rb + rr, c8)) = kres[rr];
-        {
+        if (wq != 0 || wh != 1) {   // (warp 4 would hold L's upper-right block: zero, not stored)
             float d[32];
             tmem_ld32(tl + 32 * wh, d);
             tmem_wait_ld();
-            if (wq < 2) {   // L[r][s] = beta_r (K_dec K_inv^T)[r][s] for s < r (fp32, pitch 65)
-                const int r = 32 * wq + lane;
-                const float br = sBeta[r];
+            if (wq < 2) {   // L[r][s] = beta_r (K_dec K_inv^T)[r][s] for s < r, fp32
+                const float br = sBeta[32 * wq + lane];
+                if (wh == 0 && wq == 1) {   // L21, transposed: row s, column lane; then warp 5 may use it
 #pragma unroll
-                for (int u4 = 0; u4 < 8; ++u4) {
-                    float e[4];
+                    for (int s2 = 0; s2 < 32; ++s2) lt(S::T10, s2, lane) = br * d[s2];
+                    fence_proxy_async_smem();
+                    bar_arrive_fixed<1>(64);
+                } else {   // diagonal block L11 (warp 0) or L22 (warp 5): row lane, zero from the diagonal on
+                    const uint32_t tile = wq ? S::TB : S::T00;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int s = 32 * wh + 4 * u4 + u;
-                        e[u] = s < r ? br * d[4 * u4 + u] : 0.f;
+                    for (int u4 = 0; u4 < 8; ++u4) {
+                        float e[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) e[u] = 4 * u4 + u < lane ? br * d[4 * u4 + u] : 0.f;
+                        lt4(tile, lane, 4 * u4) = make_float4(e[0], e[1], e[2], e[3]);
                     }
-                    *reinterpret_cast<float4*>(sLI + r * kLP + 32 * wh + 4 * u4) =
-                        make_float4(e[0], e[1], e[2], e[3]);
                 }
             } else {        // Aqk[r][s] = (Q_dec K_inv^T)[r][s] for s < r, q_r . k_r for s = r (bf16 image)
                 const int r = 32 * (wq - 2) + lane;
@@ -694,41 +708,49 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
         }
-        // First step of the UT transform INV = (I + L)^{-1}: the 16x16 diagonal blocks D_b,
-        // inverted in place by the warp that drained them (warp 0: blocks 0, 1 = rows and
-        // columns 0..31; warp 5: blocks 2, 3), lane = (block, column j).  Column-oriented
-        // forward substitution: once x[s] is final it is subtracted from every later row, so
-        // the dependent chain is 15 FMAs long.
+        // First step of the UT transform INV = (I + L)^{-1}: the two 16x16 diagonal blocks D_b
+        // of a diagonal tile, inverted in place by the warp that drained it (warp 0: T00,
+        // warp 5: TB), lane = (block b, column j).  Column-oriented forward substitution: once
+        // x[s] is final it is subtracted from every later row, so the dependent chain is 15
+        // FMAs long.
         if (warp == 0 || warp == 5) {
             __syncwarp();
-            const int b = (warp == 5 ? 2 : 0) + (lane >> 4), j = lane & 15;
+            const uint32_t tile = warp == 5 ? S::TB : S::T00;
+            const int b = lane >> 4, j = lane & 15;
             float x[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
             for (int s2 = 0; s2 < 15; ++s2) {
 #pragma unroll
-                for (int r = s2 + 1; r < 16; ++r) x[r] -= sLI[(16 * b + r) * kLP + 16 * b + s2] * x[s2];
+                for (int r = s2 + 1; r < 16; ++r) x[r] -= lt(tile, 16 * b + r, 16 * b + s2) * x[s2];
             }
             __syncwarp();
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sLI[(16 * b + r) * kLP + 16 * b + j] = x[r];
+            for (int r = 0; r < 16; ++r) lt(tile, 16 * b + r, 16 * b + j) = x[r];
+            if (warp == 0) {   // A^{-T} for the 32 -> 64 product: column j of D_b is its row 16 b + j,
+                               // and the block left of D_1^T is zero (8 columns per lane)
+#pragma unroll
+                for (int r4 = 0; r4 < 16; r4 += 4)
+                    lt4(S::TAT, 16 * b + j, 16 * b + r4) = make_float4(x[r4], x[r4 + 1], x[r4 + 2], x[r4 + 3]);
+                lt4(S::TAT, 16 + j, 8 * b) = make_float4(0.f, 0.f, 0.f, 0.f);
+                lt4(S::TAT, 16 + j, 8 * b + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
             __syncwarp();
-            // 16 -> 32 for the same warp's block pair (warp 0: blocks 0, 1; warp 5: 2, 3):
-            // X = -D_hi (L_lo D_lo) into rows R .. R+15, columns Cc .. Cc+15; lane = (row r,
-            // 8 columns); T through the scratch rows 16 p .. 16 p + 15
+            // 16 -> 32 in the same tile: X = -D_1 (L_10 D_0) into rows 16..31, columns 0..15;
+            // lane = (row r, 8 columns); the product L_10 D_0 through the scratch rows
+            // 16 p .. 16 p + 15
             {
                 float* sT = sX;
                 const int p = warp == 5 ? 1 : 0, r = lane >> 1, c8 = 8 * (lane & 1);
-                const int R = 16 * (2 * p + 1), Cc = 32 * p;
                 float t[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) t[u] = 0.f;
 #pragma unroll
                 for (int s2 = 0; s2 < 16; ++s2) {
-                    const float l = sLI[(R + r) * kLP + Cc + s2];
-                    const float4 d0 = *reinterpret_cast<const float4*>(sLI + (Cc + s2) * kLP + Cc + c8);
-                    const float4 d1 = *reinterpret_cast<const float4*>(sLI + (Cc + s2) * kLP + Cc + c8 + 4);
+                    const float l = lt(tile, 16 + r, s2);
+                    const float4 d0 = lt4(tile, s2, c8);
+                    const float4 d1 = lt4(tile, s2, c8 + 4);
                     t[0] += l * d0.x; t[1] += l * d0.y; t[2] += l * d0.z; t[3] += l * d0.w;
                     t[4] += l * d1.x; t[5] += l * d1.y; t[6] += l * d1.z; t[7] += l * d1.w;
                 }
@@ -738,15 +760,36 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int u = 0; u < 8; ++u) t[u] = 0.f;
 #pragma unroll
-                for (int s2 = 0; s2 < 16; ++s2) {   // D_hi is lower triangular: its zeros add nothing
-                    const float dh = sLI[(R + r) * kLP + R + s2];
+                for (int s2 = 0; s2 < 16; ++s2) {   // D_1 is lower triangular: its zeros add nothing
+                    const float dh = lt(tile, 16 + r, 16 + s2);
                     const float4 t0 = *reinterpret_cast<const float4*>(sT + (16 * p + s2) * kTP + c8);
                     const float4 t1 = *reinterpret_cast<const float4*>(sT + (16 * p + s2) * kTP + c8 + 4);
                     t[0] -= dh * t0.x; t[1] -= dh * t0.y; t[2] -= dh * t0.z; t[3] -= dh * t0.w;
                     t[4] -= dh * t1.x; t[5] -= dh * t1.y; t[6] -= dh * t1.z; t[7] -= dh * t1.w;
                 }
-                *reinterpret_cast<float4*>(sLI + (R + r) * kLP + Cc + c8) = make_float4(t[0], t[1], t[2], t[3]);
-                *reinterpret_cast<float4*>(sLI + (R + r) * kLP + Cc + c8 + 4) = make_float4(t[4], t[5], t[6], t[7]);
+                lt4(tile, 16 + r, c8) = make_float4(t[0], t[1], t[2], t[3]);
+                lt4(tile, 16 + r, c8 + 4) = make_float4(t[4], t[5], t[6], t[7]);
+                if (warp == 0) {   // and into A^{-T}, transposed
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) lt(S::TAT, c8 + u, 16 + r) = t[u];
+                }
+            }
+            if (warp == 5) {
+                // B^{-1} is final, and L21^T once warp 1 has arrived: the first product of the
+                // 32 -> 64 step, D1 = B^{-1} (L21^T)^T -> TMEM [64, 96), runs while warp 0 still
+                // inverts A.  (Its A operand has M = 128 rows: those past B^{-1} are the other
+                // tiles, whatever they hold; product rows 32-127 are never read.)
+                fence_proxy_async_smem();
+                bar_sync_fixed<1>(64);
+                if (lane == 0) {
+                    tc_fence_after();
+                    constexpr uint32_t id = idesc_tf32(128, 32);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)   // K = 8 per product: 32 bytes of a tile row
+                        umma_tf32(tmem + 64, smem_desc(sb + S::TB + ks * 32, 16, 1024, kSwizzle128),
+                                  smem_desc(sb + S::T10 + ks * 32, 16, 1024, kSwizzle128), id, ks > 0);
+                    umma_commit(bar + 8);
+                }
             }
         }
     }
@@ -762,49 +805,54 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         bulk_s2g(rec + kRecAQ, sb + S::AQK, 8192);
     }
 
-    // ---- (3) UT transform INV = (I + L)^{-1}, in place over L ----
-    // Every entry above the diagonal of the buffer is 0 (L is strictly lower triangular and
-    // the inverse is lower triangular), so the block products below need no masks.
-    {
-        float* sT = sX;
-        KDA_TRACE_POINT(ptr_, 8192 + 18);
-        // 32 -> 64: X = -B^{-1} (L[32:64, 0:32] A^{-1}); thread (row r, 4 columns)
-        {
-            const int r = tid >> 3, c4 = 4 * (tid & 7);
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-            for (int s2 = 0; s2 < 32; ++s2) {
-                const float l = sLI[(32 + r) * kLP + s2];
-                const float4 av = *reinterpret_cast<const float4*>(sLI + s2 * kLP + c4);
-                acc.x += l * av.x; acc.y += l * av.y; acc.z += l * av.z; acc.w += l * av.w;
-            }
-            *reinterpret_cast<float4*>(sT + r * kTP + c4) = acc;
-            __syncthreads();
-            float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
-            const int smax = r | 3;   // rows r of a warp are 4 w .. 4 w + 3; B^{-1}[r][s] = 0 for s > r
-#pragma unroll 4
-            for (int s2 = 0; s2 < 32; ++s2) {
-                if (s2 > smax) break;
-                const float bi = sLI[(32 + r) * kLP + 32 + s2];
-                const float4 tv = *reinterpret_cast<const float4*>(sT + s2 * kTP + c4);
-                xo.x -= bi * tv.x; xo.y -= bi * tv.y; xo.z -= bi * tv.z; xo.w -= bi * tv.w;
-            }
-            // Abar = INV diag(beta) as a bf16 K-major A image.  This thread writes columns
-            // c4..c4+3 and 32+c4..32+c4+3 of rows r and 32 + r: the block just computed, and
-            // entries final since the 16 -> 32 step (INV[r][32..63] = 0 for r < 32).
-            const float4 b_lo = *reinterpret_cast<const float4*>(sBeta + c4);
-            const float4 b_hi = *reinterpret_cast<const float4*>(sBeta + 32 + c4);
-            auto put4 = [&](int row, int col, float4 x4, float4 b4) {
-                *reinterpret_cast<uint2*>(sm + S::ABAR + sw128_off(row, col >> 3) + (col & 4) * 2) =
-                    make_uint2(pack_bf16x2(x4.x * b4.x, x4.y * b4.y), pack_bf16x2(x4.z * b4.z, x4.w * b4.w));
-            };
-            put4(32 + r, c4, xo, b_lo);
-            put4(r, c4, *reinterpret_cast<const float4*>(sLI + r * kLP + c4), b_lo);
-            put4(r, 32 + c4, make_float4(0.f, 0.f, 0.f, 0.f), b_hi);
-            put4(32 + r, 32 + c4, *reinterpret_cast<const float4*>(sLI + (32 + r) * kLP + 32 + c4), b_hi);
-        }
-        KDA_TRACE_POINT(ptr_, 8192 + 19);
+    // ---- (3) UT transform, 32 -> 64: INV = [[A^{-1}, 0], [X, B^{-1}]] with
+    // X = -B^{-1} L21 A^{-1} (A, B the diagonal 32-blocks of I + L), on the tensor cores in
+    // tf32: D1 = B^{-1} (L21^T)^T (issued by warp 5 above, committed to the second barrier),
+    // then D2 = D1 (A^{-T})^T -> TMEM [96, 128) with D1 read from Tensor Memory, once D1 is
+    // complete (products into different accumulators are not ordered); lanes 0-31
+    // meaningful; X = -D2.  The entries of the tiles above their diagonals are 0 (L strictly
+    // lower triangular, the inverse lower triangular), so the products need no masks.
+    KDA_TRACE_POINT(ptr_, 8192 + 18);
+    if (tid == 0) {
+        v_ok = mbar_wait(bar + 8, 0);
+        tc_fence_after();
+        constexpr uint32_t id = idesc_tf32(128, 32);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            umma_tf32_tmem_a(tmem + 96, tmem + 64 + 8 * ks, smem_desc(sb + S::TAT + ks * 32, 16, 1024, kSwizzle128),
+                             id, ks > 0);
+        umma_commit(bar);
     }
+    {   // meanwhile Abar = INV diag(beta) as a bf16 K-major A image, the blocks without X:
+        // this thread writes columns c4..c4+3 and 32+c4..32+c4+3 of row r and columns 32+c4..
+        // of row 32 + r
+        const int r = tid >> 3, c4 = 4 * (tid & 7);
+        const float4 b_lo = *reinterpret_cast<const float4*>(sBeta + c4);
+        const float4 b_hi = *reinterpret_cast<const float4*>(sBeta + 32 + c4);
+        auto put4 = [&](int row, int col, float4 x4, float4 b4) {
+            *reinterpret_cast<uint2*>(sm + S::ABAR + sw128_off(row, col >> 3) + (col & 4) * 2) =
+                make_uint2(pack_bf16x2(x4.x * b4.x, x4.y * b4.y), pack_bf16x2(x4.z * b4.z, x4.w * b4.w));
+        };
+        put4(r, c4, lt4(S::T00, r, c4), b_lo);
+        put4(r, 32 + c4, make_float4(0.f, 0.f, 0.f, 0.f), b_hi);
+        put4(32 + r, 32 + c4, lt4(S::TB, r, c4), b_hi);
+    }
+    ok = mbar_wait(bar, phase) && v_ok;
+    phase ^= 1;
+    tc_fence_after();
+    if (!prep_sync_ok(ok, tid)) goto done;
+    if (wq == 0) {   // warps 0 and 4: row lane of X, columns 16 wh .. 16 wh + 15, into Abar's row 32 + lane
+        float d[16], e[16];
+        tmem_ld16(tl + 96 + 16 * wh, d);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) e[u] = -d[u] * sBeta[16 * wh + u];
+#pragma unroll
+        for (int j2 = 0; j2 < 2; ++j2)
+            *reinterpret_cast<uint4*>(sm + S::ABAR + sw128_off(32 + lane, 2 * wh + j2)) = pack_bf16x8(&e[8 * j2]);
+    }
+    KDA_TRACE_POINT(ptr_, 8192 + 19);
+    tc_fence_before();
     fence_proxy_async_smem();
     __syncthreads();
     KDA_TRACE_POINT(ptr_, 8192 + 4);
@@ -903,7 +951,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (wq < 2) {
         // Drain of P = Q_dec - Aqk W: rows r = 32 wq .., K block wh.  Both products have read W
         // by now, so its space holds the staging slots.
-        ok = __all_sync(0xffffffffu, mbar_wait(bar + 8, 0));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar + 8, 1));   // its second phase
         if (!ok) {
             if (lane == 0) kda_set_status(KDA_ERR_TIMEOUT);
         } else {

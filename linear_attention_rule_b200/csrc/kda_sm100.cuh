@@ -244,6 +244,39 @@ __device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tme
         : "memory");
 }
 
+// Instruction descriptor of tcgen05.mma kind::tf32: A and B tf32 (fp32 in memory, read with
+// a 10-bit mantissa), K-major, fp32 accumulate; K = 8 per instruction.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+    return (1u << 4)                          // D format fp32
+           | (2u << 7)                        // A format tf32
+           | (2u << 10)                       // B format tf32
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::tf32, issued by one thread.
+__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::tf32: A (M rows = TMEM lanes, one fp32 per column,
+// K-major) read from Tensor Memory.
+__device__ __forceinline__ void umma_tf32_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                                 uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on `bar` once every tcgen05.mma this thread issued before has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -288,6 +321,21 @@ __device__ __forceinline__ void sts_f4(uint32_t addr, float4 v) {
 // Named barrier among the first `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier `ID` (fixed at compile time, so that the kernel reserves only the barriers
+// it names) for `count` threads: bar_sync_fixed waits for all of them, bar_arrive_fixed
+// counts the calling warp in without waiting (its earlier shared-memory writes are ordered
+// before what the waiting threads do next).
+template <int ID>
+__device__ __forceinline__ void bar_sync_fixed(uint32_t count) {
+    static_assert(ID > 0 && ID < 16, "barrier 0 is __syncthreads' own");
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "r"(count) : "memory");
+}
+template <int ID>
+__device__ __forceinline__ void bar_arrive_fixed(uint32_t count) {
+    static_assert(ID > 0 && ID < 16, "barrier 0 is __syncthreads' own");
+    asm volatile("bar.arrive %0, %1;" ::"n"(ID), "r"(count) : "memory");
 }
 
 }  // namespace sm100
