@@ -665,10 +665,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             umma_commit(bar);
         }
-        ok = mbar_wait(bar, phase);
+        // Each thread learns of the product's completion from the barrier itself; what follows
+        // up to the next block barrier depends on nothing another warp writes first.  A wait
+        // that gave up records the timeout and the CTA runs on (every later wait is bounded too).
+        if (!mbar_wait(bar, phase)) kda_set_status(KDA_ERR_TIMEOUT);
         phase ^= 1;
         tc_fence_after();
-        if (!prep_sync_ok(ok, tid)) goto done;
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr)   // the first product has read K_inv
             *reinterpret_cast<uint4*>(sm + S::KI0 + kb * S::BLK + sw128_off(4 * rb + rr, c8)) = kres[rr];
@@ -837,10 +839,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         put4(r, 32 + c4, make_float4(0.f, 0.f, 0.f, 0.f), b_hi);
         put4(32 + r, 32 + c4, lt4(S::TB, r, c4), b_hi);
     }
-    ok = mbar_wait(bar, phase) && v_ok;
+    if (!(mbar_wait(bar, phase) && v_ok)) kda_set_status(KDA_ERR_TIMEOUT);   // as after the first product
     phase ^= 1;
     tc_fence_after();
-    if (!prep_sync_ok(ok, tid)) goto done;
     if (wq == 0) {   // warps 0 and 4: row lane of X, columns 16 wh .. 16 wh + 15, into Abar's row 32 + lane
         float d[16], e[16];
         tmem_ld16(tl + 96 + 16 * wh, d);
@@ -870,10 +871,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                       smem_desc(sb + S::KD0 + ks * 2048, S::BLK, 1024, kSwizzle128), id, ks > 0);
         umma_commit(bar);
     }
-    ok = mbar_wait(bar, phase) && v_ok;
+    if (!(mbar_wait(bar, phase) && v_ok)) kda_set_status(KDA_ERR_TIMEOUT);   // as after the first product
     phase ^= 1;
     tc_fence_after();
-    if (!prep_sync_ok(ok, tid)) goto done;
     if (wq < 2) {
         // rows r of W (column half 0) -> bf16 B image in place of K_dec (two 64-column blocks,
         // 128-byte swizzle); rows r of U (column half 1) -> four 32-column slices with a
