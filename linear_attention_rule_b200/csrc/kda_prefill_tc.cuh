@@ -536,16 +536,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         __syncthreads();
         KDA_TRACE_POINT(ptr_, 8192 + 21);
         // sums over the warps' partials, held with the halves in access order (bp, tp), then
-        // put back in channel order
+        // put back in channel order.  The two half-warps hold the same channels: half 0 reads
+        // the partials of warps 0..3, half 1 those of warps 4..7, and they swap their sums.
         float base[8], tot[8], bp[8], tp[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            bp[u] = half ? (swp ? other[u + 4] : other[u]) : 0.f;
-            bp[u + 4] = half ? (swp ? other[u] : other[u + 4]) : 0.f;
-            tp[u] = tp[u + 4] = 0.f;
-        }
+        for (int u = 0; u < 8; ++u) bp[u] = tp[u] = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
+        for (int k = 0; k < 4; ++k) {
+            const int w = 4 * half + k;
             const uint32_t xa = smem_u32(sX + w * D + 8 * cg);
             const float4 x1 = lds_f4(xa + o1), x2 = lds_f4(xa + o2);
             const float xv[8] = {x1.x, x1.y, x1.z, x1.w, x2.x, x2.y, x2.z, x2.w};
@@ -554,6 +552,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 tp[u] += xv[u];
                 if (w < warp) bp[u] += xv[u];
             }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {   // a + b on one side, b + a on the other: the same sums
+            tp[u] += __shfl_xor_sync(0xffffffffu, tp[u], 16);
+            bp[u] += __shfl_xor_sync(0xffffffffu, bp[u], 16);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {   // the rows of half 0 of this warp precede those of half 1
+            bp[u] += half ? (swp ? other[u + 4] : other[u]) : 0.f;
+            bp[u + 4] += half ? (swp ? other[u] : other[u + 4]) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
