@@ -62,10 +62,11 @@ typedef enum {
 
 typedef enum {
     KDA_F32 = 0,   /* q, k, v, out in fp32: the CUDA-core (FFMA) chunked path */
-    KDA_BF16 = 1   /* q, k, v, out in bf16: the tensor-core (tcgen05) chunked path; at
-                      dk = dv = 64 it runs as the first 64 channels of a 128-channel
-                      problem whose other channels are zero (same results, the cost of
-                      d = 128) */
+    KDA_BF16 = 1   /* q, k, v, out in bf16: the tensor-core (tcgen05) chunked path with
+                      bf16 chunk operands, fp32 accumulation, decay and state (the last
+                      doubling of the UT inverse takes tf32 operands); at dk = dv = 64 it
+                      runs as the first 64 channels of a 128-channel problem whose other
+                      channels are zero (same results, the cost of d = 128) */
 } kda_dtype;
 
 /*
