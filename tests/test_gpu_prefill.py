@@ -345,21 +345,31 @@ def test_config4_long_context_full_size_sampled_heads():
         assert e_w <= TOL[torch.bfloat16], (a, e_w)
 
 
-@pytest.mark.parametrize("lens", [[8192], [2048, 700, 0, 3333, 64]])
-def test_bf16_prefill_is_deterministic(lens):
-    """Repeated calls on the same inputs give the same bits.  The tensor-core preparation
-    passes data between warps through named barriers and between products through Tensor
-    Memory; a missing ordering there shows up as run-to-run differences far below the
-    parity tolerance, which only this comparison sees."""
-    H = 32
-    d = to_device(_inputs(lens, H, 128, torch.bfloat16, seed=23))
+@pytest.mark.parametrize("lens,H,D,windows", [
+    ([8192], 32, 128, False),
+    ([2048, 700, 0, 3333, 64], 32, 128, False),
+    ([2048, 700, 0, 3333, 64], 32, 128, True),    # a workspace of a few windows
+    ([2048, 700, 0, 3333, 64], 32, 64, False),    # d = 64 on the tensor cores
+    ([262144], 4, 128, False),                     # few long chains: the chunk-parallel scan
+])
+def test_bf16_prefill_is_deterministic(lens, H, D, windows):
+    """Repeated calls on the same inputs give the same bits.  The tensor-core kernels pass
+    data between warps through named barriers and between products through Tensor Memory;
+    a missing ordering there shows up as run-to-run differences far below the parity
+    tolerance, which only this comparison sees."""
+    d = to_device(_inputs(lens, H, D, torch.bfloat16, seed=23))
     T, N = sum(lens), len(lens)
-    ws = torch.empty(kda.kda_prefill_workspace_size(T, N, H, 128, 128, 64, torch.bfloat16),
-                     dtype=torch.uint8, device="cuda")
+    if H == 4:
+        assert kda.kda_prefill_launches(T, N, H, D, D, 64, torch.bfloat16) == 7   # the scan runs
+    size = kda.kda_prefill_workspace_size(T, N, H, D, D, 64, torch.bfloat16)
+    if windows:
+        size = kda.kda_prefill_workspace_size_min(T, N, H, D, D, 64, torch.bfloat16) + 4 * H * (90624 + 8) + 2048
+        assert kda.kda_prefill_windows(T, N, H, D, D, 64, torch.bfloat16, size) > 1
+    ws = torch.empty(size, dtype=torch.uint8, device="cuda")
     runs = []
     for _ in range(3):
-        out = torch.full((T, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
-        fin = torch.full((N, H, 128, 128), float("nan"), device="cuda")
+        out = torch.full((T, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        fin = torch.full((N, H, D, D), float("nan"), device="cuda")
         kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], out,
                         initial_state=d["s0"], final_state=fin, workspace=ws)
         torch.cuda.synchronize()
