@@ -236,15 +236,17 @@ int64_t kda_prefill_windows(int64_t total_tokens, int32_t num_seqs, int32_t H, i
 /*
  * Number of kernels one kda_prefill_ex call with these arguments launches (for capturing
  * the call in a CUDA graph or counting launches), -1 for arguments kda_prefill_ex rejects
- * as unsupported.  On the tensor-core path that is the chunk table, the emission slots
+ * as unsupported.  On the tensor-core path that is the chunk table, the order in which the
+ * recurrence takes the sequences (when num_seqs > 1: longest first), the emission slots
  * (when num_emit > 0), the preparation and the preparation of strongly decayed chunks
  * (when total_tokens > 0), and the recurrence, plus three for the chunk-parallel scan:
  * that runs, unless in_flags holds KDA_IN_SERIAL_CHAINS, when few (sequence, head) chains
  * are long: when the recurrence's four value-slice CTAs per chain would leave at least half
  * of 148 SMs idle (18 chains or fewer) and segments of 64 chunks or more result.
  * That count is for the full workspace; a call that runs in n > 1 windows
- * (kda_prefill_windows) launches the chunk table, the emission slots when num_emit > 0,
- * and three kernels per window (preparation, strongly decayed chunks, recurrence).
+ * (kda_prefill_windows) launches the chunk table, the order when num_seqs > 1, the emission
+ * slots when num_emit > 0, and three kernels per window (preparation, strongly decayed
+ * chunks, recurrence).
  * Depends on the sizes only.
  */
 int32_t kda_prefill_launches(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,

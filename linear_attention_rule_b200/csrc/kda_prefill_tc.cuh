@@ -77,11 +77,11 @@ __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + 
 __host__ inline int64_t max_chunks(int64_t total_tokens, int num_seqs) {
     return total_tokens / C + num_seqs;
 }
-// Workspace: [chunk offsets int32 (N+1)] [chunk table int2 (max_chunks)] [emission slot per
-// chunk int32 (max_chunks)] [strong-decay count int32, pad] [strong-decay units int2
-// (max_chunks x H)] [records (max_chunks x H)]
+// Workspace: [chunk offsets int32 (N+1)] [recurrence order of the sequences int32 (N+1)]
+// [chunk table int2 (max_chunks)] [emission slot per chunk int32 (max_chunks)] [strong-decay
+// count int32, pad] [strong-decay units int2 (max_chunks x H)] [records (max_chunks x H)]
 __host__ inline size_t ws_table_offset(int num_seqs) {
-    return align_up(sizeof(int32_t) * (size_t)(num_seqs + 1), 16);
+    return align_up(sizeof(int32_t) * 2 * (size_t)(num_seqs + 1), 16);
 }
 __host__ inline size_t ws_emit_offset(int64_t total_tokens, int num_seqs) {
     return align_up(ws_table_offset(num_seqs) + sizeof(int2) * (size_t)max_chunks(total_tokens, num_seqs), 16);
@@ -270,6 +270,57 @@ chunk_index_kernel(const int32_t* __restrict__ cu, int num_seqs, int64_t total,
         tab[c] = make_int2(t0, min(C, cu[n + 1] - t0));
         if (etab) etab[c] = -1;
     }
+}
+
+// The order in which the recurrence's CTAs take several sequences, written after the chunk
+// offsets (order = off + N + 1): most chunks first, ties by index, so that a long chain does
+// not start last and set the launch's tail; the identity beyond kOrderMax sequences.  Single
+// CTA of 1024 threads, a bitonic sort in its dynamic shared memory (order_smem_bytes).  Bad
+// cu_seqlens left every count 0: the identity.
+constexpr int kOrderMax = 2048;
+__host__ __device__ inline int order_pow2(int num_seqs) {
+    int p = 2;
+    while (p < num_seqs) p <<= 1;
+    return p;
+}
+__host__ inline size_t order_smem_bytes(int num_seqs) {
+    return num_seqs <= kOrderMax ? 2 * sizeof(int32_t) * (size_t)order_pow2(num_seqs) : 0;
+}
+__global__ void __launch_bounds__(1024) order_kernel(int32_t* __restrict__ off, int num_seqs) {
+    kda_grid_launch_next();   // the preparation's blocks may start loading their inputs
+    kda_grid_wait();          // the chunk offsets
+    const int tid = threadIdx.x;
+    int32_t* order = off + num_seqs + 1;
+    if (num_seqs > kOrderMax) {
+        for (int n = tid; n < num_seqs; n += 1024) order[n] = n;
+        return;
+    }
+    extern __shared__ int32_t order_smem[];
+    const int P = order_pow2(num_seqs);
+    int32_t* s_cnt = order_smem;
+    int32_t* s_idx = order_smem + P;
+    for (int i = tid; i < P; i += 1024) {
+        s_cnt[i] = i < num_seqs ? off[i + 1] - off[i] : -1;   // padding sorts last
+        s_idx[i] = i;
+    }
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < P; i += 1024) {
+                const int m = i ^ j;
+                if (m > i) {
+                    const int ci = s_cnt[i], cm = s_cnt[m], xi = s_idx[i], xm = s_idx[m];
+                    const bool m_first = cm > ci || (cm == ci && xm < xi);   // m precedes i
+                    if (((i & k) == 0) == m_first) {   // ascending runs want i first, descending m
+                        s_cnt[i] = cm; s_cnt[m] = ci;
+                        s_idx[i] = xm; s_idx[m] = xi;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int n = tid; n < num_seqs; n += 1024) order[n] = s_idx[n];
 }
 
 // Emission slots: etab[c] = e for the chunk c that ends at emission boundary e (the state
@@ -1112,7 +1163,9 @@ constexpr RecWindow kWholeProblem = {0, INT32_MAX, 1, nullptr, nullptr};
 // DIN: channels per head of the caller's outputs and states (128, or 64 with the chunk
 // tensors of a 128-channel problem whose channels from 64 on are zero: only the value slices
 // of the first 64 columns run, and only the state's first 64 rows are read or written).
-template <int NV, int DIN>
+// kOrdered: the CTAs take the sequences in the order the chunk-table kernel wrote after the
+// chunk offsets (several sequences); otherwise in index order.
+template <int NV, int DIN, bool kOrdered>
 __global__ void __launch_bounds__(kRecThreads, 1)
 rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __restrict__ tab,
            const uint8_t* __restrict__ records, const float* initial_state, float* final_state,
@@ -1121,7 +1174,6 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
            const float* __restrict__ seg_states, RecWindow win) {
     using S = RecCfg<NV>;
     constexpr int NSL = DIN / NV;   // value slices of the caller's columns
-    (void)num_seqs;
     kda_grid_wait();   // the chunk table and the records
     const int sl = blockIdx.x % NSL;
     const int h = (blockIdx.x / NSL) % H;
@@ -1144,7 +1196,7 @@ rec_kernel(int num_seqs, int H, const int32_t* __restrict__ off, const int2* __r
         if (!first) s_ld = D;
     } else {
         // this sequence's chunks inside the window [c_lo, c_hi)
-        n = unit;
+        n = kOrdered ? off[num_seqs + 1 + unit] : unit;
         const int a = off[n], b = off[n + 1];
         c_begin = max(a, win.c_lo);
         nchunks = min(b, win.c_hi) - c_begin;
@@ -1853,12 +1905,22 @@ struct RecLaunch {
     uint32_t smem;
     int nsl;   // CTAs per chain
 };
-inline RecLaunch pick_rec(int64_t chains, int din) {
+// ordered: sequences taken longest first (several sequences, no scan segments).
+inline RecLaunch pick_rec(int64_t chains, int din, bool ordered) {
     const int sms = device_sm_count();
     const bool narrow = chains * (din / 32) <= (int64_t)(sms > 0 ? sms : 148);
-    if (din == 64)
-        return narrow ? RecLaunch{rec_kernel<32, 64>, RecCfg<32>::BYTES, 2} : RecLaunch{rec_kernel<64, 64>, RecCfg<64>::BYTES, 1};
-    return narrow ? RecLaunch{rec_kernel<32, 128>, RecCfg<32>::BYTES, 4} : RecLaunch{rec_kernel<64, 128>, RecCfg<64>::BYTES, 2};
+    if (din == 64) {
+        if (ordered)
+            return narrow ? RecLaunch{rec_kernel<32, 64, true>, RecCfg<32>::BYTES, 2}
+                          : RecLaunch{rec_kernel<64, 64, true>, RecCfg<64>::BYTES, 1};
+        return narrow ? RecLaunch{rec_kernel<32, 64, false>, RecCfg<32>::BYTES, 2}
+                      : RecLaunch{rec_kernel<64, 64, false>, RecCfg<64>::BYTES, 1};
+    }
+    if (ordered)
+        return narrow ? RecLaunch{rec_kernel<32, 128, true>, RecCfg<32>::BYTES, 4}
+                      : RecLaunch{rec_kernel<64, 128, true>, RecCfg<64>::BYTES, 2};
+    return narrow ? RecLaunch{rec_kernel<32, 128, false>, RecCfg<32>::BYTES, 4}
+                  : RecLaunch{rec_kernel<64, 128, false>, RecCfg<64>::BYTES, 2};
 }
 
 inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, const float* g,
@@ -1869,6 +1931,11 @@ inline cudaError_t launch_prepare(const void* q, const void* k, const void* v, c
     const Workspace w = split_workspace(workspace, total, num_seqs, H);
     chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off, w.tab,
                                                num_emit > 0 ? w.etab : nullptr, w.strong_count, 1);
+    if (num_seqs > 1) {
+        const cudaError_t e0 = launch_after(order_kernel, dim3(1), dim3(1024), (uint32_t)order_smem_bytes(num_seqs),
+                                            stream, w.off, num_seqs);
+        if (e0 != cudaSuccess) return e0;
+    }
     if (num_emit > 0)
         emit_index_kernel<<<(num_emit + 255) / 256, 256, 0, stream>>>(cu, num_seqs, w.off, emit_pos,
                                                                        num_emit, w.etab);
@@ -1889,7 +1956,7 @@ inline cudaError_t launch_scan(const float* s0, float* sf, void* out, int num_se
     const int32_t* et = emit_states ? w.etab : nullptr;
     const bool scan = w.seg > 0 && !(in_flags & kInSerialChains);
     const int64_t units = scan ? w.max_segs : num_seqs;   // chains: sequences, or scan segments
-    const RecLaunch rl = pick_rec(units * H, din);
+    const RecLaunch rl = pick_rec(units * H, din, !scan && num_seqs > 1);
     auto rec = rl.kernel;
     const uint32_t rec_smem = rl.smem;
     const int nsl = rl.nsl;
@@ -1946,6 +2013,11 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
     const int64_t nw = (mc + window - 1) / window;
     chunk_index_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total, w.off, w.tab,
                                                num_emit > 0 ? w.etab : nullptr, counts, (int)nw);
+    if (num_seqs > 1) {
+        const cudaError_t e0 = launch_after(order_kernel, dim3(1), dim3(1024), (uint32_t)order_smem_bytes(num_seqs),
+                                            stream, w.off, num_seqs);
+        if (e0 != cudaSuccess) return e0;
+    }
     if (num_emit > 0)
         emit_index_kernel<<<(num_emit + 255) / 256, 256, 0, stream>>>(cu, num_seqs, w.off, emit_pos,
                                                                        num_emit, w.etab);
@@ -1954,7 +2026,7 @@ inline cudaError_t launch_prefill(const void* q, const void* k, const void* v, c
     PrepInputs p;
     if (total > 0 && (e = make_prep_inputs(&p, q, k, v, g, beta, num_seqs, total, H, w, in_flags, din)) != cudaSuccess)
         return e;
-    const RecLaunch rl = pick_rec((int64_t)num_seqs * H, din);
+    const RecLaunch rl = pick_rec((int64_t)num_seqs * H, din, num_seqs > 1);
     auto rec = rl.kernel;
     const uint32_t rec_smem = rl.smem;
     const int nsl = rl.nsl;

@@ -95,8 +95,9 @@ int32_t kda_prefill_launches(int64_t total_tokens, int32_t num_seqs, int32_t H, 
         return -1;
     if (num_seqs == 0) return 0;
     if (!tensor_core_path(dt, dk)) return 1;
-    // chunk table, [emission slots], preparation, strongly decayed chunks, recurrence
-    int32_t n = 1 + (num_emit > 0 ? 1 : 0) + (total_tokens > 0 ? 2 : 0) + 1;
+    // chunk table, [recurrence order of several sequences], [emission slots], preparation,
+    // strongly decayed chunks, recurrence
+    int32_t n = 1 + (num_seqs > 1 ? 1 : 0) + (num_emit > 0 ? 1 : 0) + (total_tokens > 0 ? 2 : 0) + 1;
     if (!(in_flags & KDA_IN_SERIAL_CHAINS) && kda::tc::scan_segment_chunks(total_tokens, num_seqs, H) > 0)
         n += 3;   // segment table, segment transitions, starting states
     return n;

@@ -194,7 +194,7 @@ def test_prefill_launch_count(lib):
     assert n(1 << 20, 1, 32) == 4                 # 32 chains x 4 slices already fill the SMs
     assert n(1 << 20, 1, 8) == 7                  # 8 long chains: chunk-parallel scan (+3)
     assert n(1 << 20, 1, 8, flags=kda.KDA_IN_SERIAL_CHAINS) == 4
-    assert n(8192, 16, 32) == 4                   # 512 chains fill the SMs: no scan
+    assert n(8192, 16, 32) == 5                   # 512 chains fill the SMs: no scan; +1: the sequences' order
     assert n(300, 1, 2) == 4                      # 5 chunks per chain: segments too short
     assert n(8192, 1, 32, emit=2) == 5
     assert n(0, 1, 32) == 2                       # chunk table and recurrence only
