@@ -15,6 +15,8 @@
 //
 //   chunk_index_kernel  cu_seqlens -> first chunk of every sequence and the chunk table
 //                       (first token, rows) (device side, no host sync); validates cu_seqlens.
+//   order_kernel        (several sequences) the order in which the recurrence takes them:
+//                       most chunks first.
 //   prep_kernel         one CTA of 8 warps per (chunk, head), fully parallel, 2 CTAs per SM:
 //                         TMA: g, then q and k, then v tiles (128-byte swizzled) into
 //                              shared memory, each group on its own barrier
